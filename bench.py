@@ -1,0 +1,352 @@
+"""Benchmark: chunk-causal attention at the 720p latent shape on B200.
+
+One step = one chunk of the stream at the 720p shape: two denoising-step
+attention calls (1620 queries x 24 heads x 128 over sink + 3-chunk window +
+current chunk = 8100 keys) and the clean-KV append of the chunk, through the
+C ABI of libcca.so.  The ring is prefilled with chunks 0..3, so every step sees
+the steady-state visible set (5 chunks).  Metric: algorithmic attention TFLOP/s
+(4 * Lq * Lk * H * D per call) over the whole step time, plus ms per chunk.
+
+Inputs are synthetic (seeded, see ``synth``) and resident in HBM when timing
+starts.  Steps cycle through 3 independent replicas of the state (~420 MB in
+total, more than the 126 MB L2), so no step finds the previous step's data in L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica of
+the workload: the method needs no exchange between GPUs ("replicas only"), so
+the only collectives are the barriers and the max-over-ranks of the timing.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "chunk-attn TFLOP/s & ms/chunk at 720p latent shape; % of BF16/FP8 tensor peak"
+WORKLOAD = ("720p-shaped chunk: 1620 tokens (30x54 latent grid), 24 heads x 128, sink + 3-chunk window "
+            "+ current chunk (8100 keys), 2 denoising-step attention calls + clean-KV append per chunk")
+L, H, D, W = 1620, 24, 128, 3
+LK = (1 + W + 1) * L
+FLOP_PER_CALL = 4.0 * L * LK * H * D
+CALLS_PER_STEP = 2
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self, n_skip: int = 0):
+        if not self.proc:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        rows = rows[n_skip:] or rows
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+def oracle_sample(n_q_rows: int, n_heads: int, seed: int = 1):
+    """Time the fp64 oracle on a bounded sample of the 720p attention call:
+    the first ``n_q_rows`` queries of ``n_heads`` heads over all 8100 keys."""
+    import synth
+    from oracle import chunk_attention as oca
+    g = synth.rng(seed)
+    shape_q = (n_q_rows, n_heads, D)
+    q = g.standard_normal(shape_q).astype(np.float32)
+    ks = [g.standard_normal((L, n_heads, D)).astype(np.float32) for _ in range(W + 2)]
+    vs = [g.standard_normal((L, n_heads, D)).astype(np.float32) for _ in range(W + 2)]
+    t = W + 1
+    t0 = time.perf_counter()
+    oca.chunk_attention(q, ks, vs, t, W)
+    dt = time.perf_counter() - t0
+    return 4.0 * n_q_rows * LK * n_heads * D, dt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline():
+    flop, dt = oracle_sample(L, 4)  # 4 heads of one full call (~1/6 of the call)
+    return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, 4 of 24 heads of one 720p attention call (1620 x 8100 keys), "
+                      f"{dt:.2f} s"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the oracle as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    rows, heads = 128, 1  # one 128-query tile of one head per step
+    for _ in range(args.warmup):
+        oracle_sample(rows, heads)
+    tot_flop, tot_t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, dt = oracle_sample(rows, heads)
+        tot_flop += f
+        tot_t += dt
+    value = tot_flop / tot_t / 1e12
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": L, "kv_len": LK,
+                       "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": "each step: 128 queries x 1 head of the 720p call over 8100 keys, fp64"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import synth
+    import chunk_causal_attention_b200 as cca
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.barrier()
+    c1 = synth.chunk_720p()
+    bf = lambda x: synth.as_torch_bf16(x, dev)
+
+    class Replica:
+        def __init__(self):
+            self.ring = cca.KVRing(H, D, L, W, device=dev)
+            for t in range(c1.t):
+                self.ring.append(bf(c1.ring_k[t]), bf(c1.ring_v[t]))
+            self.q = [bf(x) for x in c1.q]
+            self.k = [bf(x) for x in c1.k_cur]
+            self.v = [bf(x) for x in c1.v_cur]
+            self.out = [torch.empty((L, H, D), dtype=torch.bfloat16, device=dev) for _ in c1.q]
+            ws = cca.cca_chunk_attn_workspace_size(self.ring, L)
+            self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+
+    reps = [Replica() for _ in range(3)]
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step(rep, ev=None):
+        for s in range(CALLS_PER_STEP):
+            if ev is not None:
+                ev[2 * s].record(stream)
+            cca.cca_chunk_attn(rep.ring, rep.q[s], rep.k[s], rep.v[s], out=rep.out[s], workspace=rep.ws)
+            if ev is not None:
+                ev[2 * s + 1].record(stream)
+        rep.ring.append(rep.k[-1], rep.v[-1])  # clean K/V of the chunk (values are immaterial to timing)
+
+    for i in range(args.warmup):
+        step(reps[i % 3])
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    attn_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * CALLS_PER_STEP)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cca.cca_take_launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(reps[i % 3], attn_ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = cca.cca_take_launch_count()
+    clocks = sampler.stop() if sampler else None
+    total_ms = t_start.elapsed_time(t_end)
+    attn_ms = [attn_ev[i][2 * s].elapsed_time(attn_ev[i][2 * s + 1]) for i in range(args.steps)
+               for s in range(CALLS_PER_STEP)]
+    for r in reps:
+        torch.cuda.synchronize()
+        if int(r.ring.status.item()) != 0:
+            raise RuntimeError(f"device status {int(r.ring.status.item())}")
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # ---- end to end through the public API with host buffers (pinned), rank-local
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = lambda x: synth.as_torch_bf16(x).pin_memory()
+        hq = [pin(x) for x in c1.q]
+        hk = [pin(x) for x in c1.k_cur]
+        hv = [pin(x) for x in c1.v_cur]
+        ho = [torch.empty((L, H, D), dtype=torch.bfloat16).pin_memory() for _ in c1.q]
+        rep = reps[0]
+        dq = [torch.empty_like(x, device=dev) for x in hq]
+        dk = [torch.empty_like(x, device=dev) for x in hk]
+        dv = [torch.empty_like(x, device=dev) for x in hv]
+
+        def e2e_step():
+            for s in range(CALLS_PER_STEP):
+                dq[s].copy_(hq[s], non_blocking=True)
+                dk[s].copy_(hk[s], non_blocking=True)
+                dv[s].copy_(hv[s], non_blocking=True)
+                cca.cca_chunk_attn(rep.ring, dq[s], dk[s], dv[s], out=rep.out[s], workspace=rep.ws)
+                ho[s].copy_(rep.out[s], non_blocking=True)
+            rep.ring.append(dk[-1], dv[-1])
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = CALLS_PER_STEP * 3 * L * H * D * 2
+        d2h = CALLS_PER_STEP * L * H * D * 2
+        e2e = {"value": world * CALLS_PER_STEP * FLOP_PER_CALL / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if rank != 0:
+        return
+    peak_tf, _, peak_kind = peaks()
+    ms_step = total_ms / args.steps
+    value = world * CALLS_PER_STEP * FLOP_PER_CALL / (ms_step * 1e-3) / 1e12
+    attn_mean_ms = float(np.mean(attn_ms))
+    achieved = FLOP_PER_CALL / (attn_mean_ms * 1e-3) / 1e12
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "attn_bf16_720p.traffic.json")
+    if os.path.exists(prof):
+        try:
+            traffic = json.load(open(prof)).get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": L, "kv_len": LK, "heads": H,
+                   "head_dim": D, "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2: steps cycle 3 replicas (~420 MB)"},
+        "ms_per_chunk": ms_step,
+        "attn_us_per_call": attn_mean_ms * 1e3,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved / peak_tf, "traffic": traffic,
+                     "kernel": "attn_bf16_kernel (+ split-KV combine), per cca_chunk_attn call",
+                     "peak_kind": f"bf16 dense, {peak_kind} burst"},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

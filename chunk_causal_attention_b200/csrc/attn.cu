@@ -1,0 +1,705 @@
+// Chunk-wise causal attention over the bounded KV cache, BF16, sm_100a.
+//
+// What it computes ["JoyAI-Video-Edit 소개", section 청크 단위 자기회귀 적응;
+// "論文解説: JoyAI-Video-Edit", step 1 (§4.1)]: the queries of the current chunk
+// t attend, with one dense softmax, to every key of the visible chunks -- the
+// sink (chunk 0), the W most recent earlier chunks (from the ring) and chunk t
+// itself (bidirectional inside the chunk).  Because visibility is per whole
+// chunk, no element mask is needed: the kernel walks a list of KV chunks and
+// only masks the zero-filled tail of a chunk whose length is not a multiple of
+// the 128-row tile.
+//
+// Kernel design (sm_100a; the pages give no kernel):
+//  * one work item = two 128-row Q tiles (256 queries) of one head x a range
+//    of 128-row KV tiles; both Q tiles share every K/V tile loaded into shared
+//    memory, halving L2->SM traffic per FLOP;
+//  * warp 0 = TMA producer (Q once per item, K/V per tile, 2-stage ring);
+//    warp 1 = TMEM allocator and the single thread issuing tcgen05.mma;
+//    warps 4-7 / 8-11 = softmax warpgroups, one per Q tile, one row per thread;
+//  * TMEM (512 columns): S0 | S1 | O0 | O1.  S = Q K^T lands in TMEM; the
+//    softmax warps read it, write P (bf16) back over the first half of S, and
+//    P is the A operand of O += P V straight from TMEM;
+//  * online softmax in base 2 with the scale folded in; the running maximum is
+//    only moved (and O rescaled in TMEM) when a row's maximum grows by more
+//    than 2^8, so P never exceeds 256 and rescales are rare;
+//  * split-KV: items can cover part of the KV list; partial (O, m, l) go to the
+//    caller's workspace and a small combine kernel merges them;
+//  * every mbarrier wait is bounded; on timeout the CTA sets an abort flag,
+//    drains its in-flight TMA loads and MMAs, frees TMEM and reports
+//    CCA_DEV_TIMEOUT through the ring's status word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "ring.cuh"
+#include "sm100.cuh"
+
+namespace cca {
+
+constexpr int kBM = 128;       // query rows per Q tile (TMEM lanes)
+constexpr int kBN = 128;       // key rows per KV tile
+constexpr int kNQ = 2;         // Q tiles per work item
+constexpr int kNS = 2;         // K and V pipeline stages
+constexpr int kThreads = 384;  // 12 warps
+constexpr int kMaxVis = kMaxWindow + 2;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
+
+struct AttnArgs {
+  const __nv_bfloat16 *q;  // query rows (gather path)
+  const int32_t *q_idx;    // NULL: dense rows
+  const int32_t *n_q_dev;  // NULL: n_q = n_q_max
+  __nv_bfloat16 *out;      // [n_q_max][H][D]
+  float *ws_o;             // [n_splits][n_q_max][H][D] partial O (unnormalised)
+  float *ws_ml;            // [n_splits][n_q_max][H][2] (running max in log2 units, row sum)
+  int32_t *dev_status;
+  int n_q_max, L, H;
+  int n_pairs, n_splits;
+  int tiles_per_chunk, n_kv_tiles, n_items;
+  float scale_log2;
+  long long wait_budget;
+  int8_t slot[kMaxVis];  // ring slot of each visible chunk, -1 = current chunk
+};
+
+template <int D>
+struct AttnSmem {
+  static constexpr uint32_t kBox = 128 * 128;        // 128 rows x 128 bytes (one SW128 box)
+  static constexpr uint32_t kNBox = D / 64;          // boxes per 128-row tile
+  static constexpr uint32_t kTile = kBox * kNBox;    // bytes of one Q/K/V tile
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kK = kQ + kNQ * kTile;
+  static constexpr uint32_t kV = kK + kNS * kTile;
+  static constexpr uint32_t kBar = kV + kNS * kTile;
+  static constexpr uint32_t kNumBars = 4 + 4 * kNS + 8 + 1;
+  static constexpr uint32_t kBytes = kBar + kNumBars * 8 + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+};
+
+__device__ __forceinline__ void kv_tile_coords(const AttnArgs &a, int j, int &slot, int &row0) {
+  const int c = j / a.tiles_per_chunk;
+  row0 = (j - c * a.tiles_per_chunk) * kBN;
+  slot = a.slot[c];
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kr,
+                     const __grid_constant__ CUtensorMap tm_vr, const __grid_constant__ CUtensorMap tm_kc,
+                     const __grid_constant__ CUtensorMap tm_vc, const AttnArgs a) {
+  using namespace sm100;
+  using S = AttnSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *gbase = smem_raw + (base - raw);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + S::kBar);
+  uint64_t *q_full = bars;           // [kNQ]  producer -> MMA
+  uint64_t *q_empty = bars + 2;      // [kNQ]  MMA -> producer
+  uint64_t *k_full = bars + 4;       // [kNS]
+  uint64_t *k_empty = k_full + kNS;  // [kNS]
+  uint64_t *v_full = k_empty + kNS;  // [kNS]
+  uint64_t *v_empty = v_full + kNS;  // [kNS]
+  uint64_t *s_full = v_empty + kNS;  // [2] MMA -> softmax: S ready
+  uint64_t *p_full = s_full + 2;     // [2] softmax -> MMA: P ready (and O rescaled)
+  uint64_t *o_full = p_full + 2;     // [2] MMA -> softmax: O final for the item
+  uint64_t *o_empty = o_full + 2;    // [2] softmax -> MMA: O read out
+  uint64_t *drain = o_empty + 2;     // [1] teardown: all MMAs complete
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_q = a.n_q_dev ? min(max(*a.n_q_dev, 0), a.n_q_max) : a.n_q_max;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kBM);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], kBM);
+    }
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    if (!a.q_idx) prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_kr);
+    prefetch_tmap(&tm_vr);
+    prefetch_tmap(&tm_kc);
+    prefetch_tmap(&tm_vc);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const long long budget = a.wait_budget;
+
+  // ================================================================ producer
+  if (warp == 0) {
+    uint32_t g = 0;   // KV tiles handled by this CTA
+    uint32_t gk = 0;  // K tile loads armed
+    uint32_t gv = 0;  // V tile loads armed
+    int it = 0;       // items handled by this CTA
+    int q_armed = 0;  // Q phases armed (per tile, identical for both)
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      const int split = item % a.n_splits;
+      const int rest = item / a.n_splits;
+      const int pair = rest % a.n_pairs;
+      const int head = rest / a.n_pairs;
+      if (pair * (kNQ * kBM) >= n_q) continue;
+      const int j0 = static_cast<int>(static_cast<int64_t>(split) * a.n_kv_tiles / a.n_splits);
+      const int j1 = static_cast<int>(static_cast<int64_t>(split + 1) * a.n_kv_tiles / a.n_splits);
+      for (int i = 0; i < kNQ && ok; ++i) {
+        if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[i], (it - 1) & 1, abort_flag, budget));
+        if (!ok) break;
+        const uint32_t dstq = base + S::kQ + i * S::kTile;
+        const int row0 = pair * (kNQ * kBM) + i * kBM;
+        if (!a.q_idx) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&q_full[i], S::kTile);
+            for (uint32_t b = 0; b < S::kNBox; ++b)
+              tma_load_3d(&tm_q, &q_full[i], dstq + b * S::kBox, b * 64, head, row0);
+          }
+        } else {
+          // Gather: row r of the tile is query q_idx[row0 + r]; written in the
+          // same 128B-swizzled layout the TMA would produce.
+          constexpr int kChunks = D / 8;  // 16-byte chunks per row
+          for (int e = lane; e < kBM * kChunks; e += 32) {
+            const int r = e / kChunks, c = e % kChunks;
+            const int qr = row0 + r;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (qr < n_q) {
+              const int src = a.q_idx[qr];
+              if (src >= 0 && src < a.L) {
+                v = __ldg(reinterpret_cast<const uint4 *>(a.q + (static_cast<int64_t>(src) * a.H + head) * D) + c);
+              } else if (a.dev_status) {
+                *a.dev_status = CCA_DEV_BAD_INDEX;  // out-of-range query index: row read as zeros
+              }
+            }
+            const uint32_t box = c >> 3, cc = c & 7;
+            const uint32_t dst = dstq + box * S::kBox + r * 128 + ((cc ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
+                         "r"(v.w)
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&q_full[i]);
+        }
+      }
+      if (!ok) break;
+      q_armed = it + 1;
+      for (int j = j0; j < j1; ++j, ++g) {
+        const uint32_t stage = g % kNS, ph = (g / kNS) & 1;
+        int slot, row0;
+        kv_tile_coords(a, j, slot, row0);
+        if (g >= kNS) ok = __all_sync(0xffffffffu, mbar_wait(&k_empty[stage], ph ^ 1, abort_flag, budget));
+        if (!ok) break;
+        ++gk;
+        if (lane == 0) {
+          const uint32_t dst = base + S::kK + stage * S::kTile;
+          mbar_arrive_expect_tx(&k_full[stage], S::kTile);
+          for (uint32_t b = 0; b < S::kNBox; ++b) {
+            if (slot < 0)
+              tma_load_3d(&tm_kc, &k_full[stage], dst + b * S::kBox, b * 64, head, row0);
+            else
+              tma_load_4d(&tm_kr, &k_full[stage], dst + b * S::kBox, b * 64, head, row0, slot);
+          }
+        }
+        if (g >= kNS) ok = __all_sync(0xffffffffu, mbar_wait(&v_empty[stage], ph ^ 1, abort_flag, budget));
+        if (!ok) break;
+        ++gv;
+        if (lane == 0) {
+          const uint32_t dst = base + S::kV + stage * S::kTile;
+          mbar_arrive_expect_tx(&v_full[stage], S::kTile);
+          for (uint32_t b = 0; b < S::kNBox; ++b) {
+            if (slot < 0)
+              tma_load_3d(&tm_vc, &v_full[stage], dst + b * S::kBox, b * 64, head, row0);
+            else
+              tma_load_4d(&tm_vr, &v_full[stage], dst + b * S::kBox, b * 64, head, row0, slot);
+          }
+        }
+      }
+      ++it;
+    }
+    // Drain: wait (bounded) for the most recent armed phase of every barrier the
+    // TMA may still complete, so no copy lands in shared memory after exit.
+    if (lane == 0) {
+      for (uint32_t k = 0; k < kNS && k < gk; ++k) {
+        const uint32_t gg = gk - 1 - k;
+        mbar_drain(&k_full[gg % kNS], (gg / kNS) & 1, budget);
+      }
+      for (uint32_t k = 0; k < kNS && k < gv; ++k) {
+        const uint32_t gg = gv - 1 - k;
+        mbar_drain(&v_full[gg % kNS], (gg / kNS) & 1, budget);
+      }
+      if (q_armed > 0)
+        for (int i = 0; i < kNQ; ++i) mbar_drain(&q_full[i], (q_armed - 1) & 1, budget);
+    }
+  }
+  // ================================================================ MMA issuer
+  else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = idesc_make(1, 1, 0, 0, kBM, kBN);  // bf16, Q and K both K-major
+      constexpr uint32_t kIdescPV = idesc_make(1, 1, 0, 1, kBM, D);    // P from TMEM, V MN-major
+      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+      auto issue_qk = [&](int i, uint32_t stage) {
+        const uint32_t qa = base + S::kQ + i * S::kTile, kb = base + S::kK + stage * S::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * S::kBox + (kk & 3) * 32;
+          mma_f16_ss(tS[i], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescQK,
+                     kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int i, uint32_t stage, bool acc) {
+        const uint32_t vb = base + S::kV + stage * S::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_f16_ts(tO[i], tS[i] + kk * 8, sdesc_sw128(vb + kk * 16 * 128, S::kBox, 1024), kIdescPV,
+                     (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      uint32_t g = 0;
+      int it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+        const int split = item % a.n_splits;
+        const int pair = (item / a.n_splits) % a.n_pairs;
+        if (pair * (kNQ * kBM) >= n_q) continue;
+        const int j0 = static_cast<int>(static_cast<int64_t>(split) * a.n_kv_tiles / a.n_splits);
+        const int j1 = static_cast<int>(static_cast<int64_t>(split + 1) * a.n_kv_tiles / a.n_splits);
+        const int n = j1 - j0;
+        ok = mbar_wait(&q_full[0], it & 1, abort_flag, budget) && mbar_wait(&q_full[1], it & 1, abort_flag, budget);
+        if (!ok) break;
+        tc_fence_after();
+        for (int jj = 0; jj < n && ok; ++jj, ++g) {
+          const uint32_t stage = g % kNS, ph = (g / kNS) & 1;
+          if (!(ok = mbar_wait(&k_full[stage], ph, abort_flag, budget))) break;
+          tc_fence_after();
+          issue_qk(0, stage);
+          mma_commit(&s_full[0]);
+          if (jj > 0) {  // O1 += P1 V for the previous tile
+            const uint32_t pst = (g - 1) % kNS;
+            if (jj == 1 && it > 0 && !(ok = mbar_wait(&o_empty[1], (it - 1) & 1, abort_flag, budget))) break;
+            if (!(ok = mbar_wait(&p_full[1], (g - 1) & 1, abort_flag, budget))) break;
+            tc_fence_after();
+            issue_pv(1, pst, jj > 1);
+            mma_commit(&v_empty[pst]);
+          }
+          issue_qk(1, stage);
+          mma_commit(&s_full[1]);
+          mma_commit(&k_empty[stage]);
+          if (jj == n - 1) {
+            mma_commit(&q_empty[0]);
+            mma_commit(&q_empty[1]);
+          }
+          if (!(ok = mbar_wait(&v_full[stage], ph, abort_flag, budget))) break;
+          if (jj == 0 && it > 0 && !(ok = mbar_wait(&o_empty[0], (it - 1) & 1, abort_flag, budget))) break;
+          if (!(ok = mbar_wait(&p_full[0], g & 1, abort_flag, budget))) break;
+          tc_fence_after();
+          issue_pv(0, stage, jj > 0);
+          if (jj == n - 1) mma_commit(&o_full[0]);
+        }
+        if (!ok) break;
+        {  // O1 += P1 V for the last tile
+          const uint32_t pst = (g - 1) % kNS;
+          if (n == 1 && it > 0 && !(ok = mbar_wait(&o_empty[1], (it - 1) & 1, abort_flag, budget))) break;
+          if (!(ok = mbar_wait(&p_full[1], (g - 1) & 1, abort_flag, budget))) break;
+          tc_fence_after();
+          issue_pv(1, pst, n > 1);
+          mma_commit(&v_empty[pst]);
+          mma_commit(&o_full[1]);
+        }
+        ++it;
+      }
+      // Teardown: every MMA issued above must be complete before TMEM is freed.
+      mma_commit(drain);
+      mbar_drain(drain, 0, budget);
+    }
+    __syncwarp();
+  }
+  // ================================================================ softmax
+  else if (warp >= 4) {
+    const int wg = (warp - 4) >> 2;         // Q tile of this warpgroup
+    const int r = ((warp & 3) << 5) + lane;  // row inside the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + wg * 128u;
+    const uint32_t tO = tmem + lane_off + 256u + wg * D;
+    const float sl2 = a.scale_log2;
+    uint32_t g = 0;
+    int it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      const int split = item % a.n_splits;
+      const int rest = item / a.n_splits;
+      const int pair = rest % a.n_pairs;
+      const int head = rest / a.n_pairs;
+      if (pair * (kNQ * kBM) >= n_q) continue;
+      const int j0 = static_cast<int>(static_cast<int64_t>(split) * a.n_kv_tiles / a.n_splits);
+      const int j1 = static_cast<int>(static_cast<int64_t>(split + 1) * a.n_kv_tiles / a.n_splits);
+      float m_ref = -INFINITY, l_sum = 0.f;
+      for (int j = j0; j < j1; ++j, ++g) {
+        int slot, row0;
+        kv_tile_coords(a, j, slot, row0);
+        const int valid = min(kBN, a.L - row0);
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], g & 1, abort_flag, budget));
+        if (!ok) break;
+        tc_fence_after();
+        float x[128];
+        {
+          uint32_t u0[32], u1[32], u2[32], u3[32];
+          tmem_ld32(tS + 0, u0);
+          tmem_ld32(tS + 32, u1);
+          tmem_ld32(tS + 64, u2);
+          tmem_ld32(tS + 96, u3);
+          tmem_ld_wait32(u0);
+          tmem_ld_wait32(u1);
+          tmem_ld_wait32(u2);
+          tmem_ld_wait32(u3);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            x[c] = __uint_as_float(u0[c]);
+            x[32 + c] = __uint_as_float(u1[c]);
+            x[64 + c] = __uint_as_float(u2[c]);
+            x[96 + c] = __uint_as_float(u3[c]);
+          }
+        }
+        if (valid < kBN) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= valid) x[c] = -INFINITY;
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+        const float m_tile = mx * sl2;
+        const bool need = m_tile > m_ref + kRescaleThreshold;
+        const float m_new = need ? m_tile : m_ref;
+        const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
+        const float neg_m = -m_new;
+        uint32_t p[64];
+        float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float e0 = ex2_approx(fmaf(x[2 * c], sl2, neg_m));
+          const float e1 = ex2_approx(fmaf(x[2 * c + 1], sl2, neg_m));
+          sum0 += e0;
+          sum1 += e1;
+          p[c] = pack_bf16x2(e0, e1);
+        }
+        {
+          uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&p[0]);
+          uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&p[32]);
+          tmem_st32(tS + 0, p0);
+          tmem_st32(tS + 32, p1);
+        }
+        l_sum = l_sum * alpha + (sum0 + sum1);
+        m_ref = m_new;
+        // Rescale this row of O when the reference maximum moved (O of the
+        // previous tile is complete: S of this tile was committed after it).
+        if (j > j0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0, o);
+            tmem_ld_wait32(o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(tO + c0, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[wg]);
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_full[wg], it & 1, abort_flag, budget));
+      if (!ok) break;
+      tc_fence_after();
+      const int row = pair * (kNQ * kBM) + wg * kBM + r;
+      const bool row_ok = row < n_q;
+      if (a.n_splits == 1) {
+        const float inv = 1.f / l_sum;
+        __nv_bfloat16 *dst = a.out + (static_cast<int64_t>(row) * a.H + head) * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c0, o);
+          tmem_ld_wait32(o);
+          if (row_ok) {
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+              d4[v] = w;
+            }
+          }
+        }
+      } else {
+        const int64_t prow = (static_cast<int64_t>(split) * a.n_q_max + row) * a.H + head;
+        float *dst = a.ws_o + prow * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c0, o);
+          tmem_ld_wait32(o);
+          if (row_ok) {
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) d4[v] = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          }
+        }
+        if (row_ok) *reinterpret_cast<float2 *>(a.ws_ml + prow * 2) = make_float2(m_ref, l_sum);
+      }
+      tc_fence_before();
+      mbar_arrive(&o_empty[wg]);
+      ++it;
+    }
+  }
+
+  // ================================================================ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag && a.dev_status) atomicExch(a.dev_status, CCA_DEV_TIMEOUT);
+}
+
+// out[row][h] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s ; one warp per (row, head).
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restrict__ ws_o,
+                                                           const float *__restrict__ ws_ml,
+                                                           const int32_t *__restrict__ n_q_dev, int n_q_max, int H,
+                                                           int n_splits, __nv_bfloat16 *__restrict__ out) {
+  const int n_q = n_q_dev ? min(max(*n_q_dev, 0), n_q_max) : n_q_max;
+  const int64_t n_rows = static_cast<int64_t>(n_q) * H;
+  const int lane = threadIdx.x & 31;
+  const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t split_stride = static_cast<int64_t>(n_q_max) * H;
+  for (int64_t rh = w0; rh < n_rows; rh += nw) {
+    float mmax = -INFINITY;
+    for (int s = 0; s < n_splits; ++s) mmax = fmaxf(mmax, ws_ml[(s * split_stride + rh) * 2]);
+    float den = 0.f;
+    float acc[D / 32];
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) acc[k] = 0.f;
+    for (int s = 0; s < n_splits; ++s) {
+      const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + (s * split_stride + rh) * 2);
+      const float w = exp2f(ml.x - mmax);
+      den += w * ml.y;
+      const float *o = ws_o + (s * split_stride + rh) * D;
+#pragma unroll
+      for (int k = 0; k < D / 32; ++k) acc[k] += w * o[k * 32 + lane];
+    }
+    const float inv = 1.f / den;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) out[rh * D + k * 32 + lane] = __float2bfloat16_rn(acc[k] * inv);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [rows][H][D] (rank 3) or [slots][rows][H][D] (rank 4) bf16/e4m3 tensor; box =
+// 128 bytes of D x 1 head x 128 rows (x 1 slot), 128-byte swizzle, zero fill.
+static cca_status make_tmap(CUtensorMap *tm, const void *ptr, CUtensorMapDataType dt, int esize, int D, int H,
+                            int rows, int slots) {
+  auto enc = tmap_encoder();
+  if (!enc) return fail(CCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const int rank = slots > 0 ? 4 : 3;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(slots > 0 ? slots : 1)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * esize, static_cast<cuuint64_t>(H) * D * esize,
+                           static_cast<cuuint64_t>(rows) * H * D * esize};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / esize), 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(tm, dt, rank, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CCA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return CCA_OK;
+}
+
+struct AttnPlan {
+  int n_pairs, n_splits, n_items, grid, tiles_per_chunk, n_kv_tiles, n_vis;
+  int32_t slots[kMaxVis];
+};
+
+static int env_int(const char *name, int dflt) {
+  const char *s = std::getenv(name);
+  return s && *s ? std::atoi(s) : dflt;
+}
+
+static void plan_attention(const cca_kv_ring *ring, int n_q_max, AttnPlan &p) {
+  const cca_kv_ring_desc &d = ring->d;
+  p.n_vis = ring_visible(ring, p.slots, nullptr) + 1;  // cached chunks + the current chunk
+  p.tiles_per_chunk = (d.chunk_len + kBN - 1) / kBN;
+  p.n_kv_tiles = p.n_vis * p.tiles_per_chunk;
+  p.n_pairs = (n_q_max + kNQ * kBM - 1) / (kNQ * kBM);
+  const int sms = num_sms();
+  const int base = p.n_pairs * d.n_heads;
+  // Choose the KV split that minimises (waves x tiles per item); splits cost a
+  // combine pass, so prefer fewer on ties.  CCA_ATTN_SPLITS overrides.
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= 8 && s <= p.n_kv_tiles; ++s) {
+    const int items = base * s;
+    const int waves = (items + sms - 1) / sms;
+    const double cost = waves * std::ceil(static_cast<double>(p.n_kv_tiles) / s) * 1.0 + (s > 1 ? 2.0 : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  const int forced = env_int("CCA_ATTN_SPLITS", 0);
+  if (forced > 0) best = forced < p.n_kv_tiles ? forced : p.n_kv_tiles;
+  p.n_splits = best;
+  p.n_items = base * p.n_splits;
+  p.grid = p.n_items < sms ? p.n_items : sms;
+}
+
+static size_t workspace_bytes_for(const cca_kv_ring *ring, int n_q_max, const AttnPlan &p) {
+  if (p.n_splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(p.n_splits) * n_q_max * ring->d.n_heads;
+  return rows * (static_cast<size_t>(ring->d.head_dim) + 2) * sizeof(float) + 256;
+}
+
+template <int D>
+static cca_status launch_bf16(const cca_kv_ring *ring, const AttnPlan &p, const AttnArgs &args, const void *q,
+                              const void *k_cur, const void *v_cur, cudaStream_t st) {
+  using S = AttnSmem<D>;
+  const cca_kv_ring_desc &d = ring->d;
+  CUtensorMap tq, tkr, tvr, tkc, tvc;
+  std::memset(&tq, 0, sizeof(tq));
+  if (!args.q_idx) CCA_TRY(make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, args.n_q_max, 0));
+  CCA_TRY(make_tmap(&tkr, d.k_slots, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, d.chunk_len, 1 + d.window));
+  CCA_TRY(make_tmap(&tvr, d.v_slots, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, d.chunk_len, 1 + d.window));
+  CCA_TRY(make_tmap(&tkc, k_cur, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, d.chunk_len, 0));
+  CCA_TRY(make_tmap(&tvc, v_cur, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, d.chunk_len, 0));
+  cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(S::kAlloc));
+  if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "cca_chunk_attn: %s", cudaGetErrorString(e));
+  attn_bf16_kernel<D><<<p.grid, kThreads, S::kAlloc, st>>>(tq, tkr, tvr, tkc, tvc, args);
+  CCA_TRY(launched("attn_bf16_kernel"));
+  if (p.n_splits > 1) {
+    const int64_t warps = static_cast<int64_t>(args.n_q_max) * d.n_heads;
+    int64_t blocks = (warps + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+    if (blocks > cap) blocks = cap;
+    attn_combine_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        args.ws_o, args.ws_ml, args.n_q_dev, args.n_q_max, d.n_heads, p.n_splits, args.out);
+    CCA_TRY(launched("attn_combine_kernel"));
+  }
+  return CCA_OK;
+}
+
+}  // namespace cca
+
+using namespace cca;
+
+extern "C" {
+
+cca_status cca_chunk_attn_workspace_size(const cca_kv_ring *ring, int32_t n_q_max, size_t *bytes) {
+  if (!ring || !bytes || n_q_max < 0 || n_q_max > ring->d.chunk_len)
+    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn_workspace_size: bad argument");
+  AttnPlan p;
+  plan_attention(ring, n_q_max, p);
+  *bytes = workspace_bytes_for(ring, n_q_max, p);
+  return CCA_OK;
+}
+
+cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q, const void *k_cur, const void *v_cur,
+                          const float *q_scale, const float *kcur_scale, const float *vcur_scale,
+                          const int32_t *q_idx, const int32_t *n_q_dev, int32_t n_q_max, float softmax_scale,
+                          void *out, void *workspace, size_t workspace_bytes, cca_stream_t stream) {
+  if (!ring) return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: NULL ring");
+  const cca_kv_ring_desc &d = ring->d;
+  if (n_q_max < 0 || n_q_max > d.chunk_len)
+    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: need 0 <= n_q_max <= chunk_len (%d)", d.chunk_len);
+  if (n_q_max == 0) return CCA_OK;
+  if (!q || !k_cur || !v_cur || !out)
+    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: q, k_cur, v_cur and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out))
+    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: q, k_cur, v_cur and out must be 16-byte aligned");
+  if (d.dtype == CCA_E4M3) {
+    if (!q_scale || !kcur_scale || !vcur_scale)
+      return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: E4M3 ring needs q/kcur/vcur scales");
+    return fail(CCA_ERR_UNSUPPORTED, "cca_chunk_attn: E4M3 attention is not built yet");
+  }
+  if (q_scale || kcur_scale || vcur_scale)
+    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: BF16 ring takes no scales");
+  if ((q_idx && (reinterpret_cast<uintptr_t>(q_idx) & 3)) || (n_q_dev && (reinterpret_cast<uintptr_t>(n_q_dev) & 3)))
+    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: q_idx / n_q_dev must be 4-byte aligned");
+  AttnPlan p;
+  plan_attention(ring, n_q_max, p);
+  const size_t need = workspace_bytes_for(ring, n_q_max, p);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: workspace of %zu bytes (16-byte aligned) required", need);
+  AttnArgs args;
+  std::memset(&args, 0, sizeof(args));
+  args.q = static_cast<const __nv_bfloat16 *>(q);
+  args.q_idx = q_idx;
+  args.n_q_dev = n_q_dev;
+  args.out = static_cast<__nv_bfloat16 *>(out);
+  if (need > 0) {
+    args.ws_o = static_cast<float *>(workspace);
+    const size_t rows = static_cast<size_t>(p.n_splits) * n_q_max * d.n_heads;
+    args.ws_ml = args.ws_o + rows * d.head_dim;
+  }
+  args.dev_status = d.dev_status;
+  args.n_q_max = n_q_max;
+  args.L = d.chunk_len;
+  args.H = d.n_heads;
+  args.n_pairs = p.n_pairs;
+  args.n_splits = p.n_splits;
+  args.tiles_per_chunk = p.tiles_per_chunk;
+  args.n_kv_tiles = p.n_kv_tiles;
+  args.n_items = p.n_items;
+  const double scale = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(d.head_dim));
+  args.scale_log2 = static_cast<float>(scale * 1.4426950408889634);  // scale * log2(e)
+  args.wait_budget = static_cast<long long>(env_int("CCA_WAIT_BUDGET_MCYCLES", 4000)) * 1000000LL;
+  for (int c = 0; c < kMaxVis; ++c) args.slot[c] = -1;
+  for (int c = 0; c + 1 < p.n_vis; ++c) args.slot[c] = static_cast<int8_t>(p.slots[c]);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.head_dim == 128) return launch_bf16<128>(ring, p, args, q, k_cur, v_cur, st);
+  return launch_bf16<64>(ring, p, args, q, k_cur, v_cur, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,355 @@
+// Bounded KV cache: ring handle, slot arithmetic, clean-KV append (+ e4m3
+// quantisation), and the stand-alone e4m3 quantiser.
+//
+// The cache keeps the first chunk forever (global sink) plus the W most recent
+// chunks, evicting the oldest non-sink chunk ["JoyAI-Video-Edit 소개", section
+// 30 FPS를 만드는 실시간 배포 파이프라인; "論文解説: JoyAI-Video-Edit", §5 loop].
+// Layout choice of this library: slot 0 = chunk 0, chunk t >= 1 -> slot
+// 1 + (t-1) mod W, so an append overwrites exactly the evicted chunk and no data
+// ever moves.
+#include <cuda_fp8.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "ring.cuh"
+
+namespace cca {
+
+std::string &last_error() {
+  static thread_local std::string s;
+  return s;
+}
+int64_t &launch_counter() {
+  static thread_local int64_t n = 0;
+  return n;
+}
+
+int num_sms() {
+  static std::mutex mu;
+  static std::vector<int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev >= static_cast<int>(cache.size())) cache.resize(dev + 1, 0);
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+int ring_slot_of(const cca_kv_ring *r, int64_t chunk) {
+  if (chunk == 0) return 0;
+  return 1 + static_cast<int>((chunk - 1) % r->d.window);
+}
+
+int ring_visible(const cca_kv_ring *r, int32_t *slots, int64_t *chunk_ids) {
+  // Cached chunks visible from the current chunk t = n_appended, logical order.
+  const int64_t t = r->n_appended;
+  int n = 0;
+  if (t == 0) return 0;
+  if (slots) slots[n] = 0;
+  if (chunk_ids) chunk_ids[n] = 0;
+  ++n;
+  const int64_t lo = t - r->d.window > 1 ? t - r->d.window : 1;
+  for (int64_t c = lo; c < t; ++c) {
+    if (slots) slots[n] = ring_slot_of(r, c);
+    if (chunk_ids) chunk_ids[n] = c;
+    ++n;
+  }
+  return n;
+}
+
+size_t dtype_bytes(cca_dtype t) { return t == CCA_E4M3 ? 1 : (t == CCA_BF16 ? 2 : 4); }
+
+// ------------------------------------------------------------------ kernels
+// bf16 (or fp32 -> bf16 RNE) copy of K and V into one ring slot; 16-byte
+// vectors, grid-stride, blockIdx.y selects K (0) or V (1).
+template <bool kF32>
+__global__ void __launch_bounds__(256) append_bf16_kernel(const void *__restrict__ k_src,
+                                                          const void *__restrict__ v_src,
+                                                          uint4 *__restrict__ k_dst,
+                                                          uint4 *__restrict__ v_dst, int64_t n_vec) {
+  const void *src = blockIdx.y == 0 ? k_src : v_src;
+  uint4 *dst = blockIdx.y == 0 ? k_dst : v_dst;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_vec; i += stride) {
+    if constexpr (!kF32) {
+      dst[i] = __ldcs(reinterpret_cast<const uint4 *>(src) + i);
+    } else {
+      const float4 a = __ldcs(reinterpret_cast<const float4 *>(src) + 2 * i);
+      const float4 b = __ldcs(reinterpret_cast<const float4 *>(src) + 2 * i + 1);
+      __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+      __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+      uint4 o;
+      o.x = *reinterpret_cast<uint32_t *>(&p0);
+      o.y = *reinterpret_cast<uint32_t *>(&p1);
+      o.z = *reinterpret_cast<uint32_t *>(&p2);
+      o.w = *reinterpret_cast<uint32_t *>(&p3);
+      dst[i] = o;
+    }
+  }
+}
+
+// Loads 8 consecutive elements (16 B of bf16, 32 B of fp32) as floats.
+template <bool kF32>
+__device__ __forceinline__ void load8(const void *base, int64_t elem, float (&x)[8]) {
+  if constexpr (kF32) {
+    const float4 a = *reinterpret_cast<const float4 *>(static_cast<const float *>(base) + elem);
+    const float4 b = *reinterpret_cast<const float4 *>(static_cast<const float *>(base) + elem + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  } else {
+    const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(base) + elem);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      x[2 * j] = __uint_as_float(w[j] << 16);
+      x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+  }
+}
+
+// Per-head absmax of up to two tensors x[n_tok][H][D].  grid = (blocks, H,
+// n_tensors); each block strides over tokens of its head and folds its maximum
+// into amax_bits[tensor][h] with atomicMax on the float's bit pattern (valid
+// ordering for non-negative floats).
+template <bool kF32>
+__global__ void __launch_bounds__(256) absmax_kernel(const void *__restrict__ x0, const void *__restrict__ x1,
+                                                     unsigned *amax0, unsigned *amax1, int n_tok, int H,
+                                                     int D) {
+  const void *x = blockIdx.z == 0 ? x0 : x1;
+  unsigned *amax = blockIdx.z == 0 ? amax0 : amax1;
+  const int h = blockIdx.y;
+  const int vec_per_row = D / 8;
+  const int rows_per_iter = blockDim.x / vec_per_row;
+  const int r0 = threadIdx.x / vec_per_row, c = threadIdx.x % vec_per_row;
+  float m = 0.f;
+  if (r0 < rows_per_iter) {
+    for (int l = blockIdx.x * rows_per_iter + r0; l < n_tok; l += gridDim.x * rows_per_iter) {
+      float v[8];
+      load8<kF32>(x, (static_cast<int64_t>(l) * H + h) * D + c * 8, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < static_cast<int>(blockDim.x / 32); ++w) m = fmaxf(m, red[w]);
+    atomicMax(amax + h, __float_as_uint(m));
+  }
+}
+
+__global__ void zero_u32_kernel(unsigned *a, unsigned *b, int n) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    a[i] = 0u;
+    if (b) b[i] = 0u;
+  }
+}
+
+// code = e4m3_rn_satfinite(x / s), s = absmax / 448 (fp32 IEEE divisions).
+template <bool kF32>
+__global__ void __launch_bounds__(256) quant_e4m3_kernel(const void *__restrict__ x0, const void *__restrict__ x1,
+                                                         const unsigned *amax0, const unsigned *amax1,
+                                                         uint8_t *__restrict__ y0, uint8_t *__restrict__ y1,
+                                                         int n_tok, int H, int D) {
+  const void *x = blockIdx.z == 0 ? x0 : x1;
+  const unsigned *amax = blockIdx.z == 0 ? amax0 : amax1;
+  uint8_t *y = blockIdx.z == 0 ? y0 : y1;
+  const int h = blockIdx.y;
+  const float a = __uint_as_float(amax[h]);
+  const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+  const int vec_per_row = D / 8;
+  const int rows_per_iter = blockDim.x / vec_per_row;
+  const int r0 = threadIdx.x / vec_per_row, c = threadIdx.x % vec_per_row;
+  if (r0 >= rows_per_iter) return;
+  for (int l = blockIdx.x * rows_per_iter + r0; l < n_tok; l += gridDim.x * rows_per_iter) {
+    const int64_t e = (static_cast<int64_t>(l) * H + h) * D + c * 8;
+    float v[8];
+    load8<kF32>(x, e, v);
+    uint32_t w[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const __nv_fp8x2_storage_t lo =
+          __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[4 * j], s), __fdiv_rn(v[4 * j + 1], s)),
+                                   __NV_SATFINITE, __NV_E4M3);
+      const __nv_fp8x2_storage_t hi =
+          __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[4 * j + 2], s), __fdiv_rn(v[4 * j + 3], s)),
+                                   __NV_SATFINITE, __NV_E4M3);
+      w[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+    *reinterpret_cast<uint2 *>(y + e) = make_uint2(w[0], w[1]);
+  }
+}
+
+// amax bits -> scale (in place): s = absmax/448, or 1 for an all-zero head.
+__global__ void finalize_scale_kernel(unsigned *a, unsigned *b, int n) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float x = __uint_as_float(a[i]);
+    reinterpret_cast<float *>(a)[i] = x > 0.f ? __fdiv_rn(x, 448.f) : 1.f;
+    if (b) {
+      const float y = __uint_as_float(b[i]);
+      reinterpret_cast<float *>(b)[i] = y > 0.f ? __fdiv_rn(y, 448.f) : 1.f;
+    }
+  }
+}
+
+// Quantise one or two [n_tok][H][D] tensors; scale arrays are [H] each.
+static cca_status quantize_pair(const void *x0, const void *x1, cca_dtype src, int n_tok, int H, int D,
+                                uint8_t *y0, uint8_t *y1, float *s0, float *s1, cudaStream_t st) {
+  const int nt = x1 ? 2 : 1;
+  unsigned *a0 = reinterpret_cast<unsigned *>(s0), *a1 = reinterpret_cast<unsigned *>(s1);
+  zero_u32_kernel<<<1, 256, 0, st>>>(a0, x1 ? a1 : nullptr, H);
+  CCA_TRY(launched("zero_u32_kernel"));
+  if (n_tok > 0) {
+    const int rows_per_block = 256 / (D / 8);
+    int bx = (n_tok + rows_per_block - 1) / rows_per_block;
+    const int target = (num_sms() * 8 + H * nt - 1) / (H * nt);  // ~8 blocks per SM in total
+    if (bx > target) bx = target > 0 ? target : 1;
+    dim3 grid(bx, H, nt);
+    if (src == CCA_F32) {
+      absmax_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D);
+      CCA_TRY(launched("absmax_kernel"));
+      quant_e4m3_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D);
+    } else {
+      absmax_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D);
+      CCA_TRY(launched("absmax_kernel"));
+      quant_e4m3_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D);
+    }
+    CCA_TRY(launched("quant_e4m3_kernel"));
+  }
+  finalize_scale_kernel<<<1, 256, 0, st>>>(a0, x1 ? a1 : nullptr, H);
+  return launched("finalize_scale_kernel");
+}
+
+}  // namespace cca
+
+using namespace cca;
+
+extern "C" {
+
+cca_status cca_kv_ring_create(const cca_kv_ring_desc *desc, cca_kv_ring **out) {
+  if (!desc || !out) return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: NULL argument");
+  const cca_kv_ring_desc &d = *desc;
+  if (d.n_heads < 1 || d.chunk_len < 1 || d.window < 0 || d.window > kMaxWindow)
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: need H >= 1, L >= 1, 0 <= W <= %d", kMaxWindow);
+  if (d.head_dim != 64 && d.head_dim != 128)
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: head_dim must be 64 or 128 (got %d)", d.head_dim);
+  if (d.dtype != CCA_BF16 && d.dtype != CCA_E4M3)
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: dtype must be CCA_BF16 or CCA_E4M3");
+  if (!d.k_slots || !d.v_slots || !aligned16(d.k_slots) || !aligned16(d.v_slots))
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: k_slots/v_slots must be non-NULL and 16-byte aligned");
+  if (d.dtype == CCA_E4M3 && (!d.k_scale || !d.v_scale))
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: E4M3 ring needs k_scale and v_scale");
+  if (d.dtype == CCA_BF16 && (d.k_scale || d.v_scale))
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: BF16 ring takes no scales");
+  cca_kv_ring *r = new (std::nothrow) cca_kv_ring;
+  if (!r) return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: out of host memory");
+  r->d = d;
+  r->n_appended = 0;
+  *out = r;
+  return CCA_OK;
+}
+
+cca_status cca_kv_ring_destroy(cca_kv_ring *ring) {
+  delete ring;
+  return CCA_OK;
+}
+
+cca_status cca_kv_ring_reset(cca_kv_ring *ring) {
+  if (!ring) return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_reset: NULL ring");
+  ring->n_appended = 0;
+  return CCA_OK;
+}
+
+cca_status cca_kv_ring_query(const cca_kv_ring *ring, int64_t *n_appended, int32_t *slots,
+                             int64_t *chunk_ids, int32_t *n_cached) {
+  if (!ring) return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_query: NULL ring");
+  if (n_appended) *n_appended = ring->n_appended;
+  const int n = ring_visible(ring, slots, chunk_ids);
+  if (n_cached) *n_cached = n;
+  return CCA_OK;
+}
+
+cca_status cca_kv_ring_restore(cca_kv_ring *ring, int64_t n_appended) {
+  if (!ring || n_appended < 0) return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_restore: bad argument");
+  ring->n_appended = n_appended;
+  return CCA_OK;
+}
+
+cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new, cca_dtype src_dtype,
+                         cca_stream_t stream) {
+  if (!ring || !k_new || !v_new) return fail(CCA_ERR_INVALID_ARG, "cca_kv_append: NULL argument");
+  if (!aligned16(k_new) || !aligned16(v_new))
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_append: k_new/v_new must be 16-byte aligned");
+  if (src_dtype != CCA_BF16 && src_dtype != CCA_F32)
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_append: src_dtype must be CCA_BF16 or CCA_F32");
+  const cca_kv_ring_desc &d = ring->d;
+  const int64_t t = ring->n_appended;
+  if (t > 0 && d.window == 0) {  // nothing but the sink is ever cached
+    ring->n_appended = t + 1;
+    return CCA_OK;
+  }
+  const int slot = ring_slot_of(ring, t);
+  const int64_t n_elem = static_cast<int64_t>(d.chunk_len) * d.n_heads * d.head_dim;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.dtype == CCA_BF16) {
+    uint4 *kd = reinterpret_cast<uint4 *>(static_cast<char *>(d.k_slots) + slot * n_elem * 2);
+    uint4 *vd = reinterpret_cast<uint4 *>(static_cast<char *>(d.v_slots) + slot * n_elem * 2);
+    const int64_t n_vec = n_elem / 8;
+    int64_t blocks = (n_vec + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
+    if (blocks > cap) blocks = cap;
+    dim3 grid(static_cast<unsigned>(blocks), 2);
+    if (src_dtype == CCA_F32)
+      append_bf16_kernel<true><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, n_vec);
+    else
+      append_bf16_kernel<false><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, n_vec);
+    CCA_TRY(launched("append_bf16_kernel"));
+  } else {
+    uint8_t *kd = static_cast<uint8_t *>(d.k_slots) + slot * n_elem;
+    uint8_t *vd = static_cast<uint8_t *>(d.v_slots) + slot * n_elem;
+    CCA_TRY(quantize_pair(k_new, v_new, src_dtype, d.chunk_len, d.n_heads, d.head_dim, kd, vd,
+                          d.k_scale + slot * d.n_heads, d.v_scale + slot * d.n_heads, st));
+  }
+  ring->n_appended = t + 1;
+  return CCA_OK;
+}
+
+cca_status cca_quant_e4m3(const void *x, cca_dtype src_dtype, int32_t n_tok, int32_t n_heads, int32_t head_dim,
+                          uint8_t *x8, float *scale, cca_stream_t stream) {
+  if (!scale || (n_tok > 0 && (!x || !x8)))
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3: NULL argument");
+  if (n_tok < 0 || n_heads < 1 || (head_dim != 64 && head_dim != 128))
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3: need n_tok >= 0, H >= 1, D in {64,128}");
+  if (src_dtype != CCA_BF16 && src_dtype != CCA_F32)
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3: src_dtype must be CCA_BF16 or CCA_F32");
+  if (n_tok > 0 && (!aligned16(x) || !aligned16(x8)))
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3: x/x8 must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3: scale must be 4-byte aligned");
+  return quantize_pair(x, nullptr, src_dtype, n_tok, n_heads, head_dim, x8, nullptr, scale, nullptr,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+const char *cca_last_error(void) { return last_error().c_str(); }
+
+int32_t cca_version(void) { return (0 << 16) | 1; }
+
+int64_t cca_take_launch_count(void) {
+  const int64_t n = launch_counter();
+  launch_counter() = 0;
+  return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,238 @@
+/*
+ * cca.h -- C ABI of libcca.so: chunk-wise causal attention over a bounded KV
+ * cache, plus the L2 token-mask cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the pages' statement of the problem:
+ *
+ *  - Chunk-wise causal attention with a global sink and a sliding window
+ *    ["JoyAI-Video-Edit 소개", section 청크 단위 자기회귀 적응 (chunk-wise
+ *    autoregressive adaptation); "論文解説: JoyAI-Video-Edit", step 1 (§4.1)]:
+ *    tokens of a chunk attend to each other bidirectionally; chunk t attends
+ *    causally to the first chunk (kept forever as a global sink) and to the W
+ *    most recent earlier chunks, so per-chunk cost and memory are constant.
+ *  - The bounded clean-KV store ["JoyAI-Video-Edit 소개", section 30 FPS를
+ *    만드는 실시간 배포 파이프라인 (deployment pipeline); "論文解説", §5 loop]:
+ *    after a chunk is generated its clean K/V are cached for the next chunk;
+ *    the store keeps the sink plus the most recent chunks, evicting the oldest
+ *    non-sink chunk.
+ *  - FP8 quantisation in deployment (same deployment section); the e4m3 format
+ *    with per-head absmax scales is this library's reading (not on the pages).
+ *  - The AR-oriented mask cache ["LiveEdit 실시간 Diffusion 기반 스트리밍
+ *    비디오 편집", sections 방법론 and 기술 상세]: mask_u = [ || z_edit,u -
+ *    z_src,u ||_2 > tau ] on the previous chunk's latents, tau set to prune
+ *    about 70 % of the tokens; active tokens are recomputed, the others reuse
+ *    the cached self-attention output.
+ *
+ * Conventions shared by every call:
+ *  - Pointers named "device" must point to device memory of the current CUDA
+ *    device; "host" pointers to host memory.  The library never allocates
+ *    device memory: the caller owns every device buffer.  The library owns only
+ *    the small host-side ring handle.
+ *  - Every call is asynchronous on the given stream (NULL = legacy default
+ *    stream) and returns a status synchronously after host-side validation and
+ *    kernel launch.  Errors raised on the device are written to the ring's
+ *    optional device status word (CCA_DEV_*), never by trapping.
+ *  - Every device buffer must be 16-byte aligned unless stated otherwise.
+ *  - Tensors are dense and row-major.  [L][H][D] means token-major: element
+ *    (l, h, d) is at ((l * H) + h) * D + d.
+ *  - Handles are not thread-safe; distinct handles are independent.
+ *  - On any non-CCA_OK status nothing has been launched unless the status is
+ *    CCA_ERR_CUDA (a launch failed part-way); cca_last_error() then describes it.
+ */
+#ifndef CCA_H
+#define CCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-compatible with cudaStream_t / CUstream. */
+typedef struct CUstream_st *cca_stream_t;
+
+typedef enum cca_status {
+  CCA_OK = 0,
+  CCA_ERR_INVALID_ARG = 1,    /* NULL pointer, misalignment, bad size or dtype   */
+  CCA_ERR_UNSUPPORTED = 2,    /* valid request this build does not implement      */
+  CCA_ERR_STATE = 3,          /* ring misuse (e.g. dtype mismatch with the ring)  */
+  CCA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed             */
+  CCA_ERR_DEVICE_TIMEOUT = 5  /* returned by host-side readers of a status word   */
+} cca_status;
+
+/* Values written by kernels into the optional device status word. */
+#define CCA_DEV_OK 0
+#define CCA_DEV_TIMEOUT 1   /* a bounded device-side wait ran out; outputs invalid */
+#define CCA_DEV_BAD_INDEX 2 /* a query index was outside [0, L); that row read as 0 */
+
+typedef enum cca_dtype {
+  CCA_BF16 = 0, /* bfloat16                                  */
+  CCA_E4M3 = 1, /* OCP fp8 e4m3fn, with fp32 per-head scales */
+  CCA_F32 = 2   /* float32                                   */
+} cca_dtype;
+
+/* ------------------------------------------------------------------------ */
+/* Bounded KV cache ("ring")                                                 */
+/* ------------------------------------------------------------------------ */
+
+typedef struct cca_kv_ring cca_kv_ring; /* opaque host-side handle */
+
+typedef struct cca_kv_ring_desc {
+  int32_t n_heads;    /* H >= 1                                                  */
+  int32_t head_dim;   /* D: 64 or 128                                            */
+  int32_t chunk_len;  /* L >= 1 tokens per chunk                                 */
+  int32_t window;     /* W >= 0 most recent non-sink chunks kept                 */
+  cca_dtype dtype;    /* CCA_BF16 or CCA_E4M3                                    */
+  void *k_slots;      /* device, [(1+W)][L][H][D] elements of dtype              */
+  void *v_slots;      /* device, same shape as k_slots                           */
+  float *k_scale;     /* device, [(1+W)][H] fp32 dequantisation scales (E4M3)    */
+  float *v_scale;     /* device, [(1+W)][H] (E4M3); both NULL for BF16           */
+  int32_t *dev_status;/* device, one int32 (CCA_DEV_*), may be NULL              */
+} cca_kv_ring_desc;
+
+/* Create a ring over caller-owned slot buffers (not cleared; nothing is read
+ * before it is written).  Slot 0 holds chunk 0 (the sink, never evicted);
+ * chunk t >= 1 lives in slot 1 + (t-1) mod W, overwriting chunk t-W.
+ * Errors: CCA_ERR_INVALID_ARG (NULL/misaligned pointers, H < 1, D not in
+ * {64,128}, L < 1, W < 0, W > 15, scales missing for E4M3). */
+cca_status cca_kv_ring_create(const cca_kv_ring_desc *desc, cca_kv_ring **out);
+
+/* Free the host handle (the caller's device buffers are untouched). */
+cca_status cca_kv_ring_destroy(cca_kv_ring *ring);
+
+/* Start a new stream: the next append becomes chunk 0 (the new sink). */
+cca_status cca_kv_ring_reset(cca_kv_ring *ring);
+
+/* Report the cache state.  n_appended (host, may be NULL) = chunks appended
+ * so far = index t of the next (current) chunk.  slots / chunk_ids (host
+ * arrays of >= 1+W entries, each may be NULL) receive, in logical order (sink
+ * first, then oldest to newest), the ring slot and chunk index of every cached
+ * chunk; *n_cached (host, may be NULL) their count.  With the caller's copy of
+ * the slot buffers this is a complete snapshot of the stream state. */
+cca_status cca_kv_ring_query(const cca_kv_ring *ring, int64_t *n_appended,
+                             int32_t *slots, int64_t *chunk_ids,
+                             int32_t *n_cached);
+
+/* Restore a snapshot: set the number of appended chunks (the slot buffers must
+ * hold the matching contents, e.g. copied back by the caller). */
+cca_status cca_kv_ring_restore(cca_kv_ring *ring, int64_t n_appended);
+
+/* Append the clean K/V of the chunk just generated (chunk t = n_appended) and
+ * advance t.  k_new / v_new: device [L][H][D] of src_dtype (CCA_BF16 or
+ * CCA_F32).  BF16 ring: bf16 copy (F32 input is rounded to nearest even).
+ * E4M3 ring: per-head absmax quantisation, scale = absmax/448 (1 if all zero),
+ * code = e4m3_rn_satfinite(x / scale) with an IEEE fp32 division; the scales
+ * go to k_scale/v_scale[slot][h].  Eviction is the overwrite of the slot.
+ * Errors: CCA_ERR_INVALID_ARG, CCA_ERR_CUDA. */
+cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new,
+                         cca_dtype src_dtype, cca_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* FP8 quantiser                                                             */
+/* ------------------------------------------------------------------------ */
+
+/* Per-head absmax e4m3 quantisation of x (device [n_tok][H][D] of src_dtype,
+ * CCA_BF16 or CCA_F32) into x8 (device [n_tok][H][D] uint8 codes) and scale
+ * (device [H] fp32), with the same rule as cca_kv_append.  n_tok may be 0
+ * (scales become 1).  Errors: CCA_ERR_INVALID_ARG, CCA_ERR_CUDA. */
+cca_status cca_quant_e4m3(const void *x, cca_dtype src_dtype, int32_t n_tok,
+                          int32_t n_heads, int32_t head_dim, uint8_t *x8,
+                          float *scale, cca_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Chunk attention                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* O = softmax(Q K^T * softmax_scale) V for the queries of the current chunk
+ * t = n_appended, over the keys/values of every visible chunk: the sink
+ * (chunk 0), chunks max(1, t-W) .. t-1 from the ring, and the current chunk
+ * itself from k_cur / v_cur (never from the ring: at a denoising step they are
+ * computed from the noisy input).  No element mask inside that set.
+ *
+ *  q, k_cur, v_cur: device [L][H][D] in the ring's dtype (BF16, or E4M3 codes
+ *      with per-head scales q_scale / kcur_scale / vcur_scale, device [H]
+ *      fp32; the scale pointers must be NULL for BF16).
+ *  q_idx: NULL (queries are rows 0 .. n_q-1 of q) or device int32 row indices
+ *      into q (the compacted active tokens of the mask cache).
+ *  n_q_dev: NULL (n_q = n_q_max) or device int32 holding n_q <= n_q_max; read
+ *      on the device, so no host synchronisation is needed.
+ *  n_q_max: host bound on n_q, 0 <= n_q_max <= L.
+ *  softmax_scale: <= 0 selects 1/sqrt(D).
+ *  out: device [n_q_max][H][D] bf16; row i holds query i (rows >= n_q are
+ *      not written).
+ *  workspace / workspace_bytes: device scratch of at least the size reported
+ *      by cca_chunk_attn_workspace_size (may be NULL if that size is 0); its
+ *      contents need not be initialised and are garbage afterwards.
+ * Errors: CCA_ERR_INVALID_ARG (NULL/misaligned pointers, n_q_max out of range,
+ *      workspace too small), CCA_ERR_STATE (ring empty while the sink is
+ *      needed is impossible: t = 0 attends to itself only), CCA_ERR_CUDA. */
+cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q,
+                          const void *k_cur, const void *v_cur,
+                          const float *q_scale, const float *kcur_scale,
+                          const float *vcur_scale, const int32_t *q_idx,
+                          const int32_t *n_q_dev, int32_t n_q_max,
+                          float softmax_scale, void *out, void *workspace,
+                          size_t workspace_bytes, cca_stream_t stream);
+
+/* Bytes of device workspace cca_chunk_attn needs for this ring and n_q_max
+ * (the split-KV partial results; 0 when no split is used). */
+cca_status cca_chunk_attn_workspace_size(const cca_kv_ring *ring, int32_t n_q_max,
+                                         size_t *bytes);
+
+/* ------------------------------------------------------------------------ */
+/* L2 token mask, compaction, scatter (LiveEdit mask cache)                 */
+/* ------------------------------------------------------------------------ */
+
+/* mask[u] = (d2[u] > tau2) with d2[u] = sum_c (edit[u][c] - src[u][c])^2 in
+ * fp32, i.e. ||edit_u - src_u||_2 > tau.
+ *  src, edit: device [n_tok][n_ch] fp32 latents of the previous chunk.
+ *  prune_quantile < 0: fixed threshold, tau2 = tau * tau (fp32).
+ *  0 < prune_quantile <= 1: dynamic threshold, tau2 = the k-th smallest d2
+ *      with k = ceil(prune_quantile * n_tok) computed in binary64, so exactly
+ *      n_tok - k tokens are active when distances are distinct (ties at the
+ *      threshold stay inactive).  Needs n_tok <= 32768.
+ *  mask: device uint8 [n_tok] (0/1).  dist2_out: device fp32 [n_tok] or NULL.
+ *  tau_out: device fp32, receives sqrt(tau2), or NULL.
+ * n_ch must be a multiple of 4 (<= 256); src/edit 16-byte aligned.
+ * Errors: CCA_ERR_INVALID_ARG, CCA_ERR_CUDA. */
+cca_status cca_token_mask_l2(const float *src, const float *edit, int32_t n_tok,
+                             int32_t n_ch, float tau, float prune_quantile,
+                             uint8_t *mask, float *dist2_out, float *tau_out,
+                             cca_stream_t stream);
+
+/* idx[0 .. n) = ascending positions u with mask[u] != 0; *n_active_dev = n.
+ *  mask: device uint8 [n_tok]; idx: device int32 [n_tok] (entries >= n are not
+ *  written); n_active_dev: device int32.  n_tok <= 2^20.
+ * Errors: CCA_ERR_INVALID_ARG, CCA_ERR_CUDA. */
+cca_status cca_compact(const uint8_t *mask, int32_t n_tok, int32_t *idx,
+                       int32_t *n_active_dev, cca_stream_t stream);
+
+/* o_cache row idx[i] <- o_compact row i for i < *n_active_dev; every other row
+ * of o_cache is left untouched (it keeps the output cached at chunk k-1).
+ *  o_compact: device [n_max][row_bytes]; o_cache: device [*][row_bytes];
+ *  idx, n_active_dev: as produced by cca_compact; n_max: host bound on n.
+ *  row_bytes must be a multiple of 16.  Errors: CCA_ERR_INVALID_ARG, CCA_ERR_CUDA. */
+cca_status cca_scatter(const void *o_compact, const int32_t *idx,
+                       const int32_t *n_active_dev, int32_t n_max,
+                       int32_t row_bytes, void *o_cache, cca_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Diagnostics                                                               */
+/* ------------------------------------------------------------------------ */
+
+/* Message describing the last error of the calling thread ("" if none). */
+const char *cca_last_error(void);
+
+/* Library version, (major << 16) | minor. */
+int32_t cca_version(void);
+
+/* Number of kernels the calling thread has launched through this library
+ * since the last call (the counter is reset by the call). */
+int64_t cca_take_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CCA_H */

@@ -18,3 +18,10 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_library():
+    """libcca.so is built in-tree (a no-op when it is up to date)."""
+    from chunk_causal_attention_b200 import build
+    build.build(quiet=True)

@@ -1,0 +1,352 @@
+"""GPU parity: every kernel of libcca.so against the fp64 oracle.
+
+Bars: bit-exact for the KV ring contents, e4m3 codes/scales, the mask,
+compaction indices and scatter; attention within max-abs 2e-2 and relative L2
+1e-2 (BF16) of the oracle run on the same bf16-rounded inputs.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import chunk_causal_attention_b200 as cca
+from oracle import chunk_attention as oca
+from oracle import fp8 as ofp8
+from oracle import kv_ring as oring
+from oracle import mask_cache as omask
+import synth
+
+pytestmark = pytest.mark.gpu
+
+BF16_MAX_ABS, BF16_REL_L2 = 2e-2, 1e-2
+FP8_MAX_ABS, FP8_REL_L2 = 6e-2, 3e-2
+
+
+def dev():
+    return torch.device("cuda:0")
+
+
+def bf(x):
+    return synth.as_torch_bf16(x, dev())
+
+
+def err(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    d = got - ref
+    return float(np.abs(d).max()), float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-300))
+
+
+def assert_attn_close(got, ref, max_abs=BF16_MAX_ABS, rel_l2=BF16_REL_L2, what=""):
+    ma, rl = err(got, ref)
+    assert ma <= max_abs and rl <= rel_l2, f"{what}: max_abs={ma:.3e} rel_l2={rl:.3e}"
+    return ma, rl
+
+
+def to_np(t):
+    return t.float().cpu().numpy()
+
+
+def check_status(ring):
+    torch.cuda.synchronize()
+    st = int(ring.status.item())
+    assert st == cca.CCA_DEV_OK, f"device status {st}"
+
+
+# ------------------------------------------------------------------ ring
+def test_ring_append_bf16_bit_exact_with_eviction():
+    s = synth.tiny(n_chunks=8)
+    ring = cca.KVRing(s.n_heads, s.head_dim, s.chunk_len, s.window, device=dev())
+    oracle = oring.KVRing(s.window)
+    for t in range(8):
+        ring.append(bf(s.k[t]), bf(s.v[t]))
+        oracle.append(s.k[t], s.v[t])
+        n, slots, ids = ring.query()
+        assert n == t + 1 and ids == oracle.chunks()
+        torch.cuda.synchronize()
+        for sl, c in zip(slots, ids):
+            assert torch.equal(ring.k_slots[sl].cpu(), bf(oracle.get(c)[0]).cpu())
+            assert torch.equal(ring.v_slots[sl].cpu(), bf(oracle.get(c)[1]).cpu())
+    check_status(ring)
+
+
+def test_ring_append_f32_source_rounds_to_nearest_even():
+    g = np.random.default_rng(5)
+    x = g.standard_normal((16, 2, 64)).astype(np.float32)
+    ring = cca.KVRing(2, 64, 16, 1, device=dev())
+    ring.append(torch.from_numpy(x).to(dev()), torch.from_numpy(-x).to(dev()))
+    torch.cuda.synchronize()
+    assert torch.equal(ring.k_slots[0].cpu(), torch.from_numpy(x).to(torch.bfloat16))
+    assert torch.equal(ring.v_slots[0].cpu(), torch.from_numpy(-x).to(torch.bfloat16))
+
+
+# ------------------------------------------------------------------ fp8
+@pytest.mark.parametrize("src_dtype", [torch.bfloat16, torch.float32])
+def test_quant_e4m3_bit_exact(src_dtype):
+    g = np.random.default_rng(6)
+    x = g.standard_t(4.0, size=(1620, 24, 128)).astype(np.float32)
+    x[:, 3] = 0.0  # an all-zero head -> scale 1
+    x[5, 7, 9] = -0.0
+    if src_dtype == torch.bfloat16:
+        x = synth.bf16_round(x)
+    xt = torch.from_numpy(x).to(dev()).to(src_dtype)
+    codes, scale = cca.cca_quant_e4m3(xt)
+    ref_codes, ref_scale = ofp8.quantize_per_head(x)
+    torch.cuda.synchronize()
+    assert np.array_equal(scale.cpu().numpy(), ref_scale)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+
+
+def test_ring_append_e4m3_bit_exact():
+    s = synth.fp8_720p(n_steps=1, n_prefill=5)
+    ring = cca.KVRing(s.n_heads, s.head_dim, s.chunk_len, s.window, dtype="e4m3", device=dev())
+    for t in range(5):
+        ring.append(bf(s.ring_k[t]), bf(s.ring_v[t]))
+    n, slots, ids = ring.query()
+    assert ids == [0, 2, 3, 4]
+    torch.cuda.synchronize()
+    for sl, c in zip(slots, ids):
+        kc, ks = ofp8.quantize_per_head(s.ring_k[c])
+        vc, vs = ofp8.quantize_per_head(s.ring_v[c])
+        assert np.array_equal(ring.k_slots[sl].cpu().numpy(), kc)
+        assert np.array_equal(ring.v_slots[sl].cpu().numpy(), vc)
+        assert np.array_equal(ring.k_scale[sl].cpu().numpy(), ks)
+        assert np.array_equal(ring.v_scale[sl].cpu().numpy(), vs)
+
+
+# ------------------------------------------------------------------ mask / compact / scatter
+def _ambiguity_guard(d2_ref, tau2, rel=1e-5):
+    assert np.all(np.abs(d2_ref - tau2) > rel * max(tau2, 1e-30)), "seeded input too close to tau"
+
+
+def test_mask_fixed_tau_tiny_bit_exact():
+    s = synth.tiny()
+    m_ref, d_ref, tau = omask.token_mask(s.src, s.edit, tau=s.tau)
+    _ambiguity_guard(d_ref ** 2, tau ** 2)
+    src, edit = torch.from_numpy(s.src).to(dev()), torch.from_numpy(s.edit).to(dev())
+    d2 = torch.empty(16, dtype=torch.float32, device=dev())
+    mask = cca.cca_token_mask_l2(src, edit, tau=s.tau, dist2=d2)
+    torch.cuda.synchronize()
+    assert np.array_equal(mask.cpu().numpy(), m_ref)
+    assert 0 < m_ref.sum() < 16
+    assert np.allclose(d2.cpu().numpy(), d_ref ** 2, rtol=1e-6)
+
+
+def test_mask_identical_latents_all_inactive():
+    s = synth.tiny()
+    src = torch.from_numpy(s.src).to(dev())
+    mask = cca.cca_token_mask_l2(src, src.clone(), tau=0.0)
+    idx, n = cca.cca_compact(mask)
+    torch.cuda.synchronize()
+    assert mask.sum().item() == 0 and n.item() == 0
+
+
+def test_mask_dynamic_tau_and_compaction_bit_exact():
+    m = synth.mask_chunk()
+    m_ref, d_ref, tau = omask.token_mask(m.src, m.edit, prune_quantile=m.prune_quantile)
+    d2s = np.sort(d_ref ** 2)
+    k = omask.prune_count(len(d_ref), m.prune_quantile)
+    assert (d2s[k] - d2s[k - 1]) > 1e-5 * d2s[k - 1], "order statistic gap too small for fp32"
+    src, edit = torch.from_numpy(m.src).to(dev()), torch.from_numpy(m.edit).to(dev())
+    tau_out = torch.empty(1, dtype=torch.float32, device=dev())
+    mask = cca.cca_token_mask_l2(src, edit, prune_quantile=m.prune_quantile, tau_out=tau_out)
+    idx, n = cca.cca_compact(mask)
+    torch.cuda.synchronize()
+    assert np.array_equal(mask.cpu().numpy(), m_ref)
+    assert n.item() == 486 == len(d_ref) - k
+    ref_idx, ref_n = omask.compact(m_ref)
+    assert np.array_equal(idx[:n.item()].cpu().numpy(), ref_idx)
+    assert abs(tau_out.item() - tau) <= 1e-5 * tau
+
+
+@pytest.mark.parametrize("n_tok,p", [(1, 0.5), (17, 0.3), (16384, 0.05), (16385, 0.9), (100000, 0.3)])
+def test_compaction_ragged_sizes(n_tok, p):
+    g = np.random.default_rng(n_tok)
+    m = (g.random(n_tok) < p).astype(np.uint8)
+    idx, n = cca.cca_compact(torch.from_numpy(m).to(dev()))
+    torch.cuda.synchronize()
+    assert n.item() == int(m.sum())
+    assert np.array_equal(idx[:n.item()].cpu().numpy(), np.flatnonzero(m).astype(np.int32))
+
+
+def test_scatter_keeps_inactive_rows():
+    g = np.random.default_rng(9)
+    mask = (g.random(1620) < 0.3).astype(np.uint8)
+    cache = synth.bf16_round(g.normal(0, 0.02, size=(1620, 24, 128)).astype(np.float32))
+    ref_idx, ref_n = omask.compact(mask)
+    oc = synth.bf16_round(g.standard_normal((ref_n, 24, 128)).astype(np.float32))
+    mt = torch.from_numpy(mask).to(dev())
+    idx, n = cca.cca_compact(mt)
+    cache_t = bf(cache)
+    cca.cca_scatter(bf(oc), idx, n, cache_t)
+    torch.cuda.synchronize()
+    expect = omask.scatter(oc, ref_idx, ref_n, cache)
+    assert torch.equal(cache_t.cpu(), synth.as_torch_bf16(expect))
+    # empty active set: cache untouched
+    zero = torch.zeros(1, dtype=torch.int32, device=dev())
+    before = cache_t.clone()
+    cca.cca_scatter(bf(oc), idx, zero, cache_t)
+    torch.cuda.synchronize()
+    assert torch.equal(before, cache_t)
+
+
+# ------------------------------------------------------------------ attention
+def run_stream(s, n_chunks, window, ring=None):
+    """Stream chunks 0..n-1: attention of chunk t (current K/V = chunk t) then append."""
+    ring = ring or cca.KVRing(s.n_heads, s.head_dim, s.chunk_len, window, device=dev())
+    outs = []
+    for t in range(n_chunks):
+        o = cca.cca_chunk_attn(ring, bf(s.q[t]), bf(s.k[t]), bf(s.v[t]))
+        outs.append(to_np(o))
+        ring.append(bf(s.k[t]), bf(s.v[t]))
+    check_status(ring)
+    return outs
+
+
+@pytest.mark.parametrize("n_chunks", [4, 8])
+def test_attention_tiny_stream(n_chunks):
+    s = synth.tiny(n_chunks=n_chunks)
+    outs = run_stream(s, n_chunks, s.window)
+    for t in range(n_chunks):
+        ref = oca.chunk_attention(s.q[t], s.k, s.v, t, s.window)
+        assert_attn_close(outs[t], ref, what=f"tiny chunk {t}")
+
+
+@pytest.mark.parametrize("D,L,H,W", [(64, 200, 3, 2), (128, 300, 2, 1), (128, 129, 1, 0), (64, 1, 2, 3)])
+def test_attention_ragged_shapes(D, L, H, W):
+    g = np.random.default_rng(D * 1000 + L)
+    n = W + 3
+    q = [synth.bf16_round(g.standard_normal((L, H, D)).astype(np.float32)) for _ in range(n)]
+    k = [synth.bf16_round(g.standard_normal((L, H, D)).astype(np.float32)) for _ in range(n)]
+    v = [synth.bf16_round(g.standard_normal((L, H, D)).astype(np.float32)) for _ in range(n)]
+    s = synth.TinyStream(H, D, L, W, q, k, v, None, None, 0.0)
+    outs = run_stream(s, n, W)
+    for t in range(n):
+        assert_attn_close(outs[t], oca.chunk_attention(q[t], k, v, t, W), what=f"D{D} L{L} t{t}")
+
+
+@pytest.fixture(scope="module")
+def c1():
+    return synth.chunk_720p()
+
+
+@pytest.fixture(scope="module")
+def c1_ring(c1):
+    ring = cca.KVRing(c1.n_heads, c1.head_dim, c1.chunk_len, c1.window, device=dev())
+    for t in range(c1.t):
+        ring.append(bf(c1.ring_k[t]), bf(c1.ring_v[t]))
+    return ring
+
+
+@pytest.fixture(scope="module")
+def c1_ref(c1):
+    return [oca.chunk_attention(c1.q[s], c1.ring_k, c1.ring_v, c1.t, c1.window, k_cur=c1.k_cur[s],
+                                v_cur=c1.v_cur[s]) for s in range(len(c1.q))]
+
+
+@pytest.mark.parametrize("splits", ["auto", "1", "3"])
+def test_attention_720p_two_steps(c1, c1_ring, c1_ref, splits, monkeypatch):
+    if splits != "auto":
+        monkeypatch.setenv("CCA_ATTN_SPLITS", splits)
+    for s in range(len(c1.q)):
+        o = cca.cca_chunk_attn(c1_ring, bf(c1.q[s]), bf(c1.k_cur[s]), bf(c1.v_cur[s]))
+        assert_attn_close(to_np(o), c1_ref[s], what=f"720p step {s} splits={splits}")
+    check_status(c1_ring)
+
+
+def test_attention_720p_is_deterministic_and_bounded_memory(c1, c1_ring):
+    a = cca.cca_chunk_attn(c1_ring, bf(c1.q[0]), bf(c1.k_cur[0]), bf(c1.v_cur[0]))
+    b = cca.cca_chunk_attn(c1_ring, bf(c1.q[0]), bf(c1.k_cur[0]), bf(c1.v_cur[0]))
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_attention_future_chunks_never_read(c1):
+    """Causality on the GPU: garbage in ring slots of evicted / not-yet-written
+    chunks does not change the output (bitwise)."""
+    ring = cca.KVRing(c1.n_heads, c1.head_dim, c1.chunk_len, 5, device=dev())
+    ring.k_slots.fill_(float("nan"))
+    ring.v_slots.fill_(float("nan"))
+    for t in range(2):
+        ring.append(bf(c1.ring_k[t]), bf(c1.ring_v[t]))
+    o1 = cca.cca_chunk_attn(ring, bf(c1.q[0]), bf(c1.k_cur[0]), bf(c1.v_cur[0]))
+    ring.k_slots[3:].fill_(1e4)
+    o2 = cca.cca_chunk_attn(ring, bf(c1.q[0]), bf(c1.k_cur[0]), bf(c1.v_cur[0]))
+    torch.cuda.synchronize()
+    assert torch.isfinite(o1.float()).all() and torch.equal(o1, o2)
+    ref = oca.chunk_attention(c1.q[0], c1.ring_k, c1.ring_v, 2, 5, k_cur=c1.k_cur[0], v_cur=c1.v_cur[0])
+    assert_attn_close(to_np(o1), ref, what="t=2 W=5")
+
+
+# ------------------------------------------------------------------ mask-cached chunk (workload 4)
+def test_mask_cached_chunk_end_to_end(c1, c1_ring, c1_ref):
+    m = synth.mask_chunk()
+    src, edit = torch.from_numpy(m.src).to(dev()), torch.from_numpy(m.edit).to(dev())
+    mask = cca.cca_token_mask_l2(src, edit, prune_quantile=m.prune_quantile)
+    idx, n = cca.cca_compact(mask)
+    n_max = 1620
+    q = bf(c1.q[0])
+    o_c = cca.cca_chunk_attn(c1_ring, q, bf(c1.k_cur[0]), bf(c1.v_cur[0]), q_idx=idx, n_q_dev=n, n_q_max=n_max)
+    cache = bf(m.o_cache)
+    cca.cca_scatter(o_c, idx, n, cache, n_max=n_max)
+    torch.cuda.synchronize()
+    check_status(c1_ring)
+    m_ref, _, _ = omask.token_mask(m.src, m.edit, prune_quantile=m.prune_quantile)
+    ref_idx, ref_n = omask.compact(m_ref)
+    assert n.item() == ref_n == 486
+    full = c1_ref[0]
+    # active rows: attention of those queries over the full KV; inactive rows: cache unchanged
+    got = to_np(cache)
+    assert_attn_close(got[ref_idx], full[ref_idx], what="active rows")
+    assert np.array_equal(got[m_ref == 0], m.o_cache[m_ref == 0])
+    # row independence: compacted row i equals the dense path's row idx[i]
+    dense = cca.cca_chunk_attn(c1_ring, q, bf(c1.k_cur[0]), bf(c1.v_cur[0]))
+    torch.cuda.synchronize()
+    diff = (o_c[:ref_n].float() - dense[torch.from_numpy(ref_idx).long().to(dev())].float()).abs().max().item()
+    assert diff <= 1e-2
+
+
+def test_mask_cached_full_and_empty_masks(c1, c1_ring, c1_ref):
+    q = bf(c1.q[0])
+    full_idx = torch.arange(1620, dtype=torch.int32, device=dev())
+    n_full = torch.tensor([1620], dtype=torch.int32, device=dev())
+    o = cca.cca_chunk_attn(c1_ring, q, bf(c1.k_cur[0]), bf(c1.v_cur[0]), q_idx=full_idx, n_q_dev=n_full)
+    torch.cuda.synchronize()
+    assert_attn_close(to_np(o), c1_ref[0], what="full mask")
+    n0 = torch.zeros(1, dtype=torch.int32, device=dev())
+    out = torch.full((1620, 24, 128), 7.0, dtype=torch.bfloat16, device=dev())
+    cca.cca_chunk_attn(c1_ring, q, bf(c1.k_cur[0]), bf(c1.v_cur[0]), q_idx=full_idx, n_q_dev=n0, out=out)
+    torch.cuda.synchronize()
+    assert (out == 7.0).all()
+
+
+# ------------------------------------------------------------------ long stream (workload 2)
+def test_long_stream_ring_and_sampled_attention():
+    ls = synth.LongStream(n_chunks=225)
+    ring = cca.KVRing(ls.n_heads, ls.head_dim, ls.chunk_len, ls.window, device=dev())
+    oracle = oring.KVRing(ls.window)
+    sampled = {0, 1, 2, 3, 4, 5, 100, 224}
+    q_fixed = bf(ls.query(0, 0))
+    for t in range(ls.n_chunks):
+        k, v = ls.next_kv()
+        if t in sampled:
+            q = ls.query(t, 0)
+            o = cca.cca_chunk_attn(ring, bf(q), bf(k), bf(v))
+            torch.cuda.synchronize()
+            past_k = {c: oracle.get(c)[0] for c in oracle.chunks()}
+            past_v = {c: oracle.get(c)[1] for c in oracle.chunks()}
+            ref = oca.chunk_attention(q, past_k, past_v, t, ls.window, k_cur=k, v_cur=v)
+            assert_attn_close(to_np(o), ref, what=f"stream chunk {t}")
+        else:
+            cca.cca_chunk_attn(ring, q_fixed, bf(k), bf(v))
+        ring.append(bf(k), bf(v))
+        oracle.append(k, v)
+        n, slots, ids = ring.query()
+        assert ids == oracle.chunks()
+        if t in sampled or t == ls.n_chunks - 1:
+            torch.cuda.synchronize()
+            for sl, c in zip(slots, ids):
+                assert torch.equal(ring.k_slots[sl].cpu(), synth.as_torch_bf16(oracle.get(c)[0]))
+    check_status(ring)
