@@ -136,9 +136,9 @@ def blas_threads():
 
 
 def cpu_baseline():
-    flop, dt = oracle_sample(L, 4)  # 4 heads of one full call (~1/6 of the call)
+    flop, dt = oracle_sample(L, H)  # one full 720p attention call
     return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"fp64 numpy oracle, 4 of 24 heads of one 720p attention call (1620 x 8100 keys), "
+            "sample": f"fp64 numpy oracle, one full 720p attention call (1620 queries x 24 heads x 8100 keys), "
                       f"{dt:.2f} s"}
 
 

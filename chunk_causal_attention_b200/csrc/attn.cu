@@ -49,6 +49,43 @@ constexpr int kNS = 2;         // K and V pipeline stages
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kMaxVis = kMaxWindow + 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
+// Pairs of score columns whose exponential runs on the FMA pipe (polynomial)
+// instead of the MUFU unit: bit k set = pair k of every 8 pairs (3 of 8 here).
+#ifndef CCA_EMU_MASK
+#define CCA_EMU_MASK 0xE0
+#endif
+constexpr unsigned kEmuMask = CCA_EMU_MASK;
+#ifndef CCA_SETMAXNREG
+#define CCA_SETMAXNREG 1
+#endif
+// Registers: the producer / MMA warpgroup needs few, the softmax warpgroups many
+// (4 x 32 x 88 + 8 x 32 x 208 = 384 x 168 = the launch budget of the block).
+constexpr bool kUseSetMaxNReg = CCA_SETMAXNREG;  // log2 units: p <= 2^8 between rescales
+
+// Debug-only event trace of CTA 0 (build with -DCCA_TRACE): 64-bit records
+// [event:8 | tile:16 | clock64:40], read back with cca_debug_trace_read().
+#ifdef CCA_TRACE
+// 4 regions of 16K records (producer, MMA, softmax warpgroup 0, 1); each
+// recording thread keeps its own counter, so a record is one plain store.
+__device__ unsigned long long g_trace[4 << 14];
+#define CCA_TRACE_EV(ev, g)                                                                              \
+  do {                                                                                                   \
+    if (blockIdx.x == 0 && trace_n < (1 << 14))                                                          \
+      g_trace[(trace_role << 14) + trace_n++] = (static_cast<unsigned long long>(ev) << 56) |             \
+                                                (static_cast<unsigned long long>((g) & 0xFFFF) << 40) |   \
+                                                (static_cast<unsigned long long>(clock64()) & 0xFFFFFFFFFFull); \
+  } while (0)
+#define CCA_TRACE_ROLE(r) \
+  int trace_n = 0;        \
+  const int trace_role = (r)
+#else
+#define CCA_TRACE_EV(ev, g) \
+  do {                      \
+  } while (0)
+#define CCA_TRACE_ROLE(r) \
+  do {                    \
+  } while (0)
+#endif
 
 struct AttnArgs {
   const __nv_bfloat16 *q;  // query rows (gather path)
@@ -63,7 +100,8 @@ struct AttnArgs {
   int tiles_per_chunk, n_kv_tiles, n_items;
   float scale_log2;
   long long wait_budget;
-  int8_t slot[kMaxVis];  // ring slot of each visible chunk, -1 = current chunk
+  int n_vis;               // visible chunks, the current one last
+  uint64_t slots_packed;   // 4-bit ring slot of visible chunk c at bits [4c, 4c+4)
 };
 
 template <int D>
@@ -80,10 +118,11 @@ struct AttnSmem {
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
+// KV tile j of the visible list -> (ring slot or -1 for the current chunk, first row).
 __device__ __forceinline__ void kv_tile_coords(const AttnArgs &a, int j, int &slot, int &row0) {
   const int c = j / a.tiles_per_chunk;
   row0 = (j - c * a.tiles_per_chunk) * kBN;
-  slot = a.slot[c];
+  slot = c == a.n_vis - 1 ? -1 : static_cast<int>((a.slots_packed >> (4 * c)) & 15u);
 }
 
 template <int D>
@@ -120,9 +159,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], kBM);
+      mbar_init(&p_full[i], kBM / 32);  // one arrive per softmax warp
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], kBM);
+      mbar_init(&o_empty[i], kBM / 32);
     }
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&k_full[s], 1);
@@ -153,6 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ================================================================ producer
   if (warp == 0) {
+    if (kUseSetMaxNReg) regs_dec<88>();
+    CCA_TRACE_ROLE(0);
     uint32_t g = 0;   // KV tiles handled by this CTA
     uint32_t gk = 0;  // K tile loads armed
     uint32_t gv = 0;  // V tile loads armed
@@ -216,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++gk;
         if (lane == 0) {
           const uint32_t dst = base + S::kK + stage * S::kTile;
+          CCA_TRACE_EV(30, g);
           mbar_arrive_expect_tx(&k_full[stage], S::kTile);
           for (uint32_t b = 0; b < S::kNBox; ++b) {
             if (slot < 0)
@@ -257,95 +299,124 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // ================================================================ MMA issuer
   else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t kIdescQK = idesc_make(1, 1, 0, 0, kBM, kBN);  // bf16, Q and K both K-major
-      constexpr uint32_t kIdescPV = idesc_make(1, 1, 0, 1, kBM, D);    // P from TMEM, V MN-major
-      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
-      auto issue_qk = [&](int i, uint32_t stage) {
-        const uint32_t qa = base + S::kQ + i * S::kTile, kb = base + S::kK + stage * S::kTile;
+    if (kUseSetMaxNReg) regs_dec<88>();
+    CCA_TRACE_ROLE(1);
+    // The whole warp runs this loop converged, so every operand below is
+    // warp-uniform; one elected lane issues each batch of tcgen05 instructions.
+    constexpr uint32_t kIdescQK = idesc_make(1, 1, 0, 0, kBM, kBN);  // bf16, Q and K both K-major
+    constexpr uint32_t kIdescPV = idesc_make(1, 1, 0, 1, kBM, D);    // P from TMEM, V MN-major
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    // Descriptors of every operand tile, built once; a K step inside a tile is
+    // an add to the (address >> 4) field.
+    const uint64_t dQ0 = sdesc_sw128(base + S::kQ, 16, 1024);
+    const uint64_t dK0 = sdesc_sw128(base + S::kK, 16, 1024);
+    const uint64_t dV0 = sdesc_sw128(base + S::kV, S::kBox, 1024);
+    auto issue_qk = [&](int i, uint32_t stage) {
+      const uint64_t qa = dQ0 + ((i * S::kTile) >> 4), kb = dK0 + ((stage * S::kTile) >> 4);
+      const uint32_t d = tm + i * 128u;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * S::kBox + (kk & 3) * 32;
-          mma_f16_ss(tS[i], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescQK,
-                     kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * S::kBox + (kk & 3) * 32) >> 4;
+          mma_f16_ss(d, qa + off, kb + off, kIdescQK, kk > 0 ? 1u : 0u);
         }
-      };
-      auto issue_pv = [&](int i, uint32_t stage, bool acc) {
-        const uint32_t vb = base + S::kV + stage * S::kTile;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_f16_ts(tO[i], tS[i] + kk * 8, sdesc_sw128(vb + kk * 16 * 128, S::kBox, 1024), kIdescPV,
-                     (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      uint32_t g = 0;
-      int it = 0;
-      bool ok = true;
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-        const int split = item % a.n_splits;
-        const int pair = (item / a.n_splits) % a.n_pairs;
-        if (pair * (kNQ * kBM) >= n_q) continue;
-        const int j0 = static_cast<int>(static_cast<int64_t>(split) * a.n_kv_tiles / a.n_splits);
-        const int j1 = static_cast<int>(static_cast<int64_t>(split + 1) * a.n_kv_tiles / a.n_splits);
-        const int n = j1 - j0;
-        ok = mbar_wait(&q_full[0], it & 1, abort_flag, budget) && mbar_wait(&q_full[1], it & 1, abort_flag, budget);
-        if (!ok) break;
-        tc_fence_after();
-        for (int jj = 0; jj < n && ok; ++jj, ++g) {
-          const uint32_t stage = g % kNS, ph = (g / kNS) & 1;
-          if (!(ok = mbar_wait(&k_full[stage], ph, abort_flag, budget))) break;
-          tc_fence_after();
-          issue_qk(0, stage);
-          mma_commit(&s_full[0]);
-          if (jj > 0) {  // O1 += P1 V for the previous tile
-            const uint32_t pst = (g - 1) % kNS;
-            if (jj == 1 && it > 0 && !(ok = mbar_wait(&o_empty[1], (it - 1) & 1, abort_flag, budget))) break;
-            if (!(ok = mbar_wait(&p_full[1], (g - 1) & 1, abort_flag, budget))) break;
-            tc_fence_after();
-            issue_pv(1, pst, jj > 1);
-            mma_commit(&v_empty[pst]);
-          }
-          issue_qk(1, stage);
-          mma_commit(&s_full[1]);
-          mma_commit(&k_empty[stage]);
-          if (jj == n - 1) {
-            mma_commit(&q_empty[0]);
-            mma_commit(&q_empty[1]);
-          }
-          if (!(ok = mbar_wait(&v_full[stage], ph, abort_flag, budget))) break;
-          if (jj == 0 && it > 0 && !(ok = mbar_wait(&o_empty[0], (it - 1) & 1, abort_flag, budget))) break;
-          if (!(ok = mbar_wait(&p_full[0], g & 1, abort_flag, budget))) break;
-          tc_fence_after();
-          issue_pv(0, stage, jj > 0);
-          if (jj == n - 1) mma_commit(&o_full[0]);
-        }
-        if (!ok) break;
-        {  // O1 += P1 V for the last tile
-          const uint32_t pst = (g - 1) % kNS;
-          if (n == 1 && it > 0 && !(ok = mbar_wait(&o_empty[1], (it - 1) & 1, abort_flag, budget))) break;
-          if (!(ok = mbar_wait(&p_full[1], (g - 1) & 1, abort_flag, budget))) break;
-          tc_fence_after();
-          issue_pv(1, pst, n > 1);
-          mma_commit(&v_empty[pst]);
-          mma_commit(&o_full[1]);
-        }
-        ++it;
       }
-      // Teardown: every MMA issued above must be complete before TMEM is freed.
-      mma_commit(drain);
-      mbar_drain(drain, 0, budget);
+      __syncwarp();
+    };
+    auto issue_pv = [&](int i, uint32_t stage, bool acc) {
+      const uint64_t vb = dV0 + ((stage * S::kTile) >> 4);
+      const uint32_t d = tm + 256u + i * D, pa = tm + i * 128u;
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_f16_ts(d, pa + kk * 8, vb + ((kk * 16 * 128) >> 4), kIdescPV, (acc || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+    };
+    auto commit = [&](uint64_t *bar) {
+      if (elect_one()) mma_commit(bar);
+      __syncwarp();
+    };
+    auto wait = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, budget));
+    };
+    uint32_t g = 0;
+    int it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      const int split = item % a.n_splits;
+      const int pair = (item / a.n_splits) % a.n_pairs;
+      if (pair * (kNQ * kBM) >= n_q) continue;
+      const int j0 = static_cast<int>(static_cast<int64_t>(split) * a.n_kv_tiles / a.n_splits);
+      const int j1 = static_cast<int>(static_cast<int64_t>(split + 1) * a.n_kv_tiles / a.n_splits);
+      const int n = j1 - j0;
+      ok = wait(&q_full[0], it & 1) && wait(&q_full[1], it & 1);
+      if (!ok) break;
+      tc_fence_after();
+      for (int jj = 0; jj < n && ok; ++jj, ++g) {
+        const uint32_t stage = g % kNS, ph = (g / kNS) & 1;
+        if (!(ok = wait(&k_full[stage], ph))) break;
+        if (lane == 0) CCA_TRACE_EV(1, g);
+        tc_fence_after();
+        issue_qk(0, stage);
+        commit(&s_full[0]);
+        if (lane == 0) CCA_TRACE_EV(2, g);
+        if (jj > 0) {  // O1 += P1 V for the previous tile
+          const uint32_t pst = (g - 1) % kNS;
+          if (jj == 1 && it > 0 && !(ok = wait(&o_empty[1], (it - 1) & 1))) break;
+          if (!(ok = wait(&p_full[1], (g - 1) & 1))) break;
+          if (lane == 0) CCA_TRACE_EV(3, g - 1);
+          tc_fence_after();
+          issue_pv(1, pst, jj > 1);
+          commit(&v_empty[pst]);
+        }
+        issue_qk(1, stage);
+        commit(&s_full[1]);
+        commit(&k_empty[stage]);
+        if (lane == 0) CCA_TRACE_EV(4, g);
+        if (jj == n - 1) {
+          commit(&q_empty[0]);
+          commit(&q_empty[1]);
+        }
+        if (!(ok = wait(&v_full[stage], ph))) break;
+        if (jj == 0 && it > 0 && !(ok = wait(&o_empty[0], (it - 1) & 1))) break;
+        if (!(ok = wait(&p_full[0], g & 1))) break;
+        if (lane == 0) CCA_TRACE_EV(5, g);
+        tc_fence_after();
+        issue_pv(0, stage, jj > 0);
+        if (lane == 0) CCA_TRACE_EV(6, g);
+        if (jj == n - 1) commit(&o_full[0]);
+      }
+      if (!ok) break;
+      {  // O1 += P1 V for the last tile
+        const uint32_t pst = (g - 1) % kNS;
+        if (n == 1 && it > 0 && !(ok = wait(&o_empty[1], (it - 1) & 1))) break;
+        if (!(ok = wait(&p_full[1], (g - 1) & 1))) break;
+        tc_fence_after();
+        issue_pv(1, pst, n > 1);
+        commit(&v_empty[pst]);
+        commit(&o_full[1]);
+      }
+      ++it;
     }
+    // Teardown: every MMA issued above must be complete before TMEM is freed.
+    commit(drain);
+    if (lane == 0) mbar_drain(drain, 0, budget);
     __syncwarp();
   }
+  else if (warp < 4) {
+    if (kUseSetMaxNReg) regs_dec<88>();
+  }
   // ================================================================ softmax
-  else if (warp >= 4) {
+  else {
+    if (kUseSetMaxNReg) regs_inc<208>();
     const int wg = (warp - 4) >> 2;         // Q tile of this warpgroup
     const int r = ((warp & 3) << 5) + lane;  // row inside the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + wg * 128u;
     const uint32_t tO = tmem + lane_off + 256u + wg * D;
     const float sl2 = a.scale_log2;
+    CCA_TRACE_ROLE(2 + wg);
     uint32_t g = 0;
     int it = 0;
     bool ok = true;
@@ -364,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int valid = min(kBN, a.L - row0);
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], g & 1, abort_flag, budget));
         if (!ok) break;
+        if (lane == 0 && (warp & 3) == 0) CCA_TRACE_EV(10 + 10 * wg, g);
         tc_fence_after();
         float x[128];
         {
@@ -389,31 +461,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (c >= valid) x[c] = -INFINITY;
         }
-        float mx = x[0];
+        // Row maximum: 8 independent 3-input max chains, then a short tree.
+        float mx;
+        {
+          float acc[8];
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+          for (int k = 0; k < 8; ++k) acc[k] = x[k];
+#pragma unroll
+          for (int c = 8; c < 128; c += 16) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = fmax3(acc[k], x[c + k], x[c + 8 + k > 127 ? 127 : c + 8 + k]);
+          }
+          mx = fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
+        }
+        if (lane == 0 && (warp & 3) == 0) CCA_TRACE_EV(11 + 10 * wg, g);
         const float m_tile = mx * sl2;
         const bool need = m_tile > m_ref + kRescaleThreshold;
         const float m_new = need ? m_tile : m_ref;
         const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
-        const float neg_m = -m_new;
-        uint32_t p[64];
-        float sum0 = 0.f, sum1 = 0.f;
+        // p = 2^(x * scale_log2 - m_new), packed f32x2 FMAs, 4 packed partial sums,
+        // bf16 pairs stored to TMEM over the first 64 columns of S, 16 at a time.
+        const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_new, -m_new);
+        uint64_t sums[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float e0 = ex2_approx(fmaf(x[2 * c], sl2, neg_m));
-          const float e1 = ex2_approx(fmaf(x[2 * c + 1], sl2, neg_m));
-          sum0 += e0;
-          sum1 += e1;
-          p[c] = pack_bf16x2(e0, e1);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t p16[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int i = q4 * 32 + 2 * c;
+            float e0, e1;
+            f2_unpack(f2_fma(f2_pack(x[i], x[i + 1]), sl2_2, negm_2), e0, e1);
+            if ((kEmuMask >> (c & 7)) & 1) {
+              exp2_poly_pair(e0, e1);  // FMA pipe
+            } else {
+              e0 = ex2_approx(e0);  // MUFU
+              e1 = ex2_approx(e1);
+            }
+            sums[c & 3] = f2_add(sums[c & 3], f2_pack(e0, e1));
+            p16[c] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tS + q4 * 16, p16);
         }
-        {
-          uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&p[0]);
-          uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&p[32]);
-          tmem_st32(tS + 0, p0);
-          tmem_st32(tS + 32, p1);
-        }
-        l_sum = l_sum * alpha + (sum0 + sum1);
+        float s_lo, s_hi, t_lo, t_hi;
+        f2_unpack(f2_add(f2_add(sums[0], sums[1]), f2_add(sums[2], sums[3])), s_lo, s_hi);
+        (void)t_lo;
+        (void)t_hi;
+        l_sum = l_sum * alpha + (s_lo + s_hi);
         m_ref = m_new;
         // Rescale this row of O when the reference maximum moved (O of the
         // previous tile is complete: S of this tile was committed after it).
@@ -430,7 +523,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[wg]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[wg]);
+        if (lane == 0 && (warp & 3) == 0) CCA_TRACE_EV(12 + 10 * wg, g);
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(&o_full[wg], it & 1, abort_flag, budget));
@@ -476,7 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row_ok) *reinterpret_cast<float2 *>(a.ws_ml + prow * 2) = make_float2(m_ref, l_sum);
       }
       tc_fence_before();
-      mbar_arrive(&o_empty[wg]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[wg]);
       ++it;
     }
   }
@@ -636,6 +732,18 @@ using namespace cca;
 
 extern "C" {
 
+#ifdef CCA_TRACE
+// Trace builds only: copy the 4 x 16K trace records to host and clear them.
+int cca_debug_trace_read(unsigned long long *host, int max_n) {
+  const int n = max_n < (4 << 14) ? max_n : (4 << 14);
+  cudaDeviceSynchronize();
+  cudaMemcpyFromSymbol(host, g_trace, n * sizeof(unsigned long long));
+  static unsigned long long zeros[4 << 14];
+  cudaMemcpyToSymbol(g_trace, zeros, sizeof(zeros));
+  return n;
+}
+#endif
+
 cca_status cca_chunk_attn_workspace_size(const cca_kv_ring *ring, int32_t n_q_max, size_t *bytes) {
   if (!ring || !bytes || n_q_max < 0 || n_q_max > ring->d.chunk_len)
     return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn_workspace_size: bad argument");
@@ -695,8 +803,9 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q, const void *k_
   const double scale = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(d.head_dim));
   args.scale_log2 = static_cast<float>(scale * 1.4426950408889634);  // scale * log2(e)
   args.wait_budget = static_cast<long long>(env_int("CCA_WAIT_BUDGET_MCYCLES", 4000)) * 1000000LL;
-  for (int c = 0; c < kMaxVis; ++c) args.slot[c] = -1;
-  for (int c = 0; c + 1 < p.n_vis; ++c) args.slot[c] = static_cast<int8_t>(p.slots[c]);
+  args.n_vis = p.n_vis;
+  args.slots_packed = 0;
+  for (int c = 0; c + 1 < p.n_vis; ++c) args.slots_packed |= static_cast<uint64_t>(p.slots[c] & 15) << (4 * c);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d.head_dim == 128) return launch_bf16<128>(ring, p, args, q, k_cur, v_cur, st);
   return launch_bf16<64>(ring, p, args, q, k_cur, v_cur, st);

@@ -62,6 +62,17 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, long 
   }
 }
 
+// One lane of the (converged) warp returns true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_3d(const CUtensorMap *tm, uint64_t *bar, uint32_t dst, int c0, int c1,
                                             int c2) {
@@ -199,11 +210,83 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       CCA_W8(0), CCA_W8(8), CCA_W8(16), CCA_W8(24)
       : "memory");
 }
+#define CCA_W4(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3])
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      CCA_W4(0), CCA_W4(4), CCA_W4(8), CCA_W4(12)
+      : "memory");
+}
+#undef CCA_W4
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 #undef CCA_R8
 #undef CCA_RW8
 #undef CCA_W8
+
+// Per-warpgroup register budget change (all warps of the warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Packed pair of fp32 values in one 64-bit register (Blackwell f32x2 ALU ops).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^a, 2^b on the FMA pipe: n = round(x) via the 1.5 * 2^23 trick, f = x - n,
+// 2^f by a degree-3 minimax polynomial (relative error 7.5e-5, fitted by
+// chunk_causal_attention_b200/exp2_poly.py), and 2^n inserted by adding n << 23
+// to the bit pattern.  Inputs are clamped at -126 (results below 2^-126 are
+// immaterial next to the bf16 rounding of P).
+__device__ __forceinline__ void exp2_poly_pair(float &a, float &b) {
+  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+  constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(a, -126.f), fmaxf(b, -126.f));
+  const uint64_t t = f2_add(x, f2_pack(kMagic, kMagic));
+  const uint64_t r = f2_add(t, f2_pack(-kMagic, -kMagic));
+  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f2_pack(kC3, kC3), f, f2_pack(kC2, kC2));
+  p = f2_fma(p, f, f2_pack(kC1, kC1));
+  p = f2_fma(p, f, f2_pack(kC0, kC0));
+  float pa, pb, ta, tb;
+  f2_unpack(p, pa, pb);
+  f2_unpack(t, ta, tb);
+  a = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
+  b = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
