@@ -21,7 +21,7 @@ import torch
 
 __all__ = [
     "CCA_BF16", "CCA_E4M3", "CCA_F32", "CcaError", "KVRing", "lib", "lib_path", "EXPORTED",
-    "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size",
+    "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc",
     "cca_token_mask_l2", "cca_compact", "cca_scatter", "cca_version", "cca_take_launch_count",
 ]
 
@@ -34,8 +34,8 @@ _STATUS = {0: "CCA_OK", 1: "CCA_ERR_INVALID_ARG", 2: "CCA_ERR_UNSUPPORTED", 3: "
 EXPORTED = (
     "cca_kv_ring_create", "cca_kv_ring_destroy", "cca_kv_ring_reset", "cca_kv_ring_query",
     "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn",
-    "cca_chunk_attn_workspace_size", "cca_token_mask_l2", "cca_compact", "cca_scatter",
-    "cca_last_error", "cca_version", "cca_take_launch_count",
+    "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_token_mask_l2", "cca_compact",
+    "cca_scatter", "cca_last_error", "cca_version", "cca_take_launch_count",
 )
 
 
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
         "cca_quant_e4m3": [vp, ctypes.c_int, i32, i32, i32, vp, vp, vp],
         "cca_chunk_attn": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp],
         "cca_chunk_attn_workspace_size": [vp, i32, ctypes.POINTER(sz)],
+        "cca_chunk_attn_noalloc": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp],
         "cca_token_mask_l2": [vp, vp, i32, i32, f32, f32, vp, vp, vp, vp],
         "cca_compact": [vp, i32, vp, vp, vp],
         "cca_scatter": [vp, vp, vp, i32, i32, vp, vp],
@@ -260,6 +261,28 @@ def cca_chunk_attn(ring: KVRing, q: torch.Tensor, k_cur: torch.Tensor, v_cur: to
                                 _ptr(n_q_dev, "n_q_dev", torch.int32), int(n_q_max), float(softmax_scale),
                                 _ptr(out, "out", torch.bfloat16), _ptr(workspace, "workspace"), ws_bytes,
                                 _stream(stream)), "cca_chunk_attn")
+    return out
+
+
+def cca_chunk_attn_noalloc(ring: KVRing, q: torch.Tensor, k_cur: torch.Tensor, v_cur: torch.Tensor,
+                           q_scale=None, kcur_scale=None, vcur_scale=None, q_idx: Optional[torch.Tensor] = None,
+                           n_q_dev: Optional[torch.Tensor] = None, n_q_max: Optional[int] = None,
+                           softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """cca_chunk_attn without a workspace argument: for callers that cannot give
+    the library device scratch memory (see include/cca.h).  Scratch comes from an
+    array built into libcca.so that all calls share, so calls must not overlap on
+    the GPU.  ``out`` must be provided by callers that may not allocate at all."""
+    if n_q_max is None:
+        n_q_max = q_idx.shape[0] if q_idx is not None else q.shape[0]
+    if out is None:
+        out = torch.empty((n_q_max, ring.n_heads, ring.head_dim), dtype=torch.bfloat16, device=q.device)
+    _check(lib().cca_chunk_attn_noalloc(ring.handle, _ptr(q, "q"), _ptr(k_cur, "k_cur"), _ptr(v_cur, "v_cur"),
+                                        _ptr(q_scale, "q_scale"), _ptr(kcur_scale, "kcur_scale"),
+                                        _ptr(vcur_scale, "vcur_scale"), _ptr(q_idx, "q_idx", torch.int32),
+                                        _ptr(n_q_dev, "n_q_dev", torch.int32), int(n_q_max), float(softmax_scale),
+                                        _ptr(out, "out", torch.bfloat16), _stream(stream)),
+           "cca_chunk_attn_noalloc")
     return out
 
 

@@ -812,3 +812,65 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q, const void *k_
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free variant
+// Some callers cannot hand this library a scratch buffer: a real-time stream
+// loop that must not call the device allocator once it is running (an
+// allocation can synchronise the device and stall the stream), or a host
+// application that owns every device allocation itself and exposes no
+// allocator to plug-ins.  cca_chunk_attn_noalloc serves them from one scratch
+// array that lives in this library's device image.
+namespace cca {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB per GPU that loads the library
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array on the current device, looked up once
+// per device.  In host code the array's name is only a stand-in, never a
+// device address, so it must go through cudaGetSymbolAddress.
+static cca_status noalloc_scratch(void **out) {
+  static std::mutex mu;
+  static void *addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "cca_chunk_attn_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(CCA_ERR_UNSUPPORTED, "cca_chunk_attn_noalloc: device index %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(CCA_ERR_CUDA, "cca_chunk_attn_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return CCA_OK;
+}
+
+}  // namespace cca
+
+extern "C" {
+
+cca_status cca_chunk_attn_noalloc(const cca_kv_ring *ring, const void *q, const void *k_cur, const void *v_cur,
+                                  const float *q_scale, const float *kcur_scale, const float *vcur_scale,
+                                  const int32_t *q_idx, const int32_t *n_q_dev, int32_t n_q_max,
+                                  float softmax_scale, void *out, cca_stream_t stream) {
+  if (!ring) return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn_noalloc: NULL ring");
+  if (n_q_max < 0 || n_q_max > ring->d.chunk_len)
+    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn_noalloc: need 0 <= n_q_max <= chunk_len (%d)",
+                ring->d.chunk_len);
+  AttnPlan p;
+  plan_attention(ring, n_q_max, p);
+  const size_t need = workspace_bytes_for(ring, n_q_max, p);
+  if (need > kNoAllocScratchBytes)
+    return fail(CCA_ERR_INVALID_ARG,
+                "cca_chunk_attn_noalloc: this call needs %zu bytes of scratch, more than the %zu-byte built-in "
+                "array; use cca_chunk_attn with a caller-provided workspace",
+                need, kNoAllocScratchBytes);
+  void *scratch = nullptr;
+  CCA_TRY(noalloc_scratch(&scratch));
+  return cca_chunk_attn(ring, q, k_cur, v_cur, q_scale, kcur_scale, vcur_scale, q_idx, n_q_dev, n_q_max,
+                        softmax_scale, out, scratch, kNoAllocScratchBytes, stream);
+}
+
+}  // extern "C"

@@ -180,6 +180,31 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q,
 cca_status cca_chunk_attn_workspace_size(const cca_kv_ring *ring, int32_t n_q_max,
                                          size_t *bytes);
 
+/* Allocation-free cca_chunk_attn (no counterpart on the pages: a service for
+ * callers that cannot provide device scratch memory, such as a real-time
+ * stream loop that must not call the device allocator once running, or a host
+ * application that owns every device allocation and gives plug-ins no
+ * allocator).  Same arguments and results as cca_chunk_attn without the
+ * workspace: the split-KV partial results go to a 64 MiB array compiled into
+ * this library, which every GPU that loads the library holds until the
+ * process exits.
+ *  - No cudaMalloc, cudaFree or other allocating call is made.  The first call
+ *    on each device looks the array's device address up once
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents
+ *    (nothing in it needs to start at zero).  Calls that may overlap on the
+ *    GPU (different streams, or different host threads) race on it: serialise
+ *    them, or use cca_chunk_attn with separate workspaces.
+ *  - Errors: as cca_chunk_attn, plus CCA_ERR_INVALID_ARG when the call needs
+ *    more scratch than the array holds (the message gives both sizes). */
+cca_status cca_chunk_attn_noalloc(const cca_kv_ring *ring, const void *q,
+                                  const void *k_cur, const void *v_cur,
+                                  const float *q_scale, const float *kcur_scale,
+                                  const float *vcur_scale, const int32_t *q_idx,
+                                  const int32_t *n_q_dev, int32_t n_q_max,
+                                  float softmax_scale, void *out,
+                                  cca_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* L2 token mask, compaction, scatter (LiveEdit mask cache)                 */
 /* ------------------------------------------------------------------------ */
