@@ -167,6 +167,149 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ extra workloads (rank-local)
+def _timed(fn, reps, stream, warm=3):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def extra_workloads(dev, stream, peak_tf, peak_gbs):
+    """FP8 720p attention, the mask-cached chunk, the 225-chunk latency drift and
+    the memory-bound kernels' bandwidth.  Each is timed with CUDA events."""
+    import torch
+    import synth
+    import chunk_causal_attention_b200 as cca
+    bf = lambda x: synth.as_torch_bf16(x, dev)
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # L2 flush between reps
+
+    # ---- e4m3 attention at the 720p shape (Student-t inputs)
+    s3 = synth.fp8_720p(n_steps=1)
+    ring8 = cca.KVRing(H, D, L, W, dtype="e4m3", device=dev)
+    for t in range(s3.t):
+        ring8.append(bf(s3.ring_k[t]), bf(s3.ring_v[t]))
+    q8, qs = cca.cca_quant_e4m3(bf(s3.q[0]))
+    k8, ks = cca.cca_quant_e4m3(bf(s3.k_cur[0]))
+    v8, vs = cca.cca_quant_e4m3(bf(s3.v_cur[0]))
+    o8 = torch.empty((L, H, D), dtype=torch.bfloat16, device=dev)
+    ws8 = torch.empty(max(cca.cca_chunk_attn_workspace_size(ring8, L), 16), dtype=torch.uint8, device=dev)
+
+    t8 = _timed(lambda: cca.cca_chunk_attn(ring8, q8, k8, v8, q_scale=qs, kcur_scale=ks, vcur_scale=vs,
+                                             out=o8, workspace=ws8), 50, stream)
+    us8 = float(np.median(t8)) * 1e3
+    out["fp8_720p"] = {"attn_us_per_call": us8, "tflops": FLOP_PER_CALL / (us8 * 1e-6) / 1e12,
+                       "frac_of_fp8_peak": FLOP_PER_CALL / (us8 * 1e-6) / 1e12 / (2 * peak_tf),
+                       "note": "QK^T on e4m3 tensor cores, PV in fp16 (P kept 16-bit); fp8 peak = 2 x bf16 measured"}
+
+    # ---- mask-cached chunk: mask (dynamic tau) + compaction + active-query attention + scatter
+    c1 = synth.chunk_720p(n_steps=1)
+    m = synth.mask_chunk()
+    ring = cca.KVRing(H, D, L, W, device=dev)
+    for t in range(c1.t):
+        ring.append(bf(c1.ring_k[t]), bf(c1.ring_v[t]))
+    q, kc, vc = bf(c1.q[0]), bf(c1.k_cur[0]), bf(c1.v_cur[0])
+    src, edit = torch.from_numpy(m.src).to(dev), torch.from_numpy(m.edit).to(dev)
+    cache = bf(m.o_cache)
+    mask = torch.empty(L, dtype=torch.uint8, device=dev)
+    idx = torch.empty(L, dtype=torch.int32, device=dev)
+    n_act = torch.empty(1, dtype=torch.int32, device=dev)
+    oc = torch.empty((L, H, D), dtype=torch.bfloat16, device=dev)
+    wsm = torch.empty(max(cca.cca_chunk_attn_workspace_size(ring, L), 16), dtype=torch.uint8, device=dev)
+
+    def chunk4():
+        cca.cca_token_mask_l2(src, edit, prune_quantile=m.prune_quantile, mask=mask)
+        cca.cca_compact(mask, idx, n_act)
+        cca.cca_chunk_attn(ring, q, kc, vc, q_idx=idx, n_q_dev=n_act, n_q_max=L, out=oc, workspace=wsm)
+        cca.cca_scatter(oc, idx, n_act, cache, n_max=L)
+    t4 = _timed(chunk4, 50, stream)
+    t4a = _timed(lambda: cca.cca_chunk_attn(ring, q, kc, vc, q_idx=idx, n_q_dev=n_act, n_q_max=L, out=oc,
+                                            workspace=wsm), 50, stream)
+    n_active = int(n_act.item())
+    flop4 = 4.0 * n_active * LK * H * D
+    out["mask_cached_720p"] = {"n_active": n_active, "ms_per_chunk": float(np.median(t4)),
+                               "attn_us": float(np.median(t4a)) * 1e3,
+                               "attn_tflops": flop4 / (float(np.median(t4a)) * 1e-3) / 1e12}
+
+    # ---- long stream: per-chunk latency over 225 chunks (AR(1) K/V made on the device).
+    # Three passes (fresh ring each); per-chunk medians over the passes damp
+    # clock changes of the shared, power-capped GPU.
+    def stream_pass(seed):
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed)
+        ring2 = cca.KVRing(H, D, L, W, device=dev)
+        xk = torch.randn((L, H, D), generator=gen, device=dev)
+        xv = torch.randn((L, H, D), generator=gen, device=dev)
+        qq = torch.randn((2, L, H, D), generator=gen, device=dev).to(torch.bfloat16)
+        o2 = torch.empty((L, H, D), dtype=torch.bfloat16, device=dev)
+        ws2 = torch.empty(max(cca.cca_chunk_attn_workspace_size(ring2, L), 16), dtype=torch.uint8, device=dev)
+        lat = []
+        for t in range(225):
+            kb, vb = xk.to(torch.bfloat16), xv.to(torch.bfloat16)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for st in range(CALLS_PER_STEP):
+                cca.cca_chunk_attn(ring2, qq[st], kb, vb, out=o2, workspace=ws2)
+            ring2.append(kb, vb)
+            b.record(stream)
+            lat.append((a, b))
+            xk = 0.9 * xk + 0.44 * torch.randn((L, H, D), generator=gen, device=dev)
+            xv = 0.9 * xv + 0.44 * torch.randn((L, H, D), generator=gen, device=dev)
+        torch.cuda.synchronize()
+        return np.array([a.elapsed_time(b) for a, b in lat])
+    passes = np.stack([stream_pass(2 + k) for k in range(3)])
+    ms = np.median(passes, axis=0)
+    early, late = float(np.median(ms[5:30])), float(np.median(ms[200:225]))
+    slope = float(np.polyfit(np.arange(5, 225), ms[5:225], 1)[0])
+    drift_each = [float((np.median(p[200:225]) - np.median(p[5:30])) / np.median(p[5:30]) * 100) for p in passes]
+    out["long_stream_225"] = {"ms_per_chunk_median_5_29": early, "ms_per_chunk_median_200_224": late,
+                              "drift_pct": (late - early) / early * 100.0, "drift_pct_each_pass": drift_each,
+                              "ols_slope_ms_per_chunk": slope, "first_chunks_ms": [float(x) for x in ms[:5]],
+                              "passes": 3}
+
+    # ---- memory-bound kernels (bandwidth, L2 flushed before each rep)
+    def bw(fn, nbytes, reps=20):
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        t = float(np.median(ts)) * 1e-3
+        return {"us": t * 1e6, "gbs": nbytes / t / 1e9, "frac_of_hbm": nbytes / t / 1e9 / peak_gbs}
+    ringa = cca.KVRing(H, D, L, W, device=dev)
+    kk, vv = bf(c1.ring_k[0]), bf(c1.ring_v[0])
+    out["append_720p"] = bw(lambda: ringa.append(kk, vv), 4 * L * H * D * 2)
+    nbig = 1 << 24
+    srcb = torch.randn((nbig, 16), device=dev)
+    editb = srcb + 0.5 * torch.randn((nbig, 16), device=dev)
+    maskb = torch.empty(nbig, dtype=torch.uint8, device=dev)
+    out["mask_fixed_16M_tokens"] = bw(lambda: cca.cca_token_mask_l2(srcb, editb, tau=2.0, mask=maskb),
+                                      nbig * (2 * 16 * 4 + 1))
+    out["mask_dynamic_720p_us"] = float(np.median(_timed(
+        lambda: cca.cca_token_mask_l2(src, edit, prune_quantile=0.7, mask=mask), 50, stream))) * 1e3
+    ncomp = 1 << 20
+    mc = (torch.rand(ncomp, device=dev) < 0.3).to(torch.uint8)
+    idxc = torch.empty(ncomp, dtype=torch.int32, device=dev)
+    nc = torch.empty(1, dtype=torch.int32, device=dev)
+    cca.cca_compact(mc, idxc, nc)
+    torch.cuda.synchronize()
+    out["compact_1M_tokens"] = bw(lambda: cca.cca_compact(mc, idxc, nc), ncomp + 4 * int(nc.item()))
+    out["scatter_720p"] = bw(lambda: cca.cca_scatter(oc, idx, n_act, cache, n_max=L), 2 * n_active * H * D * 2)
+    return out
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args, rank, world, local_rank):
     import torch
@@ -312,6 +455,10 @@ def run_gpu(args, rank, world, local_rank):
         "clocks": clocks,
         "e2e": e2e,
     }
+    if args.extras:
+        peak_tf_, peak_gbs_, _ = peaks()
+        line["extra"] = extra_workloads(torch.device("cuda", local_rank), torch.cuda.current_stream(), peak_tf_,
+                                        peak_gbs_)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
@@ -325,6 +472,8 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extras", type=int, default=1, help="also time the fp8, mask-cached, long-stream and "
+                    "memory-bound workloads (rank 0, extra keys)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))

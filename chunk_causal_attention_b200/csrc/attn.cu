@@ -1,4 +1,4 @@
-// Chunk-wise causal attention over the bounded KV cache, BF16, sm_100a.
+// Chunk-wise causal attention over the bounded KV cache, BF16 and FP8 e4m3, sm_100a.
 //
 // What it computes ["JoyAI-Video-Edit 소개", section 청크 단위 자기회귀 적응;
 // "論文解説: JoyAI-Video-Edit", step 1 (§4.1)]: the queries of the current chunk
@@ -22,14 +22,18 @@
 //  * online softmax in base 2 with the scale folded in; the running maximum is
 //    only moved (and O rescaled in TMEM) when a row's maximum grows by more
 //    than 2^8, so P never exceeds 256 and rescales are rare;
-//  * split-KV: items can cover part of the KV list; partial (O, m, l) go to the
-//    caller's workspace and a small combine kernel merges them;
+//  * persistent schedule computed on the device from the query count: each CTA
+//    first takes whole (query pair, head) items; the remaining items are split
+//    evenly over all CTAs along the KV list, their partial (O, m, l) go to the
+//    caller's workspace and a small combine kernel merges only those;
 //  * every mbarrier wait is bounded; on timeout the CTA sets an abort flag,
 //    drains its in-flight TMA loads and MMAs, frees TMEM and reports
 //    CCA_DEV_TIMEOUT through the ring's status word.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <cmath>
 #include <cstdlib>
@@ -88,32 +92,40 @@ __device__ unsigned long long g_trace[4 << 14];
 #endif
 
 struct AttnArgs {
-  const __nv_bfloat16 *q;  // query rows (gather path)
+  const void *q;           // query rows (gather path): [L][H][D] of the ring's element type
   const int32_t *q_idx;    // NULL: dense rows
   const int32_t *n_q_dev;  // NULL: n_q = n_q_max
   __nv_bfloat16 *out;      // [n_q_max][H][D]
-  float *ws_o;             // [n_splits][n_q_max][H][D] partial O (unnormalised)
-  float *ws_ml;            // [n_splits][n_q_max][H][2] (running max in log2 units, row sum)
+  float *ws_o;             // [2 x grid][256][D] partial O of split items (unnormalised)
+  float *ws_ml;            // [2 x grid][256][2] (running max in log2 units, row sum)
   int32_t *dev_status;
+  // e4m3 only: per-head dequantisation scales of Q, of the current chunk's K/V
+  // ([H]) and of the ring slots' K/V ([(1+W)][H]).
+  const float *q_scale, *kcur_scale, *vcur_scale, *k_scale, *v_scale;
   int n_q_max, L, H;
-  int n_pairs, n_splits;
-  int tiles_per_chunk, n_kv_tiles, n_items;
+  int tiles_per_chunk, n_kv_tiles;
   float scale_log2;
   long long wait_budget;
   int n_vis;               // visible chunks, the current one last
   uint64_t slots_packed;   // 4-bit ring slot of visible chunk c at bits [4c, 4c+4)
 };
 
-template <int D>
+// Shared-memory plan.  Q/K/V tiles arrive by TMA as 128-row x 128-byte boxes
+// with the 128-byte swizzle (two boxes per tile for bf16 D=128).  For e4m3, V
+// tiles are expanded to fp16 in a separate buffer for the 16-bit PV MMA.
+template <int D, bool kFp8>
 struct AttnSmem {
-  static constexpr uint32_t kBox = 128 * 128;        // 128 rows x 128 bytes (one SW128 box)
-  static constexpr uint32_t kNBox = D / 64;          // boxes per 128-row tile
-  static constexpr uint32_t kTile = kBox * kNBox;    // bytes of one Q/K/V tile
+  static constexpr uint32_t kEsz = kFp8 ? 1 : 2;             // bytes per Q/K/V element
+  static constexpr uint32_t kBox = 128 * 128;                // 128 rows x 128 bytes
+  static constexpr uint32_t kNBox = D * kEsz / 128;          // boxes per 128-row tile
+  static constexpr uint32_t kTile = kBox * kNBox;            // bytes of one loaded Q/K/V tile
+  static constexpr uint32_t kV16Tile = kFp8 ? 128 * D * 2 : 0;
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + kNQ * kTile;
   static constexpr uint32_t kV = kK + kNS * kTile;
-  static constexpr uint32_t kBar = kV + kNS * kTile;
-  static constexpr uint32_t kNumBars = 4 + 4 * kNS + 8 + 1;
+  static constexpr uint32_t kV16 = kV + kNS * kTile;
+  static constexpr uint32_t kBar = kV16 + kNS * kV16Tile;
+  static constexpr uint32_t kNumBars = 4 + 6 * kNS + 8 + 1;
   static constexpr uint32_t kBytes = kBar + kNumBars * 8 + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
@@ -125,34 +137,93 @@ __device__ __forceinline__ void kv_tile_coords(const AttnArgs &a, int j, int &sl
   slot = c == a.n_vis - 1 ? -1 : static_cast<int>((a.slots_packed >> (4 * c)) & 15u);
 }
 
-template <int D>
+__device__ __forceinline__ int vis_slot(const AttnArgs &a, int c) {
+  return c == a.n_vis - 1 ? -1 : static_cast<int>((a.slots_packed >> (4 * c)) & 15u);
+}
+
+// ---- work schedule (identical in every role, the combine kernel included)
+// Items are (query pair, head), pair-major, for the pairs holding the first n_q
+// queries.  With G CTAs: CTA c takes items c, c + G, ... for q = items / G full
+// rounds; the r = items % G remaining items form a list of r * n_kv KV tiles cut
+// into G near-equal ranges, so CTA c also takes 0, 1 or 2 partial segments.
+// Partial segment k (0 or 1) of CTA c writes workspace slot 2c + k.
+struct Sched {
+  int n_items, q, r;
+  int64_t tr;  // KV tiles in the remainder list
+};
+struct Seg {
+  int pair, head, j0, j1, slot;  // slot < 0: whole item, direct output
+};
+
+__device__ __forceinline__ Sched make_sched(int n_q, int H, int n_kv, int G) {
+  Sched s;
+  s.n_items = ((n_q + kNQ * kBM - 1) / (kNQ * kBM)) * H;
+  s.q = s.n_items / G;
+  s.r = s.n_items % G;
+  s.tr = static_cast<int64_t>(s.r) * n_kv;
+  return s;
+}
+
+__device__ __forceinline__ bool get_seg(const Sched &s, int H, int n_kv, int G, int c, int k, Seg &g) {
+  if (k < s.q) {
+    const int u = c + k * G;
+    g = {u / H, u % H, 0, n_kv, -1};
+    return true;
+  }
+  k -= s.q;
+  const int64_t lo = static_cast<int64_t>(c) * s.tr / G, hi = static_cast<int64_t>(c + 1) * s.tr / G;
+  if (lo >= hi || k > 1) return false;
+  const int64_t u0 = lo / n_kv;
+  if (k == 0) {
+    const int u = s.q * G + static_cast<int>(u0);
+    const int64_t e0 = hi < (u0 + 1) * n_kv ? hi : (u0 + 1) * n_kv;
+    g = {u / H, u % H, static_cast<int>(lo - u0 * n_kv), static_cast<int>(e0 - u0 * n_kv), 2 * c};
+    return true;
+  }
+  if (hi <= (u0 + 1) * n_kv) return false;
+  const int u = s.q * G + static_cast<int>(u0) + 1;
+  g = {u / H, u % H, 0, static_cast<int>(hi - (u0 + 1) * n_kv), 2 * c + 1};
+  return true;
+}
+
+// Dequantisation scale of chunk (slot) for one head: ring slot or current chunk.
+__device__ __forceinline__ float chunk_scale(const float *ring, const float *cur, int slot, int H, int head) {
+  return slot < 0 ? __ldg(cur + head) : __ldg(ring + slot * H + head);
+}
+
+template <int D, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kr,
-                     const __grid_constant__ CUtensorMap tm_vr, const __grid_constant__ CUtensorMap tm_kc,
-                     const __grid_constant__ CUtensorMap tm_vc, const AttnArgs a) {
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kr,
+                const __grid_constant__ CUtensorMap tm_vr, const __grid_constant__ CUtensorMap tm_kc,
+                const __grid_constant__ CUtensorMap tm_vc, const AttnArgs a) {
   using namespace sm100;
-  using S = AttnSmem<D>;
+  using S = AttnSmem<D, kFp8>;
+  static_assert(!kFp8 || D == 128, "e4m3 path is built for head_dim 128");
+  constexpr int kBoxElems = 128 / S::kEsz;  // elements of D per TMA box
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t *gbase = smem_raw + (base - raw);
   uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + S::kBar);
-  uint64_t *q_full = bars;           // [kNQ]  producer -> MMA
-  uint64_t *q_empty = bars + 2;      // [kNQ]  MMA -> producer
-  uint64_t *k_full = bars + 4;       // [kNS]
-  uint64_t *k_empty = k_full + kNS;  // [kNS]
-  uint64_t *v_full = k_empty + kNS;  // [kNS]
-  uint64_t *v_empty = v_full + kNS;  // [kNS]
-  uint64_t *s_full = v_empty + kNS;  // [2] MMA -> softmax: S ready
-  uint64_t *p_full = s_full + 2;     // [2] softmax -> MMA: P ready (and O rescaled)
-  uint64_t *o_full = p_full + 2;     // [2] MMA -> softmax: O final for the item
-  uint64_t *o_empty = o_full + 2;    // [2] softmax -> MMA: O read out
-  uint64_t *drain = o_empty + 2;     // [1] teardown: all MMAs complete
+  uint64_t *q_full = bars;              // [kNQ]  producer -> MMA
+  uint64_t *q_empty = bars + 2;         // [kNQ]  MMA -> producer
+  uint64_t *k_full = bars + 4;          // [kNS]
+  uint64_t *k_empty = k_full + kNS;     // [kNS]
+  uint64_t *v_full = k_empty + kNS;     // [kNS]  V tile landed
+  uint64_t *v_empty = v_full + kNS;     // [kNS]  V tile consumed (MMA, or the e4m3 expanders)
+  uint64_t *v16_full = v_empty + kNS;   // [kNS]  e4m3: fp16 V ready
+  uint64_t *v16_empty = v16_full + kNS; // [kNS]  e4m3: fp16 V consumed by the MMAs
+  uint64_t *s_full = v16_empty + kNS;   // [2] MMA -> softmax: S ready
+  uint64_t *p_full = s_full + 2;        // [2] softmax -> MMA: P ready (and O rescaled)
+  uint64_t *o_full = p_full + 2;        // [2] MMA -> softmax: O final for the item
+  uint64_t *o_empty = o_full + 2;       // [2] softmax -> MMA: O read out
+  uint64_t *drain = o_empty + 2;        // [1] teardown: all MMAs complete
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_q = a.n_q_dev ? min(max(*a.n_q_dev, 0), a.n_q_max) : a.n_q_max;
+  const Sched sch = make_sched(n_q, a.H, a.n_kv_tiles, gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -167,7 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
+      mbar_init(&v_empty[s], kFp8 ? 2 : 1);  // e4m3: released by the two expander warps
+      mbar_init(&v16_full[s], 2);
+      mbar_init(&v16_empty[s], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -200,14 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;       // items handled by this CTA
     int q_armed = 0;  // Q phases armed (per tile, identical for both)
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-      const int split = item % a.n_splits;
-      const int rest = item / a.n_splits;
-      const int pair = rest % a.n_pairs;
-      const int head = rest / a.n_pairs;
-      if (pair * (kNQ * kBM) >= n_q) continue;
-      const int j0 = static_cast<int>(static_cast<int64_t>(split) * a.n_kv_tiles / a.n_splits);
-      const int j1 = static_cast<int>(static_cast<int64_t>(split + 1) * a.n_kv_tiles / a.n_splits);
+    for (int kseg = 0; ok; ++kseg) {
+      Seg sg;
+      if (!get_seg(sch, a.H, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      const int pair = sg.pair, head = sg.head, j0 = sg.j0, j1 = sg.j1;
       for (int i = 0; i < kNQ && ok; ++i) {
         if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[i], (it - 1) & 1, abort_flag, budget));
         if (!ok) break;
@@ -217,30 +286,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             mbar_arrive_expect_tx(&q_full[i], S::kTile);
             for (uint32_t b = 0; b < S::kNBox; ++b)
-              tma_load_3d(&tm_q, &q_full[i], dstq + b * S::kBox, b * 64, head, row0);
+              tma_load_3d(&tm_q, &q_full[i], dstq + b * S::kBox, b * kBoxElems, head, row0);
           }
         } else {
-          // Gather: row r of the tile is query q_idx[row0 + r]; written in the
-          // same 128B-swizzled layout the TMA would produce.
-          constexpr int kChunks = D / 8;  // 16-byte chunks per row
-          for (int e = lane; e < kBM * kChunks; e += 32) {
-            const int r = e / kChunks, c = e % kChunks;
-            const int qr = row0 + r;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (qr < n_q) {
-              const int src = a.q_idx[qr];
-              if (src >= 0 && src < a.L) {
-                v = __ldg(reinterpret_cast<const uint4 *>(a.q + (static_cast<int64_t>(src) * a.H + head) * D) + c);
-              } else if (a.dev_status) {
-                *a.dev_status = CCA_DEV_BAD_INDEX;  // out-of-range query index: row read as zeros
-              }
+          // Gather: row r of the tile is query q_idx[row0 + r], copied with
+          // cp.async (zero-filled for rows past n_q) into the same 128B-swizzled
+          // layout the TMA would produce.  Lane l first reads the indices of rows
+          // l, l+32, l+64, l+96; every 16-byte copy is then issued back to back.
+          constexpr int kChunks = D * S::kEsz / 16;  // 16-byte chunks per row (8 or 16)
+          constexpr int kRowsPerPass = 32 / kChunks;
+          const uint8_t *qb = static_cast<const uint8_t *>(a.q);
+          int src_row[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int qr = row0 + lane + 32 * k;
+            int sr = qr < n_q ? __ldg(a.q_idx + qr) : -1;
+            if (qr < n_q && (sr < 0 || sr >= a.L)) {
+              if (a.dev_status) *a.dev_status = CCA_DEV_BAD_INDEX;  // out-of-range index: row read as zeros
+              sr = -1;
             }
+            src_row[k] = sr;
+          }
+          const int c = lane % kChunks;
+#pragma unroll 4
+          for (int r0 = 0; r0 < kBM; r0 += kRowsPerPass) {
+            const int r = r0 + lane / kChunks;
+            const int k = r >> 5;
+            const int v = k == 0 ? src_row[0] : k == 1 ? src_row[1] : k == 2 ? src_row[2] : src_row[3];
+            const int sr = __shfl_sync(0xffffffffu, v, r & 31);
+            const uint8_t *src = qb + (static_cast<int64_t>(sr < 0 ? 0 : sr) * a.H + head) * D * S::kEsz + c * 16;
             const uint32_t box = c >> 3, cc = c & 7;
             const uint32_t dst = dstq + box * S::kBox + r * 128 + ((cc ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
-                         "r"(v.w)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sr < 0 ? 0 : 16)
                          : "memory");
           }
+          asm volatile("cp.async.wait_all;" ::: "memory");
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&q_full[i]);
@@ -261,9 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&k_full[stage], S::kTile);
           for (uint32_t b = 0; b < S::kNBox; ++b) {
             if (slot < 0)
-              tma_load_3d(&tm_kc, &k_full[stage], dst + b * S::kBox, b * 64, head, row0);
+              tma_load_3d(&tm_kc, &k_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0);
             else
-              tma_load_4d(&tm_kr, &k_full[stage], dst + b * S::kBox, b * 64, head, row0, slot);
+              tma_load_4d(&tm_kr, &k_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
           }
         }
         if (g >= kNS) ok = __all_sync(0xffffffffu, mbar_wait(&v_empty[stage], ph ^ 1, abort_flag, budget));
@@ -274,9 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&v_full[stage], S::kTile);
           for (uint32_t b = 0; b < S::kNBox; ++b) {
             if (slot < 0)
-              tma_load_3d(&tm_vc, &v_full[stage], dst + b * S::kBox, b * 64, head, row0);
+              tma_load_3d(&tm_vc, &v_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0);
             else
-              tma_load_4d(&tm_vr, &v_full[stage], dst + b * S::kBox, b * 64, head, row0, slot);
+              tma_load_4d(&tm_vr, &v_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
           }
         }
       }
@@ -303,28 +383,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     CCA_TRACE_ROLE(1);
     // The whole warp runs this loop converged, so every operand below is
     // warp-uniform; one elected lane issues each batch of tcgen05 instructions.
-    constexpr uint32_t kIdescQK = idesc_make(1, 1, 0, 0, kBM, kBN);  // bf16, Q and K both K-major
-    constexpr uint32_t kIdescPV = idesc_make(1, 1, 0, 1, kBM, D);    // P from TMEM, V MN-major
+    // QK: bf16 x bf16 (kind::f16) or e4m3 x e4m3 (kind::f8f6f4), both K-major.
+    // PV: P (bf16, or fp16 for the e4m3 path) from TMEM, V MN-major in smem.
+    constexpr uint32_t kIdescQK = kFp8 ? idesc_make(0, 0, 0, 0, kBM, kBN) : idesc_make(1, 1, 0, 0, kBM, kBN);
+    constexpr uint32_t kIdescPV = kFp8 ? idesc_make(0, 0, 0, 1, kBM, D) : idesc_make(1, 1, 0, 1, kBM, D);
+    constexpr int kQKSteps = D * S::kEsz / 32;  // 32 bytes of K per MMA
     const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
     // Descriptors of every operand tile, built once; a K step inside a tile is
     // an add to the (address >> 4) field.
     const uint64_t dQ0 = sdesc_sw128(base + S::kQ, 16, 1024);
     const uint64_t dK0 = sdesc_sw128(base + S::kK, 16, 1024);
-    const uint64_t dV0 = sdesc_sw128(base + S::kV, S::kBox, 1024);
+    const uint64_t dV0 = kFp8 ? sdesc_sw128(base + S::kV16, 128 * 128, 1024) : sdesc_sw128(base + S::kV, S::kBox, 1024);
+    constexpr uint32_t kVStageBytes = kFp8 ? S::kV16Tile : S::kTile;
+    uint64_t *pv_full = kFp8 ? v16_full : v_full;
+    uint64_t *pv_empty = kFp8 ? v16_empty : v_empty;
     auto issue_qk = [&](int i, uint32_t stage) {
       const uint64_t qa = dQ0 + ((i * S::kTile) >> 4), kb = dK0 + ((stage * S::kTile) >> 4);
       const uint32_t d = tm + i * 128u;
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < kQKSteps; ++kk) {
           const uint32_t off = ((kk >> 2) * S::kBox + (kk & 3) * 32) >> 4;
-          mma_f16_ss(d, qa + off, kb + off, kIdescQK, kk > 0 ? 1u : 0u);
+          if constexpr (kFp8)
+            mma_f8_ss(d, qa + off, kb + off, kIdescQK, kk > 0 ? 1u : 0u);
+          else
+            mma_f16_ss(d, qa + off, kb + off, kIdescQK, kk > 0 ? 1u : 0u);
         }
       }
       __syncwarp();
     };
     auto issue_pv = [&](int i, uint32_t stage, bool acc) {
-      const uint64_t vb = dV0 + ((stage * S::kTile) >> 4);
+      const uint64_t vb = dV0 + ((stage * kVStageBytes) >> 4);
       const uint32_t d = tm + 256u + i * D, pa = tm + i * 128u;
       if (elect_one()) {
 #pragma unroll
@@ -343,12 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t g = 0;
     int it = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-      const int split = item % a.n_splits;
-      const int pair = (item / a.n_splits) % a.n_pairs;
-      if (pair * (kNQ * kBM) >= n_q) continue;
-      const int j0 = static_cast<int>(static_cast<int64_t>(split) * a.n_kv_tiles / a.n_splits);
-      const int j1 = static_cast<int>(static_cast<int64_t>(split + 1) * a.n_kv_tiles / a.n_splits);
+    for (int kseg = 0; ok; ++kseg) {
+      Seg sg;
+      if (!get_seg(sch, a.H, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      const int j0 = sg.j0, j1 = sg.j1;
       const int n = j1 - j0;
       ok = wait(&q_full[0], it & 1) && wait(&q_full[1], it & 1);
       if (!ok) break;
@@ -368,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) CCA_TRACE_EV(3, g - 1);
           tc_fence_after();
           issue_pv(1, pst, jj > 1);
-          commit(&v_empty[pst]);
+          commit(&pv_empty[pst]);
         }
         issue_qk(1, stage);
         commit(&s_full[1]);
@@ -378,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           commit(&q_empty[0]);
           commit(&q_empty[1]);
         }
-        if (!(ok = wait(&v_full[stage], ph))) break;
+        if (!(ok = wait(&pv_full[stage], ph))) break;
         if (jj == 0 && it > 0 && !(ok = wait(&o_empty[0], (it - 1) & 1))) break;
         if (!(ok = wait(&p_full[0], g & 1))) break;
         if (lane == 0) CCA_TRACE_EV(5, g);
@@ -394,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait(&p_full[1], (g - 1) & 1))) break;
         tc_fence_after();
         issue_pv(1, pst, n > 1);
-        commit(&v_empty[pst]);
+        commit(&pv_empty[pst]);
         commit(&o_full[1]);
       }
       ++it;
@@ -404,8 +491,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_drain(drain, 0, budget);
     __syncwarp();
   }
+  // ================================================================ e4m3 V expanders
   else if (warp < 4) {
     if (kUseSetMaxNReg) regs_dec<88>();
+    if constexpr (kFp8) {
+      // Warps 2-3 turn each landed e4m3 V tile (128 rows x 128 bytes, swizzled)
+      // into an fp16 tile (two 128 x 64 boxes, swizzled) for the PV MMA.  The
+      // conversion is exact: every e4m3 value is an fp16 value.
+      const int t = threadIdx.x - 64;  // 0..63
+      uint32_t g = 0;
+      bool ok = true;
+      for (int kseg = 0; ok; ++kseg) {
+        Seg sg;
+        if (!get_seg(sch, a.H, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+        const int j0 = sg.j0, j1 = sg.j1;
+        for (int j = j0; j < j1; ++j, ++g) {
+          const uint32_t stage = g % kNS, ph = (g / kNS) & 1;
+          ok = __all_sync(0xffffffffu, mbar_wait(&v_full[stage], ph, abort_flag, budget));
+          if (ok && g >= kNS) ok = __all_sync(0xffffffffu, mbar_wait(&v16_empty[stage], ph ^ 1, abort_flag, budget));
+          if (!ok) break;
+          const uint32_t src = base + S::kV + stage * S::kTile;
+          const uint32_t dst = base + S::kV16 + stage * S::kV16Tile;
+#pragma unroll 4
+          for (int e = t; e < 128 * 8; e += 64) {  // 16-byte source chunks
+            const int r = e >> 3, c = e & 7;
+            uint32_t w[4];
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(src + r * 128 + ((c ^ (r & 7)) << 4)));
+            uint32_t h[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[k] & 0xffffu), __NV_E4M3);
+              const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[k] >> 16), __NV_E4M3);
+              h[2 * k] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
+              h[2 * k + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
+            }
+            // elements 16c .. 16c+15 -> box (c >> 2), 16-byte chunks 2(c&3) and 2(c&3)+1
+            const uint32_t ob = dst + (c >> 2) * (128 * 128) + r * 128;
+            const uint32_t c0 = (2 * (c & 3)) ^ (r & 7), c1 = (2 * (c & 3) + 1) ^ (r & 7);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ob + (c0 << 4)), "r"(h[0]), "r"(h[1]),
+                         "r"(h[2]), "r"(h[3])
+                         : "memory");
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ob + (c1 << 4)), "r"(h[4]), "r"(h[5]),
+                         "r"(h[6]), "r"(h[7])
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&v16_full[stage]);
+            mbar_arrive(&v_empty[stage]);
+          }
+        }
+      }
+    }
   }
   // ================================================================ softmax
   else {
@@ -415,24 +555,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + wg * 128u;
     const uint32_t tO = tmem + lane_off + 256u + wg * D;
-    const float sl2 = a.scale_log2;
     CCA_TRACE_ROLE(2 + wg);
     uint32_t g = 0;
     int it = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-      const int split = item % a.n_splits;
-      const int rest = item / a.n_splits;
-      const int pair = rest % a.n_pairs;
-      const int head = rest / a.n_pairs;
-      if (pair * (kNQ * kBM) >= n_q) continue;
-      const int j0 = static_cast<int>(static_cast<int64_t>(split) * a.n_kv_tiles / a.n_splits);
-      const int j1 = static_cast<int>(static_cast<int64_t>(split + 1) * a.n_kv_tiles / a.n_splits);
+    for (int kseg = 0; ok; ++kseg) {
+      Seg sg;
+      if (!get_seg(sch, a.H, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      const int pair = sg.pair, head = sg.head, j0 = sg.j0, j1 = sg.j1;
+      // e4m3: scores carry the factor s_q * s_k(chunk); V's factor s_v(chunk) is
+      // folded into P relative to the largest s_v of the visible chunks, which
+      // the epilogue multiplies back.
+      float s_q = 1.f, s_vmax = 1.f;
+      if constexpr (kFp8) {
+        s_q = __ldg(a.q_scale + head);
+        s_vmax = 0.f;
+        for (int c = 0; c < a.n_vis; ++c)
+          s_vmax = fmaxf(s_vmax, chunk_scale(a.v_scale, a.vcur_scale, vis_slot(a, c), a.H, head));
+        if (!(s_vmax > 0.f)) s_vmax = 1.f;
+      }
       float m_ref = -INFINITY, l_sum = 0.f;
       for (int j = j0; j < j1; ++j, ++g) {
         int slot, row0;
         kv_tile_coords(a, j, slot, row0);
         const int valid = min(kBN, a.L - row0);
+        float sl2 = a.scale_log2, pf = 1.f;
+        if constexpr (kFp8) {
+          sl2 *= s_q * chunk_scale(a.k_scale, a.kcur_scale, slot, a.H, head);
+          pf = chunk_scale(a.v_scale, a.vcur_scale, slot, a.H, head) / s_vmax;
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], g & 1, abort_flag, budget));
         if (!ok) break;
         if (lane == 0 && (warp & 3) == 0) CCA_TRACE_EV(10 + 10 * wg, g);
@@ -480,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_new = need ? m_tile : m_ref;
         const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
         // p = 2^(x * scale_log2 - m_new), packed f32x2 FMAs, 4 packed partial sums,
-        // bf16 pairs stored to TMEM over the first 64 columns of S, 16 at a time.
+        // 16-bit pairs stored to TMEM over the first 64 columns of S, 16 at a time.
         const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_new, -m_new);
         uint64_t sums[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -498,14 +649,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               e1 = ex2_approx(e1);
             }
             sums[c & 3] = f2_add(sums[c & 3], f2_pack(e0, e1));
-            p16[c] = pack_bf16x2(e0, e1);
+            if constexpr (kFp8)
+              p16[c] = pack_f16x2(e0 * pf, e1 * pf);
+            else
+              p16[c] = pack_bf16x2(e0, e1);
           }
           tmem_st16(tS + q4 * 16, p16);
         }
-        float s_lo, s_hi, t_lo, t_hi;
+        float s_lo, s_hi;
         f2_unpack(f2_add(f2_add(sums[0], sums[1]), f2_add(sums[2], sums[3])), s_lo, s_hi);
-        (void)t_lo;
-        (void)t_hi;
         l_sum = l_sum * alpha + (s_lo + s_hi);
         m_ref = m_new;
         // Rescale this row of O when the reference maximum moved (O of the
@@ -533,8 +685,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int row = pair * (kNQ * kBM) + wg * kBM + r;
       const bool row_ok = row < n_q;
-      if (a.n_splits == 1) {
-        const float inv = 1.f / l_sum;
+      if (sg.slot < 0) {
+        const float inv = s_vmax / l_sum;
         __nv_bfloat16 *dst = a.out + (static_cast<int64_t>(row) * a.H + head) * D;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -555,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        const int64_t prow = (static_cast<int64_t>(split) * a.n_q_max + row) * a.H + head;
+        const int64_t prow = static_cast<int64_t>(sg.slot) * (kNQ * kBM) + wg * kBM + r;
         float *dst = a.ws_o + prow * D;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -565,7 +717,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (row_ok) {
             uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) d4[v] = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+            for (int v = 0; v < 8; ++v)
+              d4[v] = make_uint4(__float_as_uint(__uint_as_float(o[4 * v]) * s_vmax),
+                                 __float_as_uint(__uint_as_float(o[4 * v + 1]) * s_vmax),
+                                 __float_as_uint(__uint_as_float(o[4 * v + 2]) * s_vmax),
+                                 __float_as_uint(__uint_as_float(o[4 * v + 3]) * s_vmax));
           }
         }
         if (row_ok) *reinterpret_cast<float2 *>(a.ws_ml + prow * 2) = make_float2(m_ref, l_sum);
@@ -587,36 +743,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && *abort_flag && a.dev_status) atomicExch(a.dev_status, CCA_DEV_TIMEOUT);
 }
 
-// out[row][h] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s ; one warp per (row, head).
+// Merge of the partial segments of the split items: one warp per (item, row),
+// out[row][head] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s over the CTAs
+// whose KV range meets the item.  The schedule is recomputed from n_q exactly as
+// the attention kernel (launched with G CTAs) computed it.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restrict__ ws_o,
                                                            const float *__restrict__ ws_ml,
                                                            const int32_t *__restrict__ n_q_dev, int n_q_max, int H,
-                                                           int n_splits, __nv_bfloat16 *__restrict__ out) {
+                                                           int n_kv, int G, __nv_bfloat16 *__restrict__ out) {
   const int n_q = n_q_dev ? min(max(*n_q_dev, 0), n_q_max) : n_q_max;
-  const int64_t n_rows = static_cast<int64_t>(n_q) * H;
+  const Sched sch = make_sched(n_q, H, n_kv, G);
+  if (sch.r == 0) return;
   const int lane = threadIdx.x & 31;
+  const int64_t n_work = static_cast<int64_t>(sch.r) * (kNQ * kBM);
   const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t split_stride = static_cast<int64_t>(n_q_max) * H;
-  for (int64_t rh = w0; rh < n_rows; rh += nw) {
+  for (int64_t w = w0; w < n_work; w += nw) {
+    const int ur = static_cast<int>(w / (kNQ * kBM)), rr = static_cast<int>(w % (kNQ * kBM));
+    const int u = sch.q * G + ur, pair = u / H, head = u % H;
+    const int row = pair * (kNQ * kBM) + rr;
+    if (row >= n_q) continue;
+    const int64_t t0 = static_cast<int64_t>(ur) * n_kv, t1 = t0 + n_kv;  // the item's tiles in the list
+    int c_lo = static_cast<int>(t0 * G / sch.tr) - 1;
+    int c_hi = static_cast<int>((t1 * G + sch.tr - 1) / sch.tr) + 1;
+    c_lo = c_lo < 0 ? 0 : c_lo;
+    c_hi = c_hi > G - 1 ? G - 1 : c_hi;
     float mmax = -INFINITY;
-    for (int s = 0; s < n_splits; ++s) mmax = fmaxf(mmax, ws_ml[(s * split_stride + rh) * 2]);
+    for (int c = c_lo; c <= c_hi; ++c) {
+      const int64_t lo = static_cast<int64_t>(c) * sch.tr / G, hi = static_cast<int64_t>(c + 1) * sch.tr / G;
+      if (lo >= hi || hi <= t0 || lo >= t1) continue;
+      const int slot = 2 * c + (lo / n_kv == ur ? 0 : 1);
+      mmax = fmaxf(mmax, ws_ml[(static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2]);
+    }
     float den = 0.f;
     float acc[D / 32];
 #pragma unroll
     for (int k = 0; k < D / 32; ++k) acc[k] = 0.f;
-    for (int s = 0; s < n_splits; ++s) {
-      const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + (s * split_stride + rh) * 2);
-      const float w = exp2f(ml.x - mmax);
-      den += w * ml.y;
-      const float *o = ws_o + (s * split_stride + rh) * D;
+    for (int c = c_lo; c <= c_hi; ++c) {
+      const int64_t lo = static_cast<int64_t>(c) * sch.tr / G, hi = static_cast<int64_t>(c + 1) * sch.tr / G;
+      if (lo >= hi || hi <= t0 || lo >= t1) continue;
+      const int64_t prow = static_cast<int64_t>(2 * c + (lo / n_kv == ur ? 0 : 1)) * (kNQ * kBM) + rr;
+      const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + prow * 2);
+      const float wgt = exp2f(ml.x - mmax);
+      den += wgt * ml.y;
+      const float *o = ws_o + prow * D;
 #pragma unroll
-      for (int k = 0; k < D / 32; ++k) acc[k] += w * o[k * 32 + lane];
+      for (int k = 0; k < D / 32; ++k) acc[k] += wgt * o[k * 32 + lane];
     }
     const float inv = 1.f / den;
+    __nv_bfloat16 *dst = out + (static_cast<int64_t>(row) * H + head) * D;
 #pragma unroll
-    for (int k = 0; k < D / 32; ++k) out[rh * D + k * 32 + lane] = __float2bfloat16_rn(acc[k] * inv);
+    for (int k = 0; k < D / 32; ++k) dst[k * 32 + lane] = __float2bfloat16_rn(acc[k] * inv);
   }
 }
 
@@ -654,7 +832,7 @@ static cca_status make_tmap(CUtensorMap *tm, const void *ptr, CUtensorMapDataTyp
 }
 
 struct AttnPlan {
-  int n_pairs, n_splits, n_items, grid, tiles_per_chunk, n_kv_tiles, n_vis;
+  int grid, tiles_per_chunk, n_kv_tiles, n_vis, max_items;
   int32_t slots[kMaxVis];
 };
 
@@ -663,64 +841,57 @@ static int env_int(const char *name, int dflt) {
   return s && *s ? std::atoi(s) : dflt;
 }
 
+// Grid: one persistent CTA per SM (CCA_ATTN_CTAS overrides), never more CTAs
+// than KV tiles of work.
 static void plan_attention(const cca_kv_ring *ring, int n_q_max, AttnPlan &p) {
   const cca_kv_ring_desc &d = ring->d;
   p.n_vis = ring_visible(ring, p.slots, nullptr) + 1;  // cached chunks + the current chunk
   p.tiles_per_chunk = (d.chunk_len + kBN - 1) / kBN;
   p.n_kv_tiles = p.n_vis * p.tiles_per_chunk;
-  p.n_pairs = (n_q_max + kNQ * kBM - 1) / (kNQ * kBM);
-  const int sms = num_sms();
-  const int base = p.n_pairs * d.n_heads;
-  // Choose the KV split that minimises (waves x tiles per item); splits cost a
-  // combine pass, so prefer fewer on ties.  CCA_ATTN_SPLITS overrides.
-  int best = 1;
-  double best_cost = 1e30;
-  for (int s = 1; s <= 8 && s <= p.n_kv_tiles; ++s) {
-    const int items = base * s;
-    const int waves = (items + sms - 1) / sms;
-    const double cost = waves * std::ceil(static_cast<double>(p.n_kv_tiles) / s) * 1.0 + (s > 1 ? 2.0 : 0.0);
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = s;
-    }
-  }
-  const int forced = env_int("CCA_ATTN_SPLITS", 0);
-  if (forced > 0) best = forced < p.n_kv_tiles ? forced : p.n_kv_tiles;
-  p.n_splits = best;
-  p.n_items = base * p.n_splits;
-  p.grid = p.n_items < sms ? p.n_items : sms;
+  p.max_items = ((n_q_max + kNQ * kBM - 1) / (kNQ * kBM)) * d.n_heads;
+  int g = env_int("CCA_ATTN_CTAS", 0);
+  if (g <= 0) g = num_sms();
+  const int64_t work = static_cast<int64_t>(p.max_items) * p.n_kv_tiles;
+  if (work < g) g = static_cast<int>(work > 0 ? work : 1);
+  p.grid = g;
 }
 
+// Partial-segment slots: 2 per CTA, 256 rows each.
 static size_t workspace_bytes_for(const cca_kv_ring *ring, int n_q_max, const AttnPlan &p) {
-  if (p.n_splits <= 1) return 0;
-  const size_t rows = static_cast<size_t>(p.n_splits) * n_q_max * ring->d.n_heads;
+  if (n_q_max == 0) return 0;
+  const size_t rows = static_cast<size_t>(2) * p.grid * (kNQ * kBM);
   return rows * (static_cast<size_t>(ring->d.head_dim) + 2) * sizeof(float) + 256;
 }
 
-template <int D>
-static cca_status launch_bf16(const cca_kv_ring *ring, const AttnPlan &p, const AttnArgs &args, const void *q,
+template <int D, bool kFp8>
+static cca_status launch_attn(const cca_kv_ring *ring, const AttnPlan &p, const AttnArgs &args, const void *q,
                               const void *k_cur, const void *v_cur, cudaStream_t st) {
-  using S = AttnSmem<D>;
+  using S = AttnSmem<D, kFp8>;
   const cca_kv_ring_desc &d = ring->d;
+  const CUtensorMapDataType dt = kFp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int es = kFp8 ? 1 : 2;
   CUtensorMap tq, tkr, tvr, tkc, tvc;
   std::memset(&tq, 0, sizeof(tq));
-  if (!args.q_idx) CCA_TRY(make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, args.n_q_max, 0));
-  CCA_TRY(make_tmap(&tkr, d.k_slots, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, d.chunk_len, 1 + d.window));
-  CCA_TRY(make_tmap(&tvr, d.v_slots, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, d.chunk_len, 1 + d.window));
-  CCA_TRY(make_tmap(&tkc, k_cur, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, d.chunk_len, 0));
-  CCA_TRY(make_tmap(&tvc, v_cur, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, d.n_heads, d.chunk_len, 0));
-  cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (!args.q_idx) CCA_TRY(make_tmap(&tq, q, dt, es, D, d.n_heads, args.n_q_max, 0));
+  CCA_TRY(make_tmap(&tkr, d.k_slots, dt, es, D, d.n_heads, d.chunk_len, 1 + d.window));
+  CCA_TRY(make_tmap(&tvr, d.v_slots, dt, es, D, d.n_heads, d.chunk_len, 1 + d.window));
+  CCA_TRY(make_tmap(&tkc, k_cur, dt, es, D, d.n_heads, d.chunk_len, 0));
+  CCA_TRY(make_tmap(&tvc, v_cur, dt, es, D, d.n_heads, d.chunk_len, 0));
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(S::kAlloc));
   if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "cca_chunk_attn: %s", cudaGetErrorString(e));
-  attn_bf16_kernel<D><<<p.grid, kThreads, S::kAlloc, st>>>(tq, tkr, tvr, tkc, tvc, args);
-  CCA_TRY(launched("attn_bf16_kernel"));
-  if (p.n_splits > 1) {
-    const int64_t warps = static_cast<int64_t>(args.n_q_max) * d.n_heads;
+  attn_kernel<D, kFp8><<<p.grid, kThreads, S::kAlloc, st>>>(tq, tkr, tvr, tkc, tvc, args);
+  CCA_TRY(launched("attn_kernel"));
+  // Split items exist unless the item count is known on the host and divides
+  // evenly over the grid.
+  const bool maybe_split = args.n_q_dev != nullptr || (p.max_items % p.grid) != 0;
+  if (maybe_split) {
+    const int64_t warps = static_cast<int64_t>(p.grid) * (kNQ * kBM);
     int64_t blocks = (warps + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
     attn_combine_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        args.ws_o, args.ws_ml, args.n_q_dev, args.n_q_max, d.n_heads, p.n_splits, args.out);
+        args.ws_o, args.ws_ml, args.n_q_dev, args.n_q_max, d.n_heads, p.n_kv_tiles, p.grid, args.out);
     CCA_TRY(launched("attn_combine_kernel"));
   }
   return CCA_OK;
@@ -769,10 +940,14 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q, const void *k_
   if (d.dtype == CCA_E4M3) {
     if (!q_scale || !kcur_scale || !vcur_scale)
       return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: E4M3 ring needs q/kcur/vcur scales");
-    return fail(CCA_ERR_UNSUPPORTED, "cca_chunk_attn: E4M3 attention is not built yet");
-  }
-  if (q_scale || kcur_scale || vcur_scale)
+    const uintptr_t m = reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(kcur_scale) |
+                        reinterpret_cast<uintptr_t>(vcur_scale);
+    if (m & 3) return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: scales must be 4-byte aligned");
+    if (d.head_dim != 128)
+      return fail(CCA_ERR_UNSUPPORTED, "cca_chunk_attn: E4M3 attention is built for head_dim 128");
+  } else if (q_scale || kcur_scale || vcur_scale) {
     return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: BF16 ring takes no scales");
+  }
   if ((q_idx && (reinterpret_cast<uintptr_t>(q_idx) & 3)) || (n_q_dev && (reinterpret_cast<uintptr_t>(n_q_dev) & 3)))
     return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: q_idx / n_q_dev must be 4-byte aligned");
   AttnPlan p;
@@ -782,24 +957,26 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q, const void *k_
     return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: workspace of %zu bytes (16-byte aligned) required", need);
   AttnArgs args;
   std::memset(&args, 0, sizeof(args));
-  args.q = static_cast<const __nv_bfloat16 *>(q);
+  args.q = q;
+  args.q_scale = q_scale;
+  args.kcur_scale = kcur_scale;
+  args.vcur_scale = vcur_scale;
+  args.k_scale = d.k_scale;
+  args.v_scale = d.v_scale;
   args.q_idx = q_idx;
   args.n_q_dev = n_q_dev;
   args.out = static_cast<__nv_bfloat16 *>(out);
   if (need > 0) {
     args.ws_o = static_cast<float *>(workspace);
-    const size_t rows = static_cast<size_t>(p.n_splits) * n_q_max * d.n_heads;
+    const size_t rows = static_cast<size_t>(2) * p.grid * (kNQ * kBM);
     args.ws_ml = args.ws_o + rows * d.head_dim;
   }
   args.dev_status = d.dev_status;
   args.n_q_max = n_q_max;
   args.L = d.chunk_len;
   args.H = d.n_heads;
-  args.n_pairs = p.n_pairs;
-  args.n_splits = p.n_splits;
   args.tiles_per_chunk = p.tiles_per_chunk;
   args.n_kv_tiles = p.n_kv_tiles;
-  args.n_items = p.n_items;
   const double scale = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(d.head_dim));
   args.scale_log2 = static_cast<float>(scale * 1.4426950408889634);  // scale * log2(e)
   args.wait_budget = static_cast<long long>(env_int("CCA_WAIT_BUDGET_MCYCLES", 4000)) * 1000000LL;
@@ -807,8 +984,9 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q, const void *k_
   args.slots_packed = 0;
   for (int c = 0; c + 1 < p.n_vis; ++c) args.slots_packed |= static_cast<uint64_t>(p.slots[c] & 15) << (4 * c);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (d.head_dim == 128) return launch_bf16<128>(ring, p, args, q, k_cur, v_cur, st);
-  return launch_bf16<64>(ring, p, args, q, k_cur, v_cur, st);
+  if (d.dtype == CCA_E4M3) return launch_attn<128, true>(ring, p, args, q, k_cur, v_cur, st);
+  if (d.head_dim == 128) return launch_attn<128, false>(ring, p, args, q, k_cur, v_cur, st);
+  return launch_attn<64, false>(ring, p, args, q, k_cur, v_cur, st);
 }
 
 }  // extern "C"

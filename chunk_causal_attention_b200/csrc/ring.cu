@@ -70,29 +70,46 @@ size_t dtype_bytes(cca_dtype t) { return t == CCA_E4M3 ? 1 : (t == CCA_BF16 ? 2 
 
 // ------------------------------------------------------------------ kernels
 // bf16 (or fp32 -> bf16 RNE) copy of K and V into one ring slot; 16-byte
-// vectors, grid-stride, blockIdx.y selects K (0) or V (1).
+// vectors, blockIdx.y selects K (0) or V (1).  Each thread keeps 4 independent
+// loads in flight before its stores (streaming loads: the source is read once).
+__device__ __forceinline__ uint4 to_bf16x8(float4 a, float4 b) {
+  __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+  __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+  uint4 o;
+  o.x = *reinterpret_cast<uint32_t *>(&p0);
+  o.y = *reinterpret_cast<uint32_t *>(&p1);
+  o.z = *reinterpret_cast<uint32_t *>(&p2);
+  o.w = *reinterpret_cast<uint32_t *>(&p3);
+  return o;
+}
+
 template <bool kF32>
 __global__ void __launch_bounds__(256) append_bf16_kernel(const void *__restrict__ k_src,
                                                           const void *__restrict__ v_src,
                                                           uint4 *__restrict__ k_dst,
                                                           uint4 *__restrict__ v_dst, int64_t n_vec) {
+  constexpr int kU = 4;
   const void *src = blockIdx.y == 0 ? k_src : v_src;
   uint4 *dst = blockIdx.y == 0 ? k_dst : v_dst;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_vec; i += stride) {
-    if constexpr (!kF32) {
-      dst[i] = __ldcs(reinterpret_cast<const uint4 *>(src) + i);
-    } else {
-      const float4 a = __ldcs(reinterpret_cast<const float4 *>(src) + 2 * i);
-      const float4 b = __ldcs(reinterpret_cast<const float4 *>(src) + 2 * i + 1);
-      __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
-      __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
-      uint4 o;
-      o.x = *reinterpret_cast<uint32_t *>(&p0);
-      o.y = *reinterpret_cast<uint32_t *>(&p1);
-      o.z = *reinterpret_cast<uint32_t *>(&p2);
-      o.w = *reinterpret_cast<uint32_t *>(&p3);
-      dst[i] = o;
+  for (int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < n_vec; i0 += kU * stride) {
+    uint4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < n_vec) {
+        if constexpr (!kF32) {
+          v[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + i);
+        } else {
+          v[u] = to_bf16x8(__ldcs(reinterpret_cast<const float4 *>(src) + 2 * i),
+                           __ldcs(reinterpret_cast<const float4 *>(src) + 2 * i + 1));
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < n_vec) dst[i] = v[u];
     }
   }
 }
@@ -307,8 +324,8 @@ cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new
     uint4 *kd = reinterpret_cast<uint4 *>(static_cast<char *>(d.k_slots) + slot * n_elem * 2);
     uint4 *vd = reinterpret_cast<uint4 *>(static_cast<char *>(d.v_slots) + slot * n_elem * 2);
     const int64_t n_vec = n_elem / 8;
-    int64_t blocks = (n_vec + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
+    int64_t blocks = (n_vec + 4 * 256 - 1) / (4 * 256);
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 4;  // x2 tensors: 8 blocks of 256 per SM
     if (blocks > cap) blocks = cap;
     dim3 grid(static_cast<unsigned>(blocks), 2);
     if (src_dtype == CCA_F32)

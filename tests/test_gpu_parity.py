@@ -2,7 +2,10 @@
 
 Bars: bit-exact for the KV ring contents, e4m3 codes/scales, the mask,
 compaction indices and scatter; attention within max-abs 2e-2 and relative L2
-1e-2 (BF16) of the oracle run on the same bf16-rounded inputs.
+1e-2 (BF16) or 6e-2 / 3e-2 (e4m3) of the oracle run on the same inputs.  The
+output is bf16, so the max-abs bar is applied on top of the rounding to that
+format (half a bf16 ulp at the oracle's value): at |O| >= 16 that rounding alone
+is 0.0625, above the e4m3 bar, and no bf16 output could meet the bar without it.
 """
 
 import math
@@ -39,9 +42,22 @@ def err(got, ref):
     return float(np.abs(d).max()), float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-300))
 
 
+def half_ulp_bf16(x):
+    """Half a unit in the last place of bf16 at |x| (8-bit significand): the
+    rounding error any bf16 output of the exact value may carry."""
+    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    _, e = np.frexp(a)  # a = m 2^e, m in [0.5, 1)
+    return np.ldexp(1.0, e - 1 - 8)
+
+
 def assert_attn_close(got, ref, max_abs=BF16_MAX_ABS, rel_l2=BF16_REL_L2, what=""):
+    """Element-wise |got - ref| <= max_abs on top of the bf16 output rounding
+    (half an ulp of bf16 at |ref|), and relative L2 over the tensor <= rel_l2."""
+    got = np.asarray(got, dtype=np.float64)
+    d = np.abs(got - ref)
+    excess = float((d - half_ulp_bf16(ref)).max())
     ma, rl = err(got, ref)
-    assert ma <= max_abs and rl <= rel_l2, f"{what}: max_abs={ma:.3e} rel_l2={rl:.3e}"
+    assert excess <= max_abs and rl <= rel_l2, f"{what}: max_abs={ma:.3e} (beyond bf16 rounding {excess:.3e}) rel_l2={rl:.3e}"
     return ma, rl
 
 
@@ -246,13 +262,15 @@ def c1_ref(c1):
                                 v_cur=c1.v_cur[s]) for s in range(len(c1.q))]
 
 
-@pytest.mark.parametrize("splits", ["auto", "1", "3"])
-def test_attention_720p_two_steps(c1, c1_ring, c1_ref, splits, monkeypatch):
-    if splits != "auto":
-        monkeypatch.setenv("CCA_ATTN_SPLITS", splits)
+@pytest.mark.parametrize("ctas", ["auto", "37", "200"])
+def test_attention_720p_two_steps(c1, c1_ring, c1_ref, ctas, monkeypatch):
+    """Default grid (1 CTA per SM: 148 whole items + 20 split items), 37 CTAs
+    (4 full rounds + 20 split items), 200 CTAs (more CTAs than items: all split)."""
+    if ctas != "auto":
+        monkeypatch.setenv("CCA_ATTN_CTAS", ctas)
     for s in range(len(c1.q)):
         o = cca.cca_chunk_attn(c1_ring, bf(c1.q[s]), bf(c1.k_cur[s]), bf(c1.v_cur[s]))
-        assert_attn_close(to_np(o), c1_ref[s], what=f"720p step {s} splits={splits}")
+        assert_attn_close(to_np(o), c1_ref[s], what=f"720p step {s} ctas={ctas}")
     check_status(c1_ring)
 
 
@@ -350,3 +368,66 @@ def test_long_stream_ring_and_sampled_attention():
             for sl, c in zip(slots, ids):
                 assert torch.equal(ring.k_slots[sl].cpu(), synth.as_torch_bf16(oracle.get(c)[0]))
     check_status(ring)
+
+
+# ------------------------------------------------------------------ e4m3 attention (workload 3)
+def _fp8_stream_ref(ring_k, ring_v, q, kc, vc, t, window):
+    """Quantisation-aware oracle: every tensor quantised per head by the oracle's
+    own e4m3 encoder, attention in fp64 on the dequantised values."""
+    deq = lambda x: ofp8.dequantize_per_head(*ofp8.quantize_per_head(x))
+    past_k = {c: deq(ring_k[c]) for c in range(t)}
+    past_v = {c: deq(ring_v[c]) for c in range(t)}
+    return oca.chunk_attention(deq(q), past_k, past_v, t, window, k_cur=deq(kc), v_cur=deq(vc))
+
+
+def _fp8_call(ring, q, kc, vc, **kw):
+    q8, qs = cca.cca_quant_e4m3(bf(q))
+    k8, ks = cca.cca_quant_e4m3(bf(kc))
+    v8, vs = cca.cca_quant_e4m3(bf(vc))
+    return cca.cca_chunk_attn(ring, q8, k8, v8, q_scale=qs, kcur_scale=ks, vcur_scale=vs, **kw)
+
+
+@pytest.mark.parametrize("ctas", ["auto", "24"])
+def test_attention_fp8_720p(ctas, monkeypatch):
+    if ctas != "auto":
+        monkeypatch.setenv("CCA_ATTN_CTAS", ctas)
+    s = synth.fp8_720p()
+    ring = cca.KVRing(s.n_heads, s.head_dim, s.chunk_len, s.window, dtype="e4m3", device=dev())
+    for t in range(s.t):
+        ring.append(bf(s.ring_k[t]), bf(s.ring_v[t]))
+    for st in range(len(s.q)):
+        o = _fp8_call(ring, s.q[st], s.k_cur[st], s.v_cur[st])
+        ref = _fp8_stream_ref(s.ring_k, s.ring_v, s.q[st], s.k_cur[st], s.v_cur[st], s.t, s.window)
+        assert_attn_close(to_np(o), ref, FP8_MAX_ABS, FP8_REL_L2, what=f"fp8 720p step {st}")
+    check_status(ring)
+
+
+def test_attention_fp8_ragged_stream_with_eviction():
+    g = np.random.default_rng(31)
+    L, H, D, W, n = 200, 2, 128, 2, 6
+    draw = lambda: synth.bf16_round(g.standard_t(4.0, size=(L, H, D)).astype(np.float32))
+    q = [draw() for _ in range(n)]
+    k = [draw() for _ in range(n)]
+    v = [draw() for _ in range(n)]
+    ring = cca.KVRing(H, D, L, W, dtype="e4m3", device=dev())
+    for t in range(n):
+        o = _fp8_call(ring, q[t], k[t], v[t])
+        ref = _fp8_stream_ref(k, v, q[t], k[t], v[t], t, W)
+        assert_attn_close(to_np(o), ref, FP8_MAX_ABS, FP8_REL_L2, what=f"fp8 ragged t={t}")
+        ring.append(bf(k[t]), bf(v[t]))
+    check_status(ring)
+
+
+def test_attention_fp8_gathered_queries():
+    s = synth.fp8_720p(n_steps=1)
+    m = synth.mask_chunk()
+    ring = cca.KVRing(s.n_heads, s.head_dim, s.chunk_len, s.window, dtype="e4m3", device=dev())
+    for t in range(s.t):
+        ring.append(bf(s.ring_k[t]), bf(s.ring_v[t]))
+    mask_ref, _, _ = omask.token_mask(m.src, m.edit, prune_quantile=m.prune_quantile)
+    idx_ref, n_ref = omask.compact(mask_ref)
+    idx = torch.from_numpy(idx_ref).to(dev())
+    n = torch.tensor([n_ref], dtype=torch.int32, device=dev())
+    o = _fp8_call(ring, s.q[0], s.k_cur[0], s.v_cur[0], q_idx=idx, n_q_dev=n, n_q_max=s.chunk_len)
+    ref = _fp8_stream_ref(s.ring_k, s.ring_v, s.q[0], s.k_cur[0], s.v_cur[0], s.t, s.window)
+    assert_attn_close(to_np(o)[:n_ref], ref[idx_ref], FP8_MAX_ABS, FP8_REL_L2, what="fp8 gathered")

@@ -34,7 +34,7 @@ def _noalloc(ring, q, k, v, out, n_q_max):
 
 def test_noalloc_matches_allocating_entry_point_on_two_calls(monkeypatch):
     dev = torch.device("cuda:0")
-    monkeypatch.setenv("CCA_ATTN_SPLITS", "3")  # make the call use the scratch array
+    monkeypatch.delenv("CCA_ATTN_CTAS", raising=False)  # default grid: 20 of 168 items are split
     c1 = synth.chunk_720p()
     ring = cca.KVRing(c1.n_heads, c1.head_dim, c1.chunk_len, c1.window, device=dev)
     for t in range(c1.t):
@@ -58,7 +58,7 @@ def test_noalloc_matches_allocating_entry_point_on_two_calls(monkeypatch):
 
 def test_noalloc_refuses_calls_beyond_its_scratch(monkeypatch):
     dev = torch.device("cuda:0")
-    monkeypatch.setenv("CCA_ATTN_SPLITS", "8")  # 8 x 1620 x 24 x 130 x 4 B > 64 MiB
+    monkeypatch.setenv("CCA_ATTN_CTAS", "400")  # 2 x 400 slots x 256 rows x 130 x 4 B > 64 MiB
     c1 = synth.chunk_720p(n_steps=1, n_prefill=1)
     ring = cca.KVRing(c1.n_heads, c1.head_dim, c1.chunk_len, c1.window, device=dev)
     ring.append(synth.as_torch_bf16(c1.ring_k[0], dev), synth.as_torch_bf16(c1.ring_v[0], dev))
