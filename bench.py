@@ -53,6 +53,23 @@ def peaks():
         return 1590.0, 6650.0, "fallback"
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity with one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, flop_per_rank_step: float, ms_per_step_max: float) -> float:
+    """Whole-job TFLOP/s: work of all replicas over the slowest rank's time."""
+    return world * flop_per_rank_step / (ms_per_step_max * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
@@ -378,10 +395,7 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
         if int(r.ring.status.item()) != 0:
             raise RuntimeError(f"device status {int(r.ring.status.item())}")
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
 
     # ---- end to end through the public API with host buffers (pinned), rank-local
     e2e = None
@@ -414,21 +428,17 @@ def run_gpu(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
         h2d = CALLS_PER_STEP * 3 * L * H * D * 2
         d2h = CALLS_PER_STEP * L * H * D * 2
-        e2e = {"value": world * CALLS_PER_STEP * FLOP_PER_CALL / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_value(world, CALLS_PER_STEP * FLOP_PER_CALL, e2e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     if rank != 0:
         return
     peak_tf, _, peak_kind = peaks()
     ms_step = total_ms / args.steps
-    value = world * CALLS_PER_STEP * FLOP_PER_CALL / (ms_step * 1e-3) / 1e12
+    value = job_value(world, CALLS_PER_STEP * FLOP_PER_CALL, ms_step)
     attn_mean_ms = float(np.mean(attn_ms))
     achieved = FLOP_PER_CALL / (attn_mean_ms * 1e-3) / 1e12
     traffic = None

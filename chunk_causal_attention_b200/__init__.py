@@ -22,7 +22,8 @@ import torch
 __all__ = [
     "CCA_BF16", "CCA_E4M3", "CCA_F32", "CcaError", "KVRing", "lib", "lib_path", "EXPORTED",
     "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc",
-    "cca_token_mask_l2", "cca_compact", "cca_scatter", "cca_version", "cca_take_launch_count",
+    "cca_token_mask_l2", "cca_compact", "cca_scatter", "cca_selftest_bounded_wait", "cca_version",
+    "cca_take_launch_count",
 ]
 
 CCA_BF16, CCA_E4M3, CCA_F32 = 0, 1, 2
@@ -35,7 +36,7 @@ EXPORTED = (
     "cca_kv_ring_create", "cca_kv_ring_destroy", "cca_kv_ring_reset", "cca_kv_ring_query",
     "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn",
     "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_token_mask_l2", "cca_compact",
-    "cca_scatter", "cca_last_error", "cca_version", "cca_take_launch_count",
+    "cca_scatter", "cca_selftest_bounded_wait", "cca_last_error", "cca_version", "cca_take_launch_count",
 )
 
 
@@ -84,6 +85,7 @@ def lib() -> ctypes.CDLL:
         "cca_token_mask_l2": [vp, vp, i32, i32, f32, f32, vp, vp, vp, vp],
         "cca_compact": [vp, i32, vp, vp, vp],
         "cca_scatter": [vp, vp, vp, i32, i32, vp, vp],
+        "cca_selftest_bounded_wait": [vp, i64, i32, vp],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -325,6 +327,13 @@ def cca_scatter(o_compact: torch.Tensor, idx: torch.Tensor, n_active: torch.Tens
                              _ptr(n_active, "n_active", torch.int32), int(n_max), int(row_bytes),
                              _ptr(o_cache, "o_cache"), _stream(stream)), "cca_scatter")
     return o_cache
+
+
+def cca_selftest_bounded_wait(status: torch.Tensor, budget_cycles: int, arrive_first: bool = False,
+                              stream=None) -> None:
+    """Run the bounded-wait self-test; status (int32[1], device) gets CCA_DEV_*."""
+    _check(lib().cca_selftest_bounded_wait(_ptr(status, "status", torch.int32), int(budget_cycles),
+                                           1 if arrive_first else 0, _stream(stream)), "cca_selftest_bounded_wait")
 
 
 def default_scale(head_dim: int) -> float:

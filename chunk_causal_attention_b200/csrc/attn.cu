@@ -142,14 +142,14 @@ __device__ __forceinline__ int vis_slot(const AttnArgs &a, int c) {
 }
 
 // ---- work schedule (identical in every role, the combine kernel included)
-// Items are (query pair, head), pair-major, for the pairs holding the first n_q
-// queries.  With G CTAs: CTA c takes items c, c + G, ... for q = items / G full
+// Items are (query pair, head), head-major (so CTAs running together share a
+// head's K/V in L2), for the pairs holding the first n_q queries.  With G CTAs: CTA c takes items c, c + G, ... for q = items / G full
 // rounds; the r = items % G remaining items form a list of r * n_kv KV tiles cut
 // into G near-equal ranges, so CTA c also takes 0, 1 or 2 partial segments.
 // Partial segment k (0 or 1) of CTA c writes workspace slot 2c + k.
 struct Sched {
-  int n_items, q, r;
-  int64_t tr;  // KV tiles in the remainder list
+  int n_items, q, r, n_pairs;  // n_pairs: query pairs holding the first n_q queries
+  int64_t tr;                  // KV tiles in the remainder list
 };
 struct Seg {
   int pair, head, j0, j1, slot;  // slot < 0: whole item, direct output
@@ -157,17 +157,19 @@ struct Seg {
 
 __device__ __forceinline__ Sched make_sched(int n_q, int H, int n_kv, int G) {
   Sched s;
-  s.n_items = ((n_q + kNQ * kBM - 1) / (kNQ * kBM)) * H;
+  s.n_pairs = (n_q + kNQ * kBM - 1) / (kNQ * kBM);
+  s.n_items = s.n_pairs * H;
   s.q = s.n_items / G;
   s.r = s.n_items % G;
   s.tr = static_cast<int64_t>(s.r) * n_kv;
   return s;
 }
 
-__device__ __forceinline__ bool get_seg(const Sched &s, int H, int n_kv, int G, int c, int k, Seg &g) {
+__device__ __forceinline__ bool get_seg(const Sched &s, int n_kv, int G, int c, int k, Seg &g) {
+  const int P = s.n_pairs > 0 ? s.n_pairs : 1;
   if (k < s.q) {
     const int u = c + k * G;
-    g = {u / H, u % H, 0, n_kv, -1};
+    g = {u % P, u / P, 0, n_kv, -1};
     return true;
   }
   k -= s.q;
@@ -177,12 +179,12 @@ __device__ __forceinline__ bool get_seg(const Sched &s, int H, int n_kv, int G, 
   if (k == 0) {
     const int u = s.q * G + static_cast<int>(u0);
     const int64_t e0 = hi < (u0 + 1) * n_kv ? hi : (u0 + 1) * n_kv;
-    g = {u / H, u % H, static_cast<int>(lo - u0 * n_kv), static_cast<int>(e0 - u0 * n_kv), 2 * c};
+    g = {u % P, u / P, static_cast<int>(lo - u0 * n_kv), static_cast<int>(e0 - u0 * n_kv), 2 * c};
     return true;
   }
   if (hi <= (u0 + 1) * n_kv) return false;
   const int u = s.q * G + static_cast<int>(u0) + 1;
-  g = {u / H, u % H, 0, static_cast<int>(hi - (u0 + 1) * n_kv), 2 * c + 1};
+  g = {u % P, u / P, 0, static_cast<int>(hi - (u0 + 1) * n_kv), 2 * c + 1};
   return true;
 }
 
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
-      if (!get_seg(sch, a.H, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
       const int pair = sg.pair, head = sg.head, j0 = sg.j0, j1 = sg.j1;
       for (int i = 0; i < kNQ && ok; ++i) {
         if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[i], (it - 1) & 1, abort_flag, budget));
@@ -434,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
-      if (!get_seg(sch, a.H, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
       const int j0 = sg.j0, j1 = sg.j1;
       const int n = j1 - j0;
       ok = wait(&q_full[0], it & 1) && wait(&q_full[1], it & 1);
@@ -503,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int kseg = 0; ok; ++kseg) {
         Seg sg;
-        if (!get_seg(sch, a.H, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+        if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
         const int j0 = sg.j0, j1 = sg.j1;
         for (int j = j0; j < j1; ++j, ++g) {
           const uint32_t stage = g % kNS, ph = (g / kNS) & 1;
@@ -561,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
-      if (!get_seg(sch, a.H, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
       const int pair = sg.pair, head = sg.head, j0 = sg.j0, j1 = sg.j1;
       // e4m3: scores carry the factor s_q * s_k(chunk); V's factor s_v(chunk) is
       // folded into P relative to the largest s_v of the visible chunks, which
@@ -746,7 +748,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Merge of the partial segments of the split items: one warp per (item, row),
 // out[row][head] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s over the CTAs
 // whose KV range meets the item.  The schedule is recomputed from n_q exactly as
-// the attention kernel (launched with G CTAs) computed it.
+// the attention kernel (launched with G CTAs) computed it.  Lane i examines
+// candidate CTA c_lo + i; the found partials are then summed by the whole warp.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restrict__ ws_o,
                                                            const float *__restrict__ ws_ml,
@@ -756,41 +759,60 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restri
   const Sched sch = make_sched(n_q, H, n_kv, G);
   if (sch.r == 0) return;
   const int lane = threadIdx.x & 31;
-  const int64_t n_work = static_cast<int64_t>(sch.r) * (kNQ * kBM);
-  const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t w = w0; w < n_work; w += nw) {
-    const int ur = static_cast<int>(w / (kNQ * kBM)), rr = static_cast<int>(w % (kNQ * kBM));
-    const int u = sch.q * G + ur, pair = u / H, head = u % H;
+  const uint32_t tr = static_cast<uint32_t>(sch.tr), uG = static_cast<uint32_t>(G);
+  const int n_work = sch.r * (kNQ * kBM);
+  const int w0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int w = w0; w < n_work; w += nw) {
+    const int ur = w / (kNQ * kBM), rr = w % (kNQ * kBM);
+    const int u = sch.q * G + ur, pair = u % sch.n_pairs, head = u / sch.n_pairs;
     const int row = pair * (kNQ * kBM) + rr;
     if (row >= n_q) continue;
-    const int64_t t0 = static_cast<int64_t>(ur) * n_kv, t1 = t0 + n_kv;  // the item's tiles in the list
-    int c_lo = static_cast<int>(t0 * G / sch.tr) - 1;
-    int c_hi = static_cast<int>((t1 * G + sch.tr - 1) / sch.tr) + 1;
-    c_lo = c_lo < 0 ? 0 : c_lo;
-    c_hi = c_hi > G - 1 ? G - 1 : c_hi;
+    const uint32_t t0 = static_cast<uint32_t>(ur) * n_kv, t1 = t0 + n_kv;  // the item's tiles in the list
+    // Covering CTAs: from the first c with hi_c > t0 to at most ceil(t1 G / tr);
+    // lanes examine 32 candidates at a time.
+    const int c_first = static_cast<int>(((t0 + 1) * uG + tr - 1) / tr) - 1;
+    const int c_last = min(G - 1, static_cast<int>((t1 * uG + tr - 1) / tr));
+    auto probe = [&](int c, int &slot) {
+      if (c > c_last) return false;
+      const uint32_t lo = static_cast<uint32_t>(c) * tr / uG, hi = static_cast<uint32_t>(c + 1) * tr / uG;
+      slot = 2 * c + (lo / n_kv == static_cast<uint32_t>(ur) ? 0 : 1);
+      return lo < hi && hi > t0 && lo < t1;
+    };
     float mmax = -INFINITY;
-    for (int c = c_lo; c <= c_hi; ++c) {
-      const int64_t lo = static_cast<int64_t>(c) * sch.tr / G, hi = static_cast<int64_t>(c + 1) * sch.tr / G;
-      if (lo >= hi || hi <= t0 || lo >= t1) continue;
-      const int slot = 2 * c + (lo / n_kv == ur ? 0 : 1);
-      mmax = fmaxf(mmax, ws_ml[(static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2]);
+    for (int cb = c_first; cb <= c_last; cb += 32) {
+      int slot;
+      if (probe(cb + lane, slot))
+        mmax = fmaxf(mmax, ws_ml[(static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2]);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
     float den = 0.f;
     float acc[D / 32];
 #pragma unroll
     for (int k = 0; k < D / 32; ++k) acc[k] = 0.f;
-    for (int c = c_lo; c <= c_hi; ++c) {
-      const int64_t lo = static_cast<int64_t>(c) * sch.tr / G, hi = static_cast<int64_t>(c + 1) * sch.tr / G;
-      if (lo >= hi || hi <= t0 || lo >= t1) continue;
-      const int64_t prow = static_cast<int64_t>(2 * c + (lo / n_kv == ur ? 0 : 1)) * (kNQ * kBM) + rr;
-      const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + prow * 2);
-      const float wgt = exp2f(ml.x - mmax);
-      den += wgt * ml.y;
-      const float *o = ws_o + prow * D;
+    for (int cb = c_first; cb <= c_last; cb += 32) {
+      int slot = 0;
+      const bool mine = probe(cb + lane, slot);
+      float wgt = 0.f;
+      if (mine) {
+        const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + (static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2);
+        wgt = exp2f(ml.x - mmax);
+        den += wgt * ml.y;
+      }
+      unsigned todo = __ballot_sync(0xffffffffu, mine);
+      while (todo) {
+        const int src = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const float ws = __shfl_sync(0xffffffffu, wgt, src);
+        const int sl = __shfl_sync(0xffffffffu, slot, src);
+        const float *o = ws_o + (static_cast<int64_t>(sl) * (kNQ * kBM) + rr) * D;
 #pragma unroll
-      for (int k = 0; k < D / 32; ++k) acc[k] += wgt * o[k * 32 + lane];
+        for (int k = 0; k < D / 32; ++k) acc[k] += ws * o[k * 32 + lane];
+      }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     const float inv = 1.f / den;
     __nv_bfloat16 *dst = out + (static_cast<int64_t>(row) * H + head) * D;
 #pragma unroll

@@ -246,6 +246,15 @@ cca_status cca_scatter(const void *o_compact, const int32_t *idx,
 /* Diagnostics                                                               */
 /* ------------------------------------------------------------------------ */
 
+/* Self-test of the device-side bounded wait used by every kernel here: one
+ * thread waits on an mbarrier phase that nothing completes (arrive_first = 0)
+ * or that it completed itself (arrive_first != 0, a positive control), giving
+ * up after budget_cycles SM clock cycles (1 .. 4e9).  *dev_status (device int32)
+ * receives CCA_DEV_TIMEOUT or CCA_DEV_OK; the context stays usable either way.
+ * No counterpart on the pages: it backs the library's failure reporting. */
+cca_status cca_selftest_bounded_wait(int32_t *dev_status, int64_t budget_cycles,
+                                     int32_t arrive_first, cca_stream_t stream);
+
 /* Message describing the last error of the calling thread ("" if none). */
 const char *cca_last_error(void);
 
