@@ -13,7 +13,8 @@
 //  * one work item = two 128-row Q tiles (256 queries) of one head x a range
 //    of 128-row KV tiles; both Q tiles share every K/V tile loaded into shared
 //    memory, halving L2->SM traffic per FLOP;
-//  * warp 0 = TMA producer (Q once per item, K/V per tile, 2-stage ring);
+//  * warp 0 = TMA producer of Q (once per item) and K (3-stage ring); warp 2 =
+//    TMA producer of V (2 stages); warp 3 = e4m3 V expander;
 //    warp 1 = TMEM allocator and the single thread issuing tcgen05.mma;
 //    warps 4-7 / 8-11 = softmax warpgroups, one per Q tile, one row per thread;
 //  * TMEM (512 columns): S0 | S1 | O0 | O1.  S = Q K^T lands in TMEM; the
@@ -49,16 +50,23 @@ namespace cca {
 constexpr int kBM = 128;       // query rows per Q tile (TMEM lanes)
 constexpr int kBN = 128;       // key rows per KV tile
 constexpr int kNQ = 2;         // Q tiles per work item
-constexpr int kNS = 2;         // K and V pipeline stages
+constexpr int kNSK = 3;        // K pipeline stages
+constexpr int kNSV = 2;        // V pipeline stages
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kMaxVis = kMaxWindow + 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
 // Pairs of score columns whose exponential runs on the FMA pipe (polynomial)
-// instead of the MUFU unit: bit k set = pair k of every 8 pairs (3 of 8 here).
+// instead of the MUFU unit: bit k set = pair k of every 8 pairs (2 of 8 here).
 #ifndef CCA_EMU_MASK
-#define CCA_EMU_MASK 0xE0
+#define CCA_EMU_MASK 0xC0
 #endif
 constexpr unsigned kEmuMask = CCA_EMU_MASK;
+// Exponentials: 0 = fp32 MUFU ex2 (+ FMA-pipe polynomial on kEmuMask pairs);
+// 1 = packed fp16 MUFU ex2 (two results per instruction).
+#ifndef CCA_EXP_MODE
+#define CCA_EXP_MODE 0
+#endif
+constexpr int kExpMode = CCA_EXP_MODE;
 #ifndef CCA_SETMAXNREG
 #define CCA_SETMAXNREG 1
 #endif
@@ -122,10 +130,10 @@ struct AttnSmem {
   static constexpr uint32_t kV16Tile = kFp8 ? 128 * D * 2 : 0;
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + kNQ * kTile;
-  static constexpr uint32_t kV = kK + kNS * kTile;
-  static constexpr uint32_t kV16 = kV + kNS * kTile;
-  static constexpr uint32_t kBar = kV16 + kNS * kV16Tile;
-  static constexpr uint32_t kNumBars = 4 + 6 * kNS + 8 + 1;
+  static constexpr uint32_t kV = kK + kNSK * kTile;
+  static constexpr uint32_t kV16 = kV + kNSV * kTile;
+  static constexpr uint32_t kBar = kV16 + kNSV * kV16Tile;
+  static constexpr uint32_t kNumBars = 4 + 2 * kNSK + 4 * kNSV + 8 + 1;
   static constexpr uint32_t kBytes = kBar + kNumBars * 8 + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
@@ -209,13 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + S::kBar);
   uint64_t *q_full = bars;              // [kNQ]  producer -> MMA
   uint64_t *q_empty = bars + 2;         // [kNQ]  MMA -> producer
-  uint64_t *k_full = bars + 4;          // [kNS]
-  uint64_t *k_empty = k_full + kNS;     // [kNS]
-  uint64_t *v_full = k_empty + kNS;     // [kNS]  V tile landed
-  uint64_t *v_empty = v_full + kNS;     // [kNS]  V tile consumed (MMA, or the e4m3 expanders)
-  uint64_t *v16_full = v_empty + kNS;   // [kNS]  e4m3: fp16 V ready
-  uint64_t *v16_empty = v16_full + kNS; // [kNS]  e4m3: fp16 V consumed by the MMAs
-  uint64_t *s_full = v16_empty + kNS;   // [2] MMA -> softmax: S ready
+  uint64_t *k_full = bars + 4;           // [kNSK]
+  uint64_t *k_empty = k_full + kNSK;     // [kNSK]
+  uint64_t *v_full = k_empty + kNSK;     // [kNSV] V tile landed
+  uint64_t *v_empty = v_full + kNSV;     // [kNSV] V tile consumed (MMA, or the e4m3 expander)
+  uint64_t *v16_full = v_empty + kNSV;   // [kNSV] e4m3: fp16 V ready
+  uint64_t *v16_empty = v16_full + kNSV; // [kNSV] e4m3: fp16 V consumed by the MMAs
+  uint64_t *s_full = v16_empty + kNSV;   // [2] MMA -> softmax: S ready
   uint64_t *p_full = s_full + 2;        // [2] softmax -> MMA: P ready (and O rescaled)
   uint64_t *o_full = p_full + 2;        // [2] MMA -> softmax: O final for the item
   uint64_t *o_empty = o_full + 2;       // [2] softmax -> MMA: O read out
@@ -236,12 +244,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_full[i], 1);
       mbar_init(&o_empty[i], kBM / 32);
     }
-    for (int s = 0; s < kNS; ++s) {
+    for (int s = 0; s < kNSK; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kNSV; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], kFp8 ? 2 : 1);  // e4m3: released by the two expander warps
-      mbar_init(&v16_full[s], 2);
+      mbar_init(&v_empty[s], 1);  // released by the MMA (bf16) or the e4m3 expander warp
+      mbar_init(&v16_full[s], 1);
       mbar_init(&v16_empty[s], 1);
     }
     mbar_init(drain, 1);
@@ -271,7 +281,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     CCA_TRACE_ROLE(0);
     uint32_t g = 0;   // KV tiles handled by this CTA
     uint32_t gk = 0;  // K tile loads armed
-    uint32_t gv = 0;  // V tile loads armed
     int it = 0;       // items handled by this CTA
     int q_armed = 0;  // Q phases armed (per tile, identical for both)
     bool ok = true;
@@ -331,10 +340,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       q_armed = it + 1;
       for (int j = j0; j < j1; ++j, ++g) {
-        const uint32_t stage = g % kNS, ph = (g / kNS) & 1;
+        const uint32_t stage = g % kNSK, ph = (g / kNSK) & 1;
         int slot, row0;
         kv_tile_coords(a, j, slot, row0);
-        if (g >= kNS) ok = __all_sync(0xffffffffu, mbar_wait(&k_empty[stage], ph ^ 1, abort_flag, budget));
+        if (g >= kNSK) ok = __all_sync(0xffffffffu, mbar_wait(&k_empty[stage], ph ^ 1, abort_flag, budget));
         if (!ok) break;
         ++gk;
         if (lane == 0) {
@@ -348,32 +357,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_4d(&tm_kr, &k_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
           }
         }
-        if (g >= kNS) ok = __all_sync(0xffffffffu, mbar_wait(&v_empty[stage], ph ^ 1, abort_flag, budget));
-        if (!ok) break;
-        ++gv;
-        if (lane == 0) {
-          const uint32_t dst = base + S::kV + stage * S::kTile;
-          mbar_arrive_expect_tx(&v_full[stage], S::kTile);
-          for (uint32_t b = 0; b < S::kNBox; ++b) {
-            if (slot < 0)
-              tma_load_3d(&tm_vc, &v_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0);
-            else
-              tma_load_4d(&tm_vr, &v_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
-          }
-        }
       }
       ++it;
     }
     // Drain: wait (bounded) for the most recent armed phase of every barrier the
     // TMA may still complete, so no copy lands in shared memory after exit.
     if (lane == 0) {
-      for (uint32_t k = 0; k < kNS && k < gk; ++k) {
+      for (uint32_t k = 0; k < kNSK && k < gk; ++k) {
         const uint32_t gg = gk - 1 - k;
-        mbar_drain(&k_full[gg % kNS], (gg / kNS) & 1, budget);
-      }
-      for (uint32_t k = 0; k < kNS && k < gv; ++k) {
-        const uint32_t gg = gv - 1 - k;
-        mbar_drain(&v_full[gg % kNS], (gg / kNS) & 1, budget);
+        mbar_drain(&k_full[gg % kNSK], (gg / kNSK) & 1, budget);
       }
       if (q_armed > 0)
         for (int i = 0; i < kNQ; ++i) mbar_drain(&q_full[i], (q_armed - 1) & 1, budget);
@@ -399,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kVStageBytes = kFp8 ? S::kV16Tile : S::kTile;
     uint64_t *pv_full = kFp8 ? v16_full : v_full;
     uint64_t *pv_empty = kFp8 ? v16_empty : v_empty;
-    auto issue_qk = [&](int i, uint32_t stage) {
+    auto issue_qk = [=](int i, uint32_t stage) {
       const uint64_t qa = dQ0 + ((i * S::kTile) >> 4), kb = dK0 + ((stage * S::kTile) >> 4);
       const uint32_t d = tm + i * 128u;
       if (elect_one()) {
@@ -414,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    auto issue_pv = [&](int i, uint32_t stage, bool acc) {
+    auto issue_pv = [=](int i, uint32_t stage, bool acc) {
       const uint64_t vb = dV0 + ((stage * kVStageBytes) >> 4);
       const uint32_t d = tm + 256u + i * D, pa = tm + i * 128u;
       if (elect_one()) {
@@ -424,11 +416,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    auto commit = [&](uint64_t *bar) {
+    auto commit = [](uint64_t *bar) {
       if (elect_one()) mma_commit(bar);
       __syncwarp();
     };
-    auto wait = [&](uint64_t *bar, uint32_t parity) {
+    auto wait = [=](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, budget));
     };
     uint32_t g = 0;
@@ -440,18 +432,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j0 = sg.j0, j1 = sg.j1;
       const int n = j1 - j0;
       ok = wait(&q_full[0], it & 1) && wait(&q_full[1], it & 1);
+      // K of the segment's first tile; later K tiles are waited for one tile
+      // ahead (after QK1), while the softmax still runs, so that PV0(g) and
+      // QK0(g+1) go to the tensor core back to back.
+      ok = ok && wait(&k_full[g % kNSK], (g / kNSK) & 1);
       if (!ok) break;
       tc_fence_after();
       for (int jj = 0; jj < n && ok; ++jj, ++g) {
-        const uint32_t stage = g % kNS, ph = (g / kNS) & 1;
-        if (!(ok = wait(&k_full[stage], ph))) break;
+        const uint32_t stage = g % kNSK;
+        const uint32_t vst = g % kNSV, vph = (g / kNSV) & 1;
         if (lane == 0) CCA_TRACE_EV(1, g);
         tc_fence_after();
         issue_qk(0, stage);
         commit(&s_full[0]);
         if (lane == 0) CCA_TRACE_EV(2, g);
         if (jj > 0) {  // O1 += P1 V for the previous tile
-          const uint32_t pst = (g - 1) % kNS;
+          const uint32_t pst = (g - 1) % kNSV;
           if (jj == 1 && it > 0 && !(ok = wait(&o_empty[1], (it - 1) & 1))) break;
           if (!(ok = wait(&p_full[1], (g - 1) & 1))) break;
           if (lane == 0) CCA_TRACE_EV(3, g - 1);
@@ -466,19 +462,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (jj == n - 1) {
           commit(&q_empty[0]);
           commit(&q_empty[1]);
+        } else {
+          if (lane == 0) CCA_TRACE_EV(7, g + 1);
+          if (!(ok = wait(&k_full[(g + 1) % kNSK], ((g + 1) / kNSK) & 1))) break;
         }
-        if (!(ok = wait(&pv_full[stage], ph))) break;
+        if (!(ok = wait(&pv_full[vst], vph))) break;
+        if (lane == 0) CCA_TRACE_EV(8, g);
         if (jj == 0 && it > 0 && !(ok = wait(&o_empty[0], (it - 1) & 1))) break;
         if (!(ok = wait(&p_full[0], g & 1))) break;
         if (lane == 0) CCA_TRACE_EV(5, g);
         tc_fence_after();
-        issue_pv(0, stage, jj > 0);
+        issue_pv(0, vst, jj > 0);
         if (lane == 0) CCA_TRACE_EV(6, g);
         if (jj == n - 1) commit(&o_full[0]);
       }
       if (!ok) break;
       {  // O1 += P1 V for the last tile
-        const uint32_t pst = (g - 1) % kNS;
+        const uint32_t pst = (g - 1) % kNSV;
         if (n == 1 && it > 0 && !(ok = wait(&o_empty[1], (it - 1) & 1))) break;
         if (!(ok = wait(&p_full[1], (g - 1) & 1))) break;
         tc_fence_after();
@@ -493,29 +493,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_drain(drain, 0, budget);
     __syncwarp();
   }
-  // ================================================================ e4m3 V expanders
-  else if (warp < 4) {
+  // ================================================================ V producer
+  else if (warp == 2) {
+    if (kUseSetMaxNReg) regs_dec<88>();
+    // V tiles run on their own warp so a V slot that frees late (after the PV
+    // MMAs) never holds back the next K loads.
+    uint32_t g = 0, gv = 0;
+    bool ok = true;
+    for (int kseg = 0; ok; ++kseg) {
+      Seg sg;
+      if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      for (int j = sg.j0; j < sg.j1; ++j, ++g) {
+        const uint32_t stage = g % kNSV, ph = (g / kNSV) & 1;
+        int slot, row0;
+        kv_tile_coords(a, j, slot, row0);
+        if (g >= kNSV) ok = __all_sync(0xffffffffu, mbar_wait(&v_empty[stage], ph ^ 1, abort_flag, budget));
+        if (!ok) break;
+        ++gv;
+        if (lane == 0) {
+          const uint32_t dst = base + S::kV + stage * S::kTile;
+          mbar_arrive_expect_tx(&v_full[stage], S::kTile);
+          for (uint32_t b = 0; b < S::kNBox; ++b) {
+            if (slot < 0)
+              tma_load_3d(&tm_vc, &v_full[stage], dst + b * S::kBox, b * kBoxElems, sg.head, row0);
+            else
+              tma_load_4d(&tm_vr, &v_full[stage], dst + b * S::kBox, b * kBoxElems, sg.head, row0, slot);
+          }
+        }
+      }
+    }
+    if (lane == 0)
+      for (uint32_t k = 0; k < kNSV && k < gv; ++k) {
+        const uint32_t gg = gv - 1 - k;
+        mbar_drain(&v_full[gg % kNSV], (gg / kNSV) & 1, budget);
+      }
+  }
+  // ================================================================ e4m3 V expander
+  else if (warp == 3) {
     if (kUseSetMaxNReg) regs_dec<88>();
     if constexpr (kFp8) {
-      // Warps 2-3 turn each landed e4m3 V tile (128 rows x 128 bytes, swizzled)
-      // into an fp16 tile (two 128 x 64 boxes, swizzled) for the PV MMA.  The
-      // conversion is exact: every e4m3 value is an fp16 value.
-      const int t = threadIdx.x - 64;  // 0..63
+      // Turns each landed e4m3 V tile (128 rows x 128 bytes, swizzled) into an
+      // fp16 tile (two 128 x 64 boxes, swizzled) for the PV MMA.  The conversion
+      // is exact: every e4m3 value is an fp16 value.
       uint32_t g = 0;
       bool ok = true;
       for (int kseg = 0; ok; ++kseg) {
         Seg sg;
         if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
-        const int j0 = sg.j0, j1 = sg.j1;
-        for (int j = j0; j < j1; ++j, ++g) {
-          const uint32_t stage = g % kNS, ph = (g / kNS) & 1;
+        for (int j = sg.j0; j < sg.j1; ++j, ++g) {
+          const uint32_t stage = g % kNSV, ph = (g / kNSV) & 1;
           ok = __all_sync(0xffffffffu, mbar_wait(&v_full[stage], ph, abort_flag, budget));
-          if (ok && g >= kNS) ok = __all_sync(0xffffffffu, mbar_wait(&v16_empty[stage], ph ^ 1, abort_flag, budget));
+          if (ok && g >= kNSV) ok = __all_sync(0xffffffffu, mbar_wait(&v16_empty[stage], ph ^ 1, abort_flag, budget));
           if (!ok) break;
           const uint32_t src = base + S::kV + stage * S::kTile;
           const uint32_t dst = base + S::kV16 + stage * S::kV16Tile;
 #pragma unroll 4
-          for (int e = t; e < 128 * 8; e += 64) {  // 16-byte source chunks
+          for (int e = lane; e < 128 * 8; e += 32) {  // 16-byte source chunks
             const int r = e >> 3, c = e & 7;
             uint32_t w[4];
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -634,7 +667,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
         // p = 2^(x * scale_log2 - m_new), packed f32x2 FMAs, 4 packed partial sums,
         // 16-bit pairs stored to TMEM over the first 64 columns of S, 16 at a time.
-        const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_new, -m_new);
+        // e4m3 + packed fp16 ex2: the V-scale ratio pf enters as log2(pf) in the
+        // exponent, so the fp16 result is P itself; its sum is divided by pf.
+        const float m_off = (kFp8 && kExpMode == 1) ? m_new - __log2f(pf) : m_new;
+        const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_off, -m_off);
         uint64_t sums[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -644,23 +680,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int i = q4 * 32 + 2 * c;
             float e0, e1;
             f2_unpack(f2_fma(f2_pack(x[i], x[i + 1]), sl2_2, negm_2), e0, e1);
-            if ((kEmuMask >> (c & 7)) & 1) {
-              exp2_poly_pair(e0, e1);  // FMA pipe
+            if constexpr (kExpMode == 1) {
+              const uint32_t h = ex2_f16x2(e0, e1);  // MUFU, two per instruction
+              f16x2_to_f32(h, e0, e1);
+              sums[c & 3] = f2_add(sums[c & 3], f2_pack(e0, e1));
+              if constexpr (kFp8)
+                p16[c] = h;
+              else
+                p16[c] = pack_bf16x2(e0, e1);
             } else {
-              e0 = ex2_approx(e0);  // MUFU
-              e1 = ex2_approx(e1);
+              if ((kEmuMask >> (c & 7)) & 1) {
+                exp2_poly_pair(e0, e1);  // FMA pipe
+              } else {
+                e0 = ex2_approx(e0);  // MUFU
+                e1 = ex2_approx(e1);
+              }
+              sums[c & 3] = f2_add(sums[c & 3], f2_pack(e0, e1));
+              if constexpr (kFp8)
+                p16[c] = pack_f16x2(e0 * pf, e1 * pf);
+              else
+                p16[c] = pack_bf16x2(e0, e1);
             }
-            sums[c & 3] = f2_add(sums[c & 3], f2_pack(e0, e1));
-            if constexpr (kFp8)
-              p16[c] = pack_f16x2(e0 * pf, e1 * pf);
-            else
-              p16[c] = pack_bf16x2(e0, e1);
           }
           tmem_st16(tS + q4 * 16, p16);
         }
         float s_lo, s_hi;
         f2_unpack(f2_add(f2_add(sums[0], sums[1]), f2_add(sums[2], sums[3])), s_lo, s_hi);
-        l_sum = l_sum * alpha + (s_lo + s_hi);
+        const float tile_sum = (kFp8 && kExpMode == 1) ? (s_lo + s_hi) / pf : (s_lo + s_hi);
+        l_sum = l_sum * alpha + tile_sum;
         m_ref = m_new;
         // Rescale this row of O when the reference maximum moved (O of the
         // previous tile is complete: S of this tile was committed after it).
