@@ -22,7 +22,8 @@ import torch
 __all__ = [
     "CCA_BF16", "CCA_E4M3", "CCA_F32", "CcaError", "KVRing", "lib", "lib_path", "EXPORTED",
     "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc",
-    "cca_token_mask_l2", "cca_compact", "cca_scatter", "cca_selftest_bounded_wait", "cca_version",
+    "cca_token_mask_l2", "cca_compact", "cca_compact_workspace_size", "cca_scatter", "cca_selftest_bounded_wait",
+    "cca_version",
     "cca_take_launch_count",
 ]
 
@@ -36,6 +37,7 @@ EXPORTED = (
     "cca_kv_ring_create", "cca_kv_ring_destroy", "cca_kv_ring_reset", "cca_kv_ring_query",
     "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn",
     "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_token_mask_l2", "cca_compact",
+    "cca_compact_workspace_size",
     "cca_scatter", "cca_selftest_bounded_wait", "cca_last_error", "cca_version", "cca_take_launch_count",
 )
 
@@ -83,7 +85,8 @@ def lib() -> ctypes.CDLL:
         "cca_chunk_attn_workspace_size": [vp, i32, ctypes.POINTER(sz)],
         "cca_chunk_attn_noalloc": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp],
         "cca_token_mask_l2": [vp, vp, i32, i32, f32, f32, vp, vp, vp, vp],
-        "cca_compact": [vp, i32, vp, vp, vp],
+        "cca_compact": [vp, i32, vp, vp, vp, sz, vp],
+        "cca_compact_workspace_size": [i32, ctypes.POINTER(sz)],
         "cca_scatter": [vp, vp, vp, i32, i32, vp, vp],
         "cca_selftest_bounded_wait": [vp, i64, i32, vp],
     }
@@ -302,16 +305,27 @@ def cca_token_mask_l2(src: torch.Tensor, edit: torch.Tensor, tau: float = 0.0, p
     return mask
 
 
+def cca_compact_workspace_size(n_tok: int) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().cca_compact_workspace_size(int(n_tok), ctypes.byref(out)), "cca_compact_workspace_size")
+    return int(out.value)
+
+
 def cca_compact(mask: torch.Tensor, idx: Optional[torch.Tensor] = None, n_active: Optional[torch.Tensor] = None,
-                stream=None):
+                workspace: Optional[torch.Tensor] = None, stream=None):
     """Ascending active positions (int32 [n_tok], first n valid) and the count (device int32[1])."""
     n = mask.shape[0]
     if idx is None:
         idx = torch.empty(max(n, 1), dtype=torch.int32, device=mask.device)
     if n_active is None:
         n_active = torch.empty(1, dtype=torch.int32, device=mask.device)
+    need = cca_compact_workspace_size(n)
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=mask.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().cca_compact(_ptr(mask, "mask", torch.uint8), n, _ptr(idx, "idx", torch.int32),
-                             _ptr(n_active, "n_active", torch.int32), _stream(stream)), "cca_compact")
+                             _ptr(n_active, "n_active", torch.int32), _ptr(workspace, "workspace"), ws_bytes,
+                             _stream(stream)), "cca_compact")
     return idx, n_active
 
 

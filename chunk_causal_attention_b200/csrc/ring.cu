@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "ring.cuh"
+#include "sm100.cuh"
 
 namespace cca {
 
@@ -83,35 +84,117 @@ __device__ __forceinline__ uint4 to_bf16x8(float4 a, float4 b) {
   return o;
 }
 
+// Each thread keeps kAppendUnroll 16-byte outputs' worth of loads in flight and
+// the grid is at most one wave (4 blocks of 256 per SM at 64 registers), so a
+// 720p chunk (2 x 9.95 MB, 486 blocks) is copied in a single round of loads.
+constexpr int kAppendUnroll = 10;
+constexpr int64_t kMaxChunkElems = int64_t(1) << 33;  // keeps 16-byte vector indices below 2^30
+constexpr int kAppendUnrollF32 = 4;  // fp32 sources: two 16-byte loads per output
+
 template <bool kF32>
-__global__ void __launch_bounds__(256) append_bf16_kernel(const void *__restrict__ k_src,
-                                                          const void *__restrict__ v_src,
-                                                          uint4 *__restrict__ k_dst,
-                                                          uint4 *__restrict__ v_dst, int64_t n_vec) {
-  constexpr int kU = 4;
+__global__ void __launch_bounds__(256, 4) append_bf16_kernel(const void *__restrict__ k_src,
+                                                             const void *__restrict__ v_src,
+                                                             uint4 *__restrict__ k_dst,
+                                                             uint4 *__restrict__ v_dst, int n_vec) {
+  constexpr int kU = kF32 ? kAppendUnrollF32 : kAppendUnroll;
   const void *src = blockIdx.y == 0 ? k_src : v_src;
   uint4 *dst = blockIdx.y == 0 ? k_dst : v_dst;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < n_vec; i0 += kU * stride) {
+  const int stride = gridDim.x * blockDim.x;  // n_vec < 2^31 is checked on the host
+  for (int i0 = blockIdx.x * blockDim.x + threadIdx.x; i0 < n_vec; i0 += kU * stride) {
     uint4 v[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int64_t i = i0 + u * stride;
-      if (i < n_vec) {
+      const unsigned i = static_cast<unsigned>(i0) + static_cast<unsigned>(u * stride);
+      if (i < static_cast<unsigned>(n_vec)) {
         if constexpr (!kF32) {
           v[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + i);
         } else {
-          v[u] = to_bf16x8(__ldcs(reinterpret_cast<const float4 *>(src) + 2 * i),
-                           __ldcs(reinterpret_cast<const float4 *>(src) + 2 * i + 1));
+          v[u] = to_bf16x8(__ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i)),
+                           __ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i) + 1));
         }
       }
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int64_t i = i0 + u * stride;
-      if (i < n_vec) dst[i] = v[u];
+      const unsigned i = static_cast<unsigned>(i0) + static_cast<unsigned>(u * stride);
+      if (i < static_cast<unsigned>(n_vec)) dst[i] = v[u];
     }
   }
+}
+
+// BF16 -> BF16 append as a TMA bulk copy: one CTA per SM, one thread issuing
+// 16 KB global->shared bulk loads (completion on an mbarrier) and shared->global
+// bulk stores from a 12-stage ring of shared memory (192 KB).  A 720p chunk is
+// 2 x 9.95 MB = 1215 pieces, about 8 per CTA, so every load is in flight at
+// once.  A stage is refilled once the store that read it has finished reading
+// (bulk_group accounting, kBulkLag stores may still be reading).  Waits are
+// bounded: on expiry the ring's status word gets CCA_DEV_TIMEOUT, the CTA waits
+// (bounded) for the loads it issued and for its stores, and returns.
+constexpr int kBulkPiece = 16384;
+__host__ __device__ inline int64_t cca_min64(int64_t a, int64_t b) { return a < b ? a : b; }
+constexpr int kBulkStages = 12;
+constexpr int kBulkLag = 4;
+constexpr long long kBulkBudget = 2000000000LL;  // clock64 cycles, about 1 s
+
+__global__ void __launch_bounds__(32, 1) append_bulk_kernel(const uint8_t *__restrict__ k_src,
+                                                           const uint8_t *__restrict__ v_src, uint8_t *k_dst,
+                                                           uint8_t *v_dst, int64_t bytes, int32_t *dev_status) {
+  extern __shared__ __align__(128) uint8_t stage_mem[];
+  __shared__ uint64_t bar[kBulkStages];
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  const int64_t per_tensor = (bytes + kBulkPiece - 1) / kBulkPiece;
+  const int64_t n_pieces = 2 * per_tensor;
+  const int64_t n_mine = (n_pieces - blockIdx.x + gridDim.x - 1) / gridDim.x;  // pieces c, c + G, ...
+  for (int s = 0; s < kBulkStages; ++s) sm100::mbar_init(&bar[s], 1);
+  abort_flag = 0;
+  sm100::fence_mbar_init();
+  const uint32_t base = smem_u32(stage_mem);
+  auto piece = [&](int64_t i, const uint8_t *&src, uint8_t *&dst, uint32_t &len) {
+    const int64_t j = blockIdx.x + i * gridDim.x;
+    const bool v = j >= per_tensor;
+    const int64_t off = (v ? j - per_tensor : j) * kBulkPiece;
+    src = (v ? v_src : k_src) + off;
+    dst = (v ? v_dst : k_dst) + off;
+    len = static_cast<uint32_t>(cca_min64(kBulkPiece, bytes - off));
+  };
+  auto issue_load = [&](int64_t i) {
+    const uint8_t *src;
+    uint8_t *dst;
+    uint32_t len;
+    piece(i, src, dst, len);
+    const int s = static_cast<int>(i % kBulkStages);
+    sm100::mbar_arrive_expect_tx(&bar[s], len);
+    sm100::bulk_load(base + s * kBulkPiece, src, len, &bar[s]);
+  };
+  int64_t issued = 0, done = 0;
+  for (; issued < n_mine && issued < kBulkStages; ++issued) issue_load(issued);
+  bool ok = true;
+  for (int64_t i = 0; i < n_mine; ++i) {
+    const int s = static_cast<int>(i % kBulkStages);
+    if (!sm100::mbar_wait(&bar[s], static_cast<uint32_t>((i / kBulkStages) & 1), &abort_flag, kBulkBudget)) {
+      ok = false;
+      break;
+    }
+    done = i + 1;
+    const uint8_t *src;
+    uint8_t *dst;
+    uint32_t len;
+    piece(i, src, dst, len);
+    sm100::bulk_store(dst, base + s * kBulkPiece, len);
+    sm100::bulk_commit();
+    const int64_t r = i + 1 - kBulkLag;  // its store has finished reading after the wait below
+    if (r >= 0 && r + kBulkStages < n_mine) {
+      asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kBulkLag - 1) : "memory");
+      issue_load(issued++);
+    }
+  }
+  if (!ok) {
+    for (int64_t i = done; i < issued; ++i)
+      sm100::mbar_drain(&bar[i % kBulkStages], static_cast<uint32_t>((i / kBulkStages) & 1), kBulkBudget);
+    if (dev_status) *dev_status = CCA_DEV_TIMEOUT;
+  }
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Loads 8 consecutive elements (16 B of bf16, 32 B of fp32) as floats.
@@ -221,6 +304,21 @@ __global__ void finalize_scale_kernel(unsigned *a, unsigned *b, int n) {
   }
 }
 
+static cca_status bulk_copy_pair(const uint8_t *k_src, const uint8_t *v_src, uint8_t *k_dst, uint8_t *v_dst,
+                                 int64_t bytes, int32_t *dev_status, cudaStream_t st) {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(append_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kBulkStages * kBulkPiece);
+  });
+  if (attr_err != cudaSuccess) return fail(CCA_ERR_CUDA, "append: %s", cudaGetErrorString(attr_err));
+  const int64_t n_pieces = 2 * ((bytes + kBulkPiece - 1) / kBulkPiece);
+  const int grid = static_cast<int>(cca_min64(num_sms(), n_pieces));
+  append_bulk_kernel<<<grid, 32, kBulkStages * kBulkPiece, st>>>(k_src, v_src, k_dst, v_dst, bytes, dev_status);
+  return launched("append_bulk_kernel");
+}
+
 // Quantise one or two [n_tok][H][D] tensors; scale arrays are [H] each.
 static cca_status quantize_pair(const void *x0, const void *x1, cca_dtype src, int n_tok, int H, int D,
                                 uint8_t *y0, uint8_t *y1, float *s0, float *s1, cudaStream_t st) {
@@ -262,6 +360,8 @@ cca_status cca_kv_ring_create(const cca_kv_ring_desc *desc, cca_kv_ring **out) {
     return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: need H >= 1, L >= 1, 0 <= W <= %d", kMaxWindow);
   if (d.head_dim != 64 && d.head_dim != 128)
     return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: head_dim must be 64 or 128 (got %d)", d.head_dim);
+  if (static_cast<int64_t>(d.chunk_len) * d.n_heads * d.head_dim > kMaxChunkElems)
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: L * H * D must be <= 2^33");
   if (d.dtype != CCA_BF16 && d.dtype != CCA_E4M3)
     return fail(CCA_ERR_INVALID_ARG, "cca_kv_ring_create: dtype must be CCA_BF16 or CCA_E4M3");
   if (!d.k_slots || !d.v_slots || !aligned16(d.k_slots) || !aligned16(d.v_slots))
@@ -324,15 +424,19 @@ cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new
     uint4 *kd = reinterpret_cast<uint4 *>(static_cast<char *>(d.k_slots) + slot * n_elem * 2);
     uint4 *vd = reinterpret_cast<uint4 *>(static_cast<char *>(d.v_slots) + slot * n_elem * 2);
     const int64_t n_vec = n_elem / 8;
-    int64_t blocks = (n_vec + 4 * 256 - 1) / (4 * 256);
-    const int64_t cap = static_cast<int64_t>(num_sms()) * 4;  // x2 tensors: 8 blocks of 256 per SM
+    const int64_t per_block = (src_dtype == CCA_F32 ? kAppendUnrollF32 : kAppendUnroll) * 256;
+    int64_t blocks = (n_vec + per_block - 1) / per_block;
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 2;  // x2 tensors: 4 blocks of 256 per SM
     if (blocks > cap) blocks = cap;
     dim3 grid(static_cast<unsigned>(blocks), 2);
-    if (src_dtype == CCA_F32)
-      append_bf16_kernel<true><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, n_vec);
-    else
-      append_bf16_kernel<false><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, n_vec);
-    CCA_TRY(launched("append_bf16_kernel"));
+    if (src_dtype == CCA_F32) {
+      append_bf16_kernel<true><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, static_cast<int>(n_vec));
+      CCA_TRY(launched("append_bf16_kernel"));
+    } else {
+      CCA_TRY(bulk_copy_pair(static_cast<const uint8_t *>(k_new), static_cast<const uint8_t *>(v_new),
+                             reinterpret_cast<uint8_t *>(kd), reinterpret_cast<uint8_t *>(vd), n_elem * 2,
+                             d.dev_status, st));
+    }
   } else {
     uint8_t *kd = static_cast<uint8_t *>(d.k_slots) + slot * n_elem;
     uint8_t *vd = static_cast<uint8_t *>(d.v_slots) + slot * n_elem;

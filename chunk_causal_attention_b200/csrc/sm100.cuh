@@ -78,6 +78,22 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, long 
   }
 }
 
+// ------------------------------------------------------------------ bulk copies (untiled, no multicast)
+// global -> shared, completion counted in bytes on an mbarrier; both addresses
+// 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_smem),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+// shared -> global in the thread's current bulk group.
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_smem), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
 // One lane of the (converged) warp returns true.
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;

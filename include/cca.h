@@ -81,7 +81,7 @@ typedef struct cca_kv_ring cca_kv_ring; /* opaque host-side handle */
 typedef struct cca_kv_ring_desc {
   int32_t n_heads;    /* H >= 1                                                  */
   int32_t head_dim;   /* D: 64 or 128                                            */
-  int32_t chunk_len;  /* L >= 1 tokens per chunk                                 */
+  int32_t chunk_len;  /* L >= 1 tokens per chunk; L * H * D <= 2^33            */
   int32_t window;     /* W >= 0 most recent non-sink chunks kept                 */
   cca_dtype dtype;    /* CCA_BF16 or CCA_E4M3                                    */
   void *k_slots;      /* device, [(1+W)][L][H][D] elements of dtype              */
@@ -228,10 +228,21 @@ cca_status cca_token_mask_l2(const float *src, const float *edit, int32_t n_tok,
 
 /* idx[0 .. n) = ascending positions u with mask[u] != 0; *n_active_dev = n.
  *  mask: device uint8 [n_tok]; idx: device int32 [n_tok] (entries >= n are not
- *  written); n_active_dev: device int32.  n_tok <= 2^20.
+ *  written); n_active_dev: device int32.
+ *  0 <= n_tok <= 2^30.  n_tok <= 16384: one CTA, workspace may be NULL.
+ *  Larger n_tok: one cooperative launch of co-resident CTAs (count, offset of
+ *  each CTA's run from the totals of the runs before it, write), which needs
+ *  a 16-byte aligned device workspace of cca_compact_workspace_size bytes
+ *  (contents need not be initialised; not shared by concurrent calls).  If
+ *  one of its bounded device-side waits runs out, *n_active_dev is set to -1
+ *  and idx is not valid.
  * Errors: CCA_ERR_INVALID_ARG, CCA_ERR_CUDA. */
 cca_status cca_compact(const uint8_t *mask, int32_t n_tok, int32_t *idx,
-                       int32_t *n_active_dev, cca_stream_t stream);
+                       int32_t *n_active_dev, void *workspace,
+                       size_t workspace_bytes, cca_stream_t stream);
+
+/* Bytes of workspace cca_compact needs for n_tok tokens (0 up to 16384). */
+cca_status cca_compact_workspace_size(int32_t n_tok, size_t *bytes);
 
 /* o_cache row idx[i] <- o_compact row i for i < *n_active_dev; every other row
  * of o_cache is left untouched (it keeps the output cached at chunk k-1).

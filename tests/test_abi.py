@@ -127,8 +127,14 @@ def test_call_validation_without_device_work(L):
     assert L.cca_token_mask_l2(vp(0x1000), vp(0x1000), 10, 16, 1.0, 1.5, vp(0x1000), None, None, None) == 1
     assert L.cca_token_mask_l2(vp(0x1000), vp(0x1000), 40000, 16, 1.0, 0.7, vp(0x1000), None, None, None) == 1
     assert L.cca_token_mask_l2(vp(0x1000), vp(0x1000), 10, 16, -1.0, -1.0, vp(0x1000), None, None, None) == 1
-    assert L.cca_compact(vp(0x1000), -1, vp(0x1000), vp(0x1000), None) == 1
-    assert L.cca_compact(vp(0x1000), 10, vp(0x1000), None, None) == 1
+    assert L.cca_compact(vp(0x1000), -1, vp(0x1000), vp(0x1000), None, 0, None) == 1
+    assert L.cca_compact(vp(0x1000), 10, vp(0x1000), None, None, 0, None) == 1
+    assert L.cca_compact(vp(0x1000), 100000, vp(0x1000), vp(0x1000), None, 0, None) == 1  # needs a workspace
+    sz = ctypes.c_size_t()
+    assert L.cca_compact_workspace_size(16384, ctypes.byref(sz)) == 0 and sz.value == 0
+    assert L.cca_compact_workspace_size(16385, ctypes.byref(sz)) == 0 and sz.value == 4096 * 8 + 16
+    assert L.cca_compact(vp(0x1000), 16385, vp(0x1000), vp(0x1000), vp(0x1000), 4096 * 8, None) == 1  # too small
+    assert L.cca_compact(vp(0x1000), (1 << 30) + 1, vp(0x1000), vp(0x1000), vp(0x1000), 1 << 30, None) == 1
     assert L.cca_scatter(vp(0x1000), vp(0x1000), vp(0x1000), 4, 20, vp(0x1000), None) == 1
     assert L.cca_scatter(None, None, None, 0, 16, None, None) == 0
     assert L.cca_quant_e4m3(vp(0x1000), cca.CCA_BF16, 4, 2, 80, vp(0x1000), vp(0x1000), None) == 1

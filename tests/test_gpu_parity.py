@@ -159,6 +159,28 @@ def test_mask_identical_latents_all_inactive():
     assert mask.sum().item() == 0 and n.item() == 0
 
 
+@pytest.mark.parametrize("n_tok", [1, 2, 255, 256, 1620, 4097, 32768])
+@pytest.mark.parametrize("q", [0.01, 0.5, 0.7, 1.0])
+def test_mask_dynamic_tau_with_ties(n_tok, q):
+    """Integer-valued latents make every d^2 an exact small integer in both
+    precisions, with many ties at the threshold: the kernel's order statistic
+    and strict-greater mask must equal the oracle's exactly (ties at tau stay
+    inactive; q = 1 leaves every token inactive)."""
+    g = np.random.default_rng(1000 + n_tok)
+    src = np.zeros((n_tok, 16), dtype=np.float32)
+    edit = g.integers(0, 3, size=(n_tok, 16)).astype(np.float32) * (g.random((n_tok, 1)) < 0.8)
+    q32 = float(np.float32(q))  # the kernel receives q as fp32
+    m_ref, _, tau = omask.token_mask(src, edit, prune_quantile=q32)
+    tau_out = torch.empty(1, dtype=torch.float32, device=dev())
+    mask = cca.cca_token_mask_l2(torch.from_numpy(src).to(dev()), torch.from_numpy(edit).to(dev()),
+                                 prune_quantile=q32, tau_out=tau_out)
+    torch.cuda.synchronize()
+    assert np.array_equal(mask.cpu().numpy(), m_ref)
+    assert tau_out.item() == np.float32(tau)
+    if q == 1.0:
+        assert m_ref.sum() == 0
+
+
 def test_mask_dynamic_tau_and_compaction_bit_exact():
     m = synth.mask_chunk()
     m_ref, d_ref, tau = omask.token_mask(m.src, m.edit, prune_quantile=m.prune_quantile)
@@ -177,14 +199,43 @@ def test_mask_dynamic_tau_and_compaction_bit_exact():
     assert abs(tau_out.item() - tau) <= 1e-5 * tau
 
 
-@pytest.mark.parametrize("n_tok,p", [(1, 0.5), (17, 0.3), (16384, 0.05), (16385, 0.9), (100000, 0.3)])
+@pytest.mark.parametrize("n_tok,p", [(1, 0.5), (17, 0.3), (16384, 0.05), (16385, 0.9), (65536, 0.3),
+                                     (65537, 0.3), (100000, 0.3), (8192 * 37 + 5, 0.5), (8192 * 1000, 0.0),
+                                     (8192 * 1000 + 1, 1.0), ((1 << 22) + 3, 0.01), ((1 << 26) + 17, 0.3)])
 def test_compaction_ragged_sizes(n_tok, p):
+    """Both paths (one CTA up to 65536 tokens, look-back scan above) against the
+    oracle on small sizes and against the closed form flatnonzero on all."""
     g = np.random.default_rng(n_tok)
     m = (g.random(n_tok) < p).astype(np.uint8)
+    mt = torch.from_numpy(m).to(dev())
+    idx, n = cca.cca_compact(mt)
+    torch.cuda.synchronize()
+    want = np.flatnonzero(m).astype(np.int32)
+    assert n.item() == want.shape[0]
+    assert np.array_equal(idx[:n.item()].cpu().numpy(), want)
+    if n_tok <= 200000:
+        ref_idx, ref_n = omask.compact(m)
+        assert ref_n == n.item() and np.array_equal(ref_idx, want)
+    # a second call reuses the same workspace: its status words are re-zeroed
+    ws = torch.full((max(cca.cca_compact_workspace_size(n_tok), 16),), 0xFF, dtype=torch.uint8, device=dev())
+    idx2, n2 = cca.cca_compact(mt, workspace=ws)
+    idx3, n3 = cca.cca_compact(mt, workspace=ws)
+    torch.cuda.synchronize()
+    assert n2.item() == n3.item() == want.shape[0]
+    assert torch.equal(idx2[:n2.item()], idx[:n.item()]) and torch.equal(idx3[:n3.item()], idx[:n.item()])
+
+
+@pytest.mark.parametrize("n_tok", [1000, 16385, 300007])
+def test_compaction_counts_any_nonzero_byte(n_tok):
+    """A token is active when its mask byte is nonzero, whatever the value."""
+    g = np.random.default_rng(7 + n_tok)
+    m = g.choice(np.array([0, 1, 2, 17, 128, 255], dtype=np.uint8), size=n_tok, p=[0.6, 0.1, 0.1, 0.1, 0.05, 0.05])
     idx, n = cca.cca_compact(torch.from_numpy(m).to(dev()))
     torch.cuda.synchronize()
-    assert n.item() == int(m.sum())
-    assert np.array_equal(idx[:n.item()].cpu().numpy(), np.flatnonzero(m).astype(np.int32))
+    want = np.flatnonzero(m).astype(np.int32)
+    ref_idx, ref_n = omask.compact(m)
+    assert ref_n == n.item() == want.shape[0]
+    assert np.array_equal(idx[:n.item()].cpu().numpy(), ref_idx)
 
 
 def test_scatter_keeps_inactive_rows():
