@@ -13,8 +13,9 @@
 //  * one work item = two 128-row Q tiles (256 queries) of one head x a range
 //    of 128-row KV tiles; both Q tiles share every K/V tile loaded into shared
 //    memory, halving L2->SM traffic per FLOP;
-//  * warp 0 = TMA producer of Q (once per item) and K (3-stage ring); warp 2 =
-//    TMA producer of V (2 stages); warp 3 = e4m3 V expander;
+//  * warp 0 = TMA producer of Q (once per item) and K (3-stage ring); bf16:
+//    warp 2 = TMA producer of V (2 stages), warp 3 idle; e4m3: warp 0 loads V
+//    too and warps 2-3 expand each e4m3 V tile to fp16 (64 rows each);
 //    warp 1 = TMEM allocator and the single thread issuing tcgen05.mma;
 //    warps 4-7 / 8-11 = softmax warpgroups, one per Q tile, one row per thread;
 //  * TMEM (512 columns): S0 | S1 | O0 | O1.  S = Q K^T lands in TMEM; the
@@ -250,8 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kNSV; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);  // released by the MMA (bf16) or the e4m3 expander warp
-      mbar_init(&v16_full[s], 1);
+      mbar_init(&v_empty[s], kFp8 ? 2 : 1);  // released by the MMA (bf16) or both e4m3 expander warps
+      mbar_init(&v16_full[s], kFp8 ? 2 : 1);
       mbar_init(&v16_empty[s], 1);
     }
     mbar_init(drain, 1);
@@ -281,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     CCA_TRACE_ROLE(0);
     uint32_t g = 0;   // KV tiles handled by this CTA
     uint32_t gk = 0;  // K tile loads armed
+    uint32_t gvk = 0; // e4m3: V tile loads armed
     int it = 0;       // items handled by this CTA
     int q_armed = 0;  // Q phases armed (per tile, identical for both)
     bool ok = true;
@@ -357,6 +359,24 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_4d(&tm_kr, &k_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
           }
         }
+        if constexpr (kFp8) {
+          // e4m3: V tiles come from this warp too; the expanders free a V slot as
+          // soon as it is converted, so it never holds back the K loads for long.
+          const uint32_t vst = g % kNSV, vph = (g / kNSV) & 1;
+          if (g >= kNSV) ok = __all_sync(0xffffffffu, mbar_wait(&v_empty[vst], vph ^ 1, abort_flag, budget));
+          if (!ok) break;
+          ++gvk;
+          if (lane == 0) {
+            const uint32_t dst = base + S::kV + vst * S::kTile;
+            mbar_arrive_expect_tx(&v_full[vst], S::kTile);
+            for (uint32_t b = 0; b < S::kNBox; ++b) {
+              if (slot < 0)
+                tma_load_3d(&tm_vc, &v_full[vst], dst + b * S::kBox, b * kBoxElems, head, row0);
+              else
+                tma_load_4d(&tm_vr, &v_full[vst], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
+            }
+          }
+        }
       }
       ++it;
     }
@@ -369,6 +389,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (q_armed > 0)
         for (int i = 0; i < kNQ; ++i) mbar_drain(&q_full[i], (q_armed - 1) & 1, budget);
+      for (uint32_t k = 0; k < kNSV && k < gvk; ++k) {
+        const uint32_t gg = gvk - 1 - k;
+        mbar_drain(&v_full[gg % kNSV], (gg / kNSV) & 1, budget);
+      }
     }
   }
   // ================================================================ MMA issuer
@@ -494,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
   // ================================================================ V producer
-  else if (warp == 2) {
+  else if (warp == 2 && !kFp8) {
     if (kUseSetMaxNReg) regs_dec<88>();
     // V tiles run on their own warp so a V slot that frees late (after the PV
     // MMAs) never holds back the next K loads.
@@ -528,13 +552,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_drain(&v_full[gg % kNSV], (gg / kNSV) & 1, budget);
       }
   }
-  // ================================================================ e4m3 V expander
-  else if (warp == 3) {
+  // ================================================================ e4m3 V expanders
+  else if (warp < 4) {
     if (kUseSetMaxNReg) regs_dec<88>();
     if constexpr (kFp8) {
-      // Turns each landed e4m3 V tile (128 rows x 128 bytes, swizzled) into an
-      // fp16 tile (two 128 x 64 boxes, swizzled) for the PV MMA.  The conversion
-      // is exact: every e4m3 value is an fp16 value.
+      // Warps 2 and 3 turn each landed e4m3 V tile (128 rows x 128 bytes,
+      // swizzled) into an fp16 tile (two 128 x 64 boxes, swizzled) for the PV
+      // MMA, 64 rows each.  The conversion is exact: every e4m3 value is an
+      // fp16 value.
       uint32_t g = 0;
       bool ok = true;
       for (int kseg = 0; ok; ++kseg) {
@@ -548,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t src = base + S::kV + stage * S::kTile;
           const uint32_t dst = base + S::kV16 + stage * S::kV16Tile;
 #pragma unroll 4
-          for (int e = lane; e < 128 * 8; e += 32) {  // 16-byte source chunks
+          for (int e = (warp - 2) * 512 + lane; e < (warp - 1) * 512; e += 32) {  // 16-byte source chunks
             const int r = e >> 3, c = e & 7;
             uint32_t w[4];
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
