@@ -134,7 +134,7 @@ struct AttnSmem {
   static constexpr uint32_t kV = kK + kNSK * kTile;
   static constexpr uint32_t kV16 = kV + kNSV * kTile;
   static constexpr uint32_t kBar = kV16 + kNSV * kV16Tile;
-  static constexpr uint32_t kNumBars = 4 + 2 * kNSK + 4 * kNSV + 8 + 1;
+  static constexpr uint32_t kNumBars = 4 + 2 * kNSK + 4 * kNSV + 8 + 1 + 2;
   static constexpr uint32_t kBytes = kBar + kNumBars * 8 + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *o_full = p_full + 2;        // [2] MMA -> softmax: O final for the item
   uint64_t *o_empty = o_full + 2;       // [2] softmax -> MMA: O read out
   uint64_t *drain = o_empty + 2;        // [1] teardown: all MMAs complete
+  uint64_t *p_half = drain + 1;         // [2] softmax -> MMA: first half of P ready (and O rescaled)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], kBM / 32);  // one arrive per softmax warp
+      mbar_init(&p_half[i], kBM / 32);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_empty[i], kBM / 32);
     }
@@ -430,12 +432,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    auto issue_pv = [=](int i, uint32_t stage, bool acc) {
+    // O_i += P_i V over K columns [16 k0, 16 k1) of the tile.
+    auto issue_pv = [=](int i, uint32_t stage, bool acc, int k0, int k1) {
       const uint64_t vb = dV0 + ((stage * kVStageBytes) >> 4);
       const uint32_t d = tm + 256u + i * D, pa = tm + i * 128u;
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
+        for (int kk = k0; kk < k1; ++kk)
           mma_f16_ts(d, pa + kk * 8, vb + ((kk * 16 * 128) >> 4), kIdescPV, (acc || kk > 0) ? 1u : 0u);
       }
       __syncwarp();
@@ -446,6 +449,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto wait = [=](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, budget));
+    };
+    // The softmax releases P in two halves (first 64 key columns, then the
+    // rest), so the first half of PV overlaps the second half of its exps.
+    auto pv_in_halves = [&](int i, uint32_t stage, bool acc, uint32_t parity) {
+      if (!wait(&p_half[i], parity)) return false;
+      tc_fence_after();
+      issue_pv(i, stage, acc, 0, kBN / 32);
+      if (!wait(&p_full[i], parity)) return false;
+      tc_fence_after();
+      issue_pv(i, stage, acc, kBN / 32, kBN / 16);
+      return true;
     };
     uint32_t g = 0;
     int it = 0;
@@ -473,10 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (jj > 0) {  // O1 += P1 V for the previous tile
           const uint32_t pst = (g - 1) % kNSV;
           if (jj == 1 && it > 0 && !(ok = wait(&o_empty[1], (it - 1) & 1))) break;
-          if (!(ok = wait(&p_full[1], (g - 1) & 1))) break;
+          if (!(ok = pv_in_halves(1, pst, jj > 1, (g - 1) & 1))) break;
           if (lane == 0) CCA_TRACE_EV(3, g - 1);
-          tc_fence_after();
-          issue_pv(1, pst, jj > 1);
           commit(&pv_empty[pst]);
         }
         issue_qk(1, stage);
@@ -493,10 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait(&pv_full[vst], vph))) break;
         if (lane == 0) CCA_TRACE_EV(8, g);
         if (jj == 0 && it > 0 && !(ok = wait(&o_empty[0], (it - 1) & 1))) break;
-        if (!(ok = wait(&p_full[0], g & 1))) break;
+        if (!(ok = pv_in_halves(0, vst, jj > 0, g & 1))) break;
         if (lane == 0) CCA_TRACE_EV(5, g);
-        tc_fence_after();
-        issue_pv(0, vst, jj > 0);
         if (lane == 0) CCA_TRACE_EV(6, g);
         if (jj == n - 1) commit(&o_full[0]);
       }
@@ -504,9 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       {  // O1 += P1 V for the last tile
         const uint32_t pst = (g - 1) % kNSV;
         if (n == 1 && it > 0 && !(ok = wait(&o_empty[1], (it - 1) & 1))) break;
-        if (!(ok = wait(&p_full[1], (g - 1) & 1))) break;
-        tc_fence_after();
-        issue_pv(1, pst, n > 1);
+        if (!(ok = pv_in_halves(1, pst, n > 1, (g - 1) & 1))) break;
         commit(&pv_empty[pst]);
         commit(&o_full[1]);
       }
@@ -696,9 +704,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         // exponent, so the fp16 result is P itself; its sum is divided by pf.
         const float m_off = (kFp8 && kExpMode == 1) ? m_new - __log2f(pf) : m_new;
         const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_off, -m_off);
+        // Rescale this row of O when the reference maximum moved (O of the
+        // previous tile is complete: S of this tile was committed after it);
+        // done before the first half of P is released to the PV MMAs.
+        if (j > j0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0, o);
+            tmem_ld_wait32(o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(tO + c0, o);
+          }
+        }
         uint64_t sums[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
+          if (q4 == 2) {  // first 64 key columns of P (and the O rescale) are in TMEM
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_half[wg]);
+          }
           uint32_t p16[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
@@ -734,19 +762,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float tile_sum = (kFp8 && kExpMode == 1) ? (s_lo + s_hi) / pf : (s_lo + s_hi);
         l_sum = l_sum * alpha + tile_sum;
         m_ref = m_new;
-        // Rescale this row of O when the reference maximum moved (O of the
-        // previous tile is complete: S of this tile was committed after it).
-        if (j > j0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c0, o);
-            tmem_ld_wait32(o);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tO + c0, o);
-          }
-        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
