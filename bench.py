@@ -501,8 +501,13 @@ def run_gpu(args, rank, world, local_rank):
     traffic = None
     prof = os.path.join(ROOT, "profiles", "attn_bf16_720p.traffic.json")
     if os.path.exists(prof):
+        # counters taken on another build of the kernel do not describe this one
         try:
-            traffic = json.load(open(prof)).get("dram_bytes_per_launch")
+            import hashlib
+            rec = json.load(open(prof))
+            src = os.path.join(ROOT, "chunk_causal_attention_b200", "csrc", "attn.cu")
+            if rec.get("attn_cu_sha256") == hashlib.sha256(open(src, "rb").read()).hexdigest():
+                traffic = rec.get("dram_bytes_per_launch")
         except Exception:
             traffic = None
     line = {
@@ -531,6 +536,48 @@ def run_gpu(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ profiling cases
+def profile_case(name: str) -> None:
+    """Run one memory-bound kernel a few times on its sweep-size input (L2 flushed
+    in between) and exit: a small, self-contained target for ncu captures."""
+    import torch
+    import chunk_causal_attention_b200 as cca
+    dev = torch.device("cuda:0")
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    if name == "compact_64M":
+        n = 1 << 26
+        mc = (torch.rand(n, device=dev) < 0.3).to(torch.uint8)
+        idx = torch.empty(n, dtype=torch.int32, device=dev)
+        na = torch.empty(1, dtype=torch.int32, device=dev)
+        ws = torch.empty(cca.cca_compact_workspace_size(n), dtype=torch.uint8, device=dev)
+        fn = lambda: cca.cca_compact(mc, idx, na, workspace=ws)
+    elif name == "append_720p":
+        ring = cca.KVRing(H, D, L, W, device=dev)
+        k = torch.randn((L, H, D), device=dev).to(torch.bfloat16)
+        v = torch.randn((L, H, D), device=dev).to(torch.bfloat16)
+        fn = lambda: ring.append(k, v)
+    elif name == "mask_fixed_16M":
+        n = 1 << 24
+        src = torch.randn((n, 16), device=dev)
+        edit = src + 0.5 * torch.randn((n, 16), device=dev)
+        mask = torch.empty(n, dtype=torch.uint8, device=dev)
+        fn = lambda: cca.cca_token_mask_l2(src, edit, tau=2.0, mask=mask)
+    elif name == "scatter_64K_rows":
+        n = 1 << 16
+        oc = torch.randn((n, H * D), device=dev).to(torch.bfloat16)
+        cache = torch.zeros((2 * n, H * D), device=dev, dtype=torch.bfloat16)
+        ids = torch.arange(0, 2 * n, 2, dtype=torch.int32, device=dev)
+        nn = torch.full((1,), n, dtype=torch.int32, device=dev)
+        fn = lambda: cca.cca_scatter(oc, ids, nn, cache)
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    for _ in range(3):
+        flush.sum()
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "ok": True}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -541,7 +588,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extras", type=int, default=1, help="also time the fp8, mask-cached, long-stream and "
                     "memory-bound workloads (rank 0, extra keys)")
+    ap.add_argument("--profile-case", default=None,
+                    help="only run one memory-bound kernel (compact_64M, append_720p, mask_fixed_16M, "
+                    "scatter_64K_rows) three times, for ncu")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
