@@ -228,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *p_full = s_full + 2;        // [2] softmax -> MMA: P ready (and O rescaled)
   uint64_t *o_full = p_full + 2;        // [2] MMA -> softmax: O final for the item
   uint64_t *o_empty = o_full + 2;       // [2] softmax -> MMA: O read out
-  uint64_t *drain = o_empty + 2;        // [1] teardown: all MMAs complete
-  uint64_t *p_half = drain + 1;         // [2] softmax -> MMA: first half of P ready (and O rescaled)
+  uint64_t *p_half = o_empty + 2;       // [2] softmax -> MMA: first half of P ready (and O rescaled)
+  uint64_t *drain = p_half + 2;         // [1] teardown: all MMAs complete
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
