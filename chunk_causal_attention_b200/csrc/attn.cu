@@ -234,6 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The combine grid (a programmatic dependent) may be scheduled from now on; it
+  // waits for this grid's completion before it reads anything.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int n_q = a.n_q_dev ? min(max(*a.n_q_dev, 0), a.n_q_max) : a.n_q_max;
   const Sched sch = make_sched(n_q, a.H, a.n_kv_tiles, gridDim.x);
 
@@ -836,12 +839,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // out[row][head] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s over the CTAs
 // whose KV range meets the item.  The schedule is recomputed from n_q exactly as
 // the attention kernel (launched with G CTAs) computed it.  Lane i examines
-// candidate CTA c_lo + i; the found partials are then summed by the whole warp.
+// candidate CTA c_first + i; the O rows of up to 8 found pieces are then loaded
+// by the whole warp at once (lane = D/32 columns) before they are summed, so a
+// row costs about two memory round trips.  Launched as a programmatic dependent
+// of the attention kernel: it is resident before the attention grid ends and
+// waits (griddepcontrol.wait) for that grid's memory before reading.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restrict__ ws_o,
                                                            const float *__restrict__ ws_ml,
                                                            const int32_t *__restrict__ n_q_dev, int n_q_max, int H,
                                                            int n_kv, int G, __nv_bfloat16 *__restrict__ out) {
+  constexpr int kV = D / 32;  // columns per lane
+  constexpr int kBatch = 8;   // pieces loaded at once
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n_q = n_q_dev ? min(max(*n_q_dev, 0), n_q_max) : n_q_max;
   const Sched sch = make_sched(n_q, H, n_kv, G);
   if (sch.r == 0) return;
@@ -856,8 +866,6 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restri
     const int row = pair * (kNQ * kBM) + rr;
     if (row >= n_q) continue;
     const uint32_t t0 = static_cast<uint32_t>(ur) * n_kv, t1 = t0 + n_kv;  // the item's tiles in the list
-    // Covering CTAs: from the first c with hi_c > t0 to at most ceil(t1 G / tr);
-    // lanes examine 32 candidates at a time.
     const int c_first = static_cast<int>(((t0 + 1) * uG + tr - 1) / tr) - 1;
     const int c_last = min(G - 1, static_cast<int>((t1 * uG + tr - 1) / tr));
     auto probe = [&](int c, int &slot) {
@@ -866,44 +874,68 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restri
       slot = 2 * c + (lo / n_kv == static_cast<uint32_t>(ur) ? 0 : 1);
       return lo < hi && hi > t0 && lo < t1;
     };
+    // pass 1: (m, l) of every piece, one lane per candidate
     float mmax = -INFINITY;
     for (int cb = c_first; cb <= c_last; cb += 32) {
       int slot;
       if (probe(cb + lane, slot))
-        mmax = fmaxf(mmax, ws_ml[(static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2]);
+        mmax = fmaxf(mmax, __ldcg(ws_ml + (static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
-    float den = 0.f;
-    float acc[D / 32];
+    float den = 0.f, acc[kV];
 #pragma unroll
-    for (int k = 0; k < D / 32; ++k) acc[k] = 0.f;
+    for (int k = 0; k < kV; ++k) acc[k] = 0.f;
     for (int cb = c_first; cb <= c_last; cb += 32) {
       int slot = 0;
       const bool mine = probe(cb + lane, slot);
       float wgt = 0.f;
       if (mine) {
-        const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + (static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2);
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(ws_ml + (static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2));
         wgt = exp2f(ml.x - mmax);
         den += wgt * ml.y;
       }
+      // pass 2: O rows of the found pieces, kBatch loads in flight per lane
       unsigned todo = __ballot_sync(0xffffffffu, mine);
       while (todo) {
-        const int src = __ffs(todo) - 1;
-        todo &= todo - 1;
-        const float ws = __shfl_sync(0xffffffffu, wgt, src);
-        const int sl = __shfl_sync(0xffffffffu, slot, src);
-        const float *o = ws_o + (static_cast<int64_t>(sl) * (kNQ * kBM) + rr) * D;
+        float ws[kBatch], x[kBatch][kV];
 #pragma unroll
-        for (int k = 0; k < D / 32; ++k) acc[k] += ws * o[k * 32 + lane];
+        for (int b = 0; b < kBatch; ++b) {
+          const int src = todo ? __ffs(todo) - 1 : 0;
+          const bool live = todo != 0;
+          todo &= todo - 1;
+          ws[b] = live ? __shfl_sync(0xffffffffu, wgt, src) : 0.f;
+          const int sl = __shfl_sync(0xffffffffu, slot, src);
+          const float *o = ws_o + (static_cast<int64_t>(sl) * (kNQ * kBM) + rr) * D + lane * kV;
+          if (live) {
+            if constexpr (kV == 4) {
+              const float4 v = __ldcg(reinterpret_cast<const float4 *>(o));
+              x[b][0] = v.x, x[b][1] = v.y, x[b][2] = v.z, x[b][3] = v.w;
+            } else {
+              const float2 v = __ldcg(reinterpret_cast<const float2 *>(o));
+              x[b][0] = v.x, x[b][1] = v.y;
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < kV; ++k) x[b][k] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b)
+#pragma unroll
+          for (int k = 0; k < kV; ++k) acc[k] += ws[b] * x[b][k];
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     const float inv = 1.f / den;
-    __nv_bfloat16 *dst = out + (static_cast<int64_t>(row) * H + head) * D;
-#pragma unroll
-    for (int k = 0; k < D / 32; ++k) dst[k * 32 + lane] = __float2bfloat16_rn(acc[k] * inv);
+    __nv_bfloat16 *dst = out + (static_cast<int64_t>(row) * H + head) * D + lane * kV;
+    if constexpr (kV == 4) {
+      *reinterpret_cast<uint2 *>(dst) = make_uint2(sm100::pack_bf16x2(acc[0] * inv, acc[1] * inv),
+                                                   sm100::pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    } else {
+      *reinterpret_cast<uint32_t *>(dst) = sm100::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    }
   }
 }
 
@@ -999,8 +1031,23 @@ static cca_status launch_attn(const cca_kv_ring *ring, const AttnPlan &p, const 
     int64_t blocks = (warps + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
-    attn_combine_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        args.ws_o, args.ws_ml, args.n_q_dev, args.n_q_max, d.n_heads, p.n_kv_tiles, p.grid, args.out);
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, attn_combine_kernel<D>, static_cast<const float *>(args.ws_o),
+                                              static_cast<const float *>(args.ws_ml), args.n_q_dev, args.n_q_max,
+                                              d.n_heads, p.n_kv_tiles, p.grid, args.out);
+    if (le != cudaSuccess) {
+      cudaGetLastError();
+      return fail(CCA_ERR_CUDA, "cca_chunk_attn: combine launch failed: %s", cudaGetErrorString(le));
+    }
     CCA_TRY(launched("attn_combine_kernel"));
   }
   return CCA_OK;
