@@ -457,33 +457,61 @@ def run_gpu(args, rank, world, local_rank):
     # ---- end to end through the public API with host buffers (pinned), rank-local
     e2e = None
     if args.e2e_steps > 0:
+        # Two buffer sets, three streams: the inputs of step k+1 go up (copy
+        # engine, s_in) while step k computes (s_c) and step k-1's outputs come
+        # down (s_out).  Every step still copies all of its inputs and outputs.
         pin = lambda x: synth.as_torch_bf16(x).pin_memory()
         hq = [pin(x) for x in c1.q]
         hk = [pin(x) for x in c1.k_cur]
         hv = [pin(x) for x in c1.v_cur]
-        ho = [torch.empty((L, H, D), dtype=torch.bfloat16).pin_memory() for _ in c1.q]
+        ho = [[torch.empty((L, H, D), dtype=torch.bfloat16).pin_memory() for _ in c1.q] for _ in range(2)]
         rep = reps[0]
-        dq = [torch.empty_like(x, device=dev) for x in hq]
-        dk = [torch.empty_like(x, device=dev) for x in hk]
-        dv = [torch.empty_like(x, device=dev) for x in hv]
+        dq = [[torch.empty_like(x, device=dev) for x in hq] for _ in range(2)]
+        dk = [[torch.empty_like(x, device=dev) for x in hk] for _ in range(2)]
+        dv = [[torch.empty_like(x, device=dev) for x in hv] for _ in range(2)]
+        do = [[torch.empty((L, H, D), dtype=torch.bfloat16, device=dev) for _ in c1.q] for _ in range(2)]
+        s_in, s_out, s_c = torch.cuda.Stream(dev), torch.cuda.Stream(dev), stream
+        ev = lambda: torch.cuda.Event()
+        in_ready, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        used = [False, False]
 
-        def e2e_step():
-            for s in range(CALLS_PER_STEP):
-                dq[s].copy_(hq[s], non_blocking=True)
-                dk[s].copy_(hk[s], non_blocking=True)
-                dv[s].copy_(hv[s], non_blocking=True)
-                cca.cca_chunk_attn(rep.ring, dq[s], dk[s], dv[s], out=rep.out[s], workspace=rep.ws)
-                ho[s].copy_(rep.out[s], non_blocking=True)
-            rep.ring.append(dk[-1], dv[-1])
+        def e2e_step(k):
+            b = k & 1
+            if used[b]:
+                s_in.wait_event(comp_done[b])  # step k-2 no longer reads this input set
+            with torch.cuda.stream(s_in):
+                for s_ in range(CALLS_PER_STEP):
+                    dq[b][s_].copy_(hq[s_], non_blocking=True)
+                    dk[b][s_].copy_(hk[s_], non_blocking=True)
+                    dv[b][s_].copy_(hv[s_], non_blocking=True)
+                in_ready[b].record(s_in)
+            s_c.wait_event(in_ready[b])
+            if used[b]:
+                s_c.wait_event(out_done[b])  # step k-2's outputs have been read back
+            for s_ in range(CALLS_PER_STEP):
+                cca.cca_chunk_attn(rep.ring, dq[b][s_], dk[b][s_], dv[b][s_], out=do[b][s_], workspace=rep.ws,
+                                   stream=s_c)
+            rep.ring.append(dk[b][-1], dv[b][-1], stream=s_c)
+            comp_done[b].record(s_c)
+            s_out.wait_event(comp_done[b])
+            with torch.cuda.stream(s_out):
+                for s_ in range(CALLS_PER_STEP):
+                    ho[b][s_].copy_(do[b][s_], non_blocking=True)
+                out_done[b].record(s_out)
+            used[b] = True
 
-        for _ in range(3):
-            e2e_step()
+        for k in range(3):
+            e2e_step(k)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
+        e0.record(s_c)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for k in range(args.e2e_steps):
+            e2e_step(k)
+        s_c.wait_event(in_ready[(args.e2e_steps - 1) & 1])
+        s_c.wait_event(out_done[(args.e2e_steps - 1) & 1])
+        e1.record(s_c)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
         h2d = CALLS_PER_STEP * 3 * L * H * D * 2
