@@ -1,5 +1,5 @@
 // Thin wrappers over the sm_100a PTX used by the attention kernel: mbarriers,
-// TMA tile loads (no multicast), tcgen05 MMA / TMEM load-store / alloc, fences.
+// TMA tile loads into the issuing CTA only, tcgen05 MMA / TMEM load-store / alloc, fences.
 #pragma once
 
 #include <cuda.h>
@@ -78,7 +78,7 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, long 
   }
 }
 
-// ------------------------------------------------------------------ bulk copies (untiled, no multicast)
+// ------------------------------------------------------------------ bulk copies (untiled, issuing CTA only)
 // global -> shared, completion counted in bytes on an mbarrier; both addresses
 // 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void *src, uint32_t bytes, uint64_t *bar) {
