@@ -439,7 +439,7 @@ def _fp8_call(ring, q, kc, vc, **kw):
 
 
 @pytest.mark.parametrize("ctas", ["auto", "24"])
-def test_attention_fp8_720p(ctas, monkeypatch):
+def test_attention_fp8_720p(ctas, monkeypatch, record_property):
     if ctas != "auto":
         monkeypatch.setenv("CCA_ATTN_CTAS", ctas)
     s = synth.fp8_720p()
@@ -450,6 +450,15 @@ def test_attention_fp8_720p(ctas, monkeypatch):
         o = _fp8_call(ring, s.q[st], s.k_cur[st], s.v_cur[st])
         ref = _fp8_stream_ref(s.ring_k, s.ring_v, s.q[st], s.k_cur[st], s.v_cur[st], s.t, s.window)
         assert_attn_close(to_np(o), ref, FP8_MAX_ABS, FP8_REL_L2, what=f"fp8 720p step {st}")
+        if st == 0 and ctas == "auto":
+            # information only: the same call against fp64 attention on the
+            # unquantised inputs (quantisation error + kernel error)
+            raw = oca.chunk_attention(s.q[st], {c: s.ring_k[c] for c in range(s.t)},
+                                      {c: s.ring_v[c] for c in range(s.t)}, s.t, s.window,
+                                      k_cur=s.k_cur[st], v_cur=s.v_cur[st])
+            d = to_np(o) - raw
+            record_property("fp8_vs_unquantised_max_abs", float(np.abs(d).max()))
+            record_property("fp8_vs_unquantised_rel_l2", float(np.linalg.norm(d) / np.linalg.norm(raw)))
     check_status(ring)
 
 
