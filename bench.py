@@ -566,8 +566,8 @@ def run_gpu(args, rank, world, local_rank):
 
 # ------------------------------------------------------------------ profiling cases
 def profile_case(name: str) -> None:
-    """Run one memory-bound kernel a few times on its sweep-size input (L2 flushed
-    in between) and exit: a small, self-contained target for ncu captures."""
+    """Run one kernel a few times on its workload (L2 flushed in between) and
+    exit: a small, self-contained target for ncu captures."""
     import torch
     import chunk_causal_attention_b200 as cca
     dev = torch.device("cuda:0")
@@ -597,6 +597,32 @@ def profile_case(name: str) -> None:
         ids = torch.arange(0, 2 * n, 2, dtype=torch.int32, device=dev)
         nn = torch.full((1,), n, dtype=torch.int32, device=dev)
         fn = lambda: cca.cca_scatter(oc, ids, nn, cache)
+    elif name == "fp8_720p":
+        import synth
+        bf = lambda x: synth.as_torch_bf16(x, dev)
+        s3 = synth.fp8_720p(n_steps=1)
+        ring8 = cca.KVRing(H, D, L, W, dtype="e4m3", device=dev)
+        for t in range(s3.t):
+            ring8.append(bf(s3.ring_k[t]), bf(s3.ring_v[t]))
+        q8, qs = cca.cca_quant_e4m3(bf(s3.q[0]))
+        k8, ks = cca.cca_quant_e4m3(bf(s3.k_cur[0]))
+        v8, vs = cca.cca_quant_e4m3(bf(s3.v_cur[0]))
+        ws8 = torch.empty(max(cca.cca_chunk_attn_workspace_size(ring8, L), 16), dtype=torch.uint8, device=dev)
+        fn = lambda: cca.cca_chunk_attn(ring8, q8, k8, v8, q_scale=qs, kcur_scale=ks, vcur_scale=vs, workspace=ws8)
+    elif name == "masked_720p":
+        import synth
+        bf = lambda x: synth.as_torch_bf16(x, dev)
+        c1 = synth.chunk_720p(n_steps=1)
+        m = synth.mask_chunk()
+        ring = cca.KVRing(H, D, L, W, device=dev)
+        for t in range(c1.t):
+            ring.append(bf(c1.ring_k[t]), bf(c1.ring_v[t]))
+        mask = cca.cca_token_mask_l2(torch.from_numpy(m.src).to(dev), torch.from_numpy(m.edit).to(dev),
+                                     prune_quantile=m.prune_quantile)
+        idx, n_act = cca.cca_compact(mask)
+        q, kc, vc = bf(c1.q[0]), bf(c1.k_cur[0]), bf(c1.v_cur[0])
+        wsm = torch.empty(max(cca.cca_chunk_attn_workspace_size(ring, L), 16), dtype=torch.uint8, device=dev)
+        fn = lambda: cca.cca_chunk_attn(ring, q, kc, vc, q_idx=idx, n_q_dev=n_act, n_q_max=L, workspace=wsm)
     else:
         raise SystemExit(f"unknown profile case {name}")
     for _ in range(3):
@@ -617,8 +643,8 @@ def main():
     ap.add_argument("--extras", type=int, default=1, help="also time the fp8, mask-cached, long-stream and "
                     "memory-bound workloads (rank 0, extra keys)")
     ap.add_argument("--profile-case", default=None,
-                    help="only run one memory-bound kernel (compact_64M, append_720p, mask_fixed_16M, "
-                    "scatter_64K_rows) three times, for ncu")
+                    help="only run one kernel three times, for ncu: compact_64M, append_720p, mask_fixed_16M, "
+                    "scatter_64K_rows, fp8_720p (e4m3 attention), masked_720p (486 gathered queries)")
     args = ap.parse_args()
     if args.profile_case:
         profile_case(args.profile_case)
