@@ -22,6 +22,7 @@ import torch
 __all__ = [
     "CCA_BF16", "CCA_E4M3", "CCA_F32", "CcaError", "KVRing", "lib", "lib_path", "EXPORTED",
     "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc",
+    "cca_chunk_attn_scatter",
     "cca_token_mask_l2", "cca_compact", "cca_compact_workspace_size", "cca_scatter", "cca_selftest_bounded_wait",
     "cca_version",
     "cca_take_launch_count",
@@ -36,7 +37,7 @@ _STATUS = {0: "CCA_OK", 1: "CCA_ERR_INVALID_ARG", 2: "CCA_ERR_UNSUPPORTED", 3: "
 EXPORTED = (
     "cca_kv_ring_create", "cca_kv_ring_destroy", "cca_kv_ring_reset", "cca_kv_ring_query",
     "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn",
-    "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_token_mask_l2", "cca_compact",
+    "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_chunk_attn_scatter", "cca_token_mask_l2", "cca_compact",
     "cca_compact_workspace_size",
     "cca_scatter", "cca_selftest_bounded_wait", "cca_last_error", "cca_version", "cca_take_launch_count",
 )
@@ -84,6 +85,7 @@ def lib() -> ctypes.CDLL:
         "cca_chunk_attn": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp],
         "cca_chunk_attn_workspace_size": [vp, i32, ctypes.POINTER(sz)],
         "cca_chunk_attn_noalloc": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp],
+        "cca_chunk_attn_scatter": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp],
         "cca_token_mask_l2": [vp, vp, i32, i32, f32, f32, vp, vp, vp, vp],
         "cca_compact": [vp, i32, vp, vp, vp, sz, vp],
         "cca_compact_workspace_size": [i32, ctypes.POINTER(sz)],
@@ -267,6 +269,28 @@ def cca_chunk_attn(ring: KVRing, q: torch.Tensor, k_cur: torch.Tensor, v_cur: to
                                 _ptr(out, "out", torch.bfloat16), _ptr(workspace, "workspace"), ws_bytes,
                                 _stream(stream)), "cca_chunk_attn")
     return out
+
+
+def cca_chunk_attn_scatter(ring: KVRing, q: torch.Tensor, k_cur: torch.Tensor, v_cur: torch.Tensor,
+                           q_idx: torch.Tensor, o_cache: torch.Tensor, q_scale=None, kcur_scale=None,
+                           vcur_scale=None, n_q_dev: Optional[torch.Tensor] = None, n_q_max: Optional[int] = None,
+                           softmax_scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """Active-query attention whose result for query i lands in row q_idx[i] of
+    o_cache ([L, H, D] bf16, updated in place); other rows are left as they are."""
+    if n_q_max is None:
+        n_q_max = q_idx.shape[0]
+    need = cca_chunk_attn_workspace_size(ring, n_q_max)
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().cca_chunk_attn_scatter(ring.handle, _ptr(q, "q"), _ptr(k_cur, "k_cur"), _ptr(v_cur, "v_cur"),
+                                        _ptr(q_scale, "q_scale"), _ptr(kcur_scale, "kcur_scale"),
+                                        _ptr(vcur_scale, "vcur_scale"), _ptr(q_idx, "q_idx", torch.int32),
+                                        _ptr(n_q_dev, "n_q_dev", torch.int32), int(n_q_max), float(softmax_scale),
+                                        _ptr(o_cache, "o_cache", torch.bfloat16), _ptr(workspace, "workspace"),
+                                        ws_bytes, _stream(stream)), "cca_chunk_attn_scatter")
+    return o_cache
 
 
 def cca_chunk_attn_noalloc(ring: KVRing, q: torch.Tensor, k_cur: torch.Tensor, v_cur: torch.Tensor,

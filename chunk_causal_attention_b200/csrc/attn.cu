@@ -104,7 +104,8 @@ struct AttnArgs {
   const void *q;           // query rows (gather path): [L][H][D] of the ring's element type
   const int32_t *q_idx;    // NULL: dense rows
   const int32_t *n_q_dev;  // NULL: n_q = n_q_max
-  __nv_bfloat16 *out;      // [n_q_max][H][D]
+  __nv_bfloat16 *out;      // [n_q_max][H][D], or [L][H][D] with scatter_out
+  int scatter_out;         // 1: query i's row goes to out row q_idx[i] (fused scatter-back)
   float *ws_o;             // [2 x grid][256][D] partial O of split items (unnormalised)
   float *ws_ml;            // [2 x grid][256][2] (running max in log2 units, row sum)
   int32_t *dev_status;
@@ -779,13 +780,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = row < n_q;
       if (sg.slot < 0) {
         const float inv = s_vmax / l_sum;
-        __nv_bfloat16 *dst = a.out + (static_cast<int64_t>(row) * a.H + head) * D;
+        const int orow = a.scatter_out && row_ok ? __ldg(a.q_idx + row) : row;
+        const bool wr_ok = row_ok && orow >= 0 && orow < (a.scatter_out ? a.L : a.n_q_max);
+        __nv_bfloat16 *dst = a.out + (static_cast<int64_t>(wr_ok ? orow : 0) * a.H + head) * D;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tO + c0, o);
           tmem_ld_wait32(o);
-          if (row_ok) {
+          if (wr_ok) {
             uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -848,7 +851,8 @@ template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restrict__ ws_o,
                                                            const float *__restrict__ ws_ml,
                                                            const int32_t *__restrict__ n_q_dev, int n_q_max, int H,
-                                                           int n_kv, int G, __nv_bfloat16 *__restrict__ out) {
+                                                           int n_kv, int G, __nv_bfloat16 *__restrict__ out,
+                                                           const int32_t *__restrict__ out_idx, int n_rows) {
   constexpr int kV = D / 32;  // columns per lane
   constexpr int kBatch = 8;   // pieces loaded at once
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -929,7 +933,9 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restri
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     const float inv = 1.f / den;
-    __nv_bfloat16 *dst = out + (static_cast<int64_t>(row) * H + head) * D + lane * kV;
+    const int orow = out_idx ? __ldg(out_idx + row) : row;  // fused scatter-back
+    if (orow < 0 || orow >= n_rows) continue;               // bad index (flagged by the gather)
+    __nv_bfloat16 *dst = out + (static_cast<int64_t>(orow) * H + head) * D + lane * kV;
     if constexpr (kV == 4) {
       *reinterpret_cast<uint2 *>(dst) = make_uint2(sm100::pack_bf16x2(acc[0] * inv, acc[1] * inv),
                                                    sm100::pack_bf16x2(acc[2] * inv, acc[3] * inv));
@@ -1043,7 +1049,9 @@ static cca_status launch_attn(const cca_kv_ring *ring, const AttnPlan &p, const 
     cfg.numAttrs = 1;
     const cudaError_t le = cudaLaunchKernelEx(&cfg, attn_combine_kernel<D>, static_cast<const float *>(args.ws_o),
                                               static_cast<const float *>(args.ws_ml), args.n_q_dev, args.n_q_max,
-                                              d.n_heads, p.n_kv_tiles, p.grid, args.out);
+                                              d.n_heads, p.n_kv_tiles, p.grid, args.out,
+                                              args.scatter_out ? args.q_idx : static_cast<const int32_t *>(nullptr),
+                                              args.scatter_out ? args.L : args.n_q_max);
     if (le != cudaSuccess) {
       cudaGetLastError();
       return fail(CCA_ERR_CUDA, "cca_chunk_attn: combine launch failed: %s", cudaGetErrorString(le));
@@ -1056,6 +1064,12 @@ static cca_status launch_attn(const cca_kv_ring *ring, const AttnPlan &p, const 
 }  // namespace cca
 
 using namespace cca;
+
+static cca_status chunk_attn_impl(const cca_kv_ring *ring, const void *q, const void *k_cur, const void *v_cur,
+                                  const float *q_scale, const float *kcur_scale, const float *vcur_scale,
+                                  const int32_t *q_idx, const int32_t *n_q_dev, int32_t n_q_max,
+                                  float softmax_scale, void *out, int scatter_out, void *workspace,
+                                  size_t workspace_bytes, cca_stream_t stream);
 
 extern "C" {
 
@@ -1084,6 +1098,28 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q, const void *k_
                           const float *q_scale, const float *kcur_scale, const float *vcur_scale,
                           const int32_t *q_idx, const int32_t *n_q_dev, int32_t n_q_max, float softmax_scale,
                           void *out, void *workspace, size_t workspace_bytes, cca_stream_t stream) {
+  return chunk_attn_impl(ring, q, k_cur, v_cur, q_scale, kcur_scale, vcur_scale, q_idx, n_q_dev, n_q_max,
+                         softmax_scale, out, 0, workspace, workspace_bytes, stream);
+}
+
+cca_status cca_chunk_attn_scatter(const cca_kv_ring *ring, const void *q, const void *k_cur, const void *v_cur,
+                                  const float *q_scale, const float *kcur_scale, const float *vcur_scale,
+                                  const int32_t *q_idx, const int32_t *n_q_dev, int32_t n_q_max,
+                                  float softmax_scale, void *o_cache, void *workspace, size_t workspace_bytes,
+                                  cca_stream_t stream) {
+  if (n_q_max > 0 && !q_idx)
+    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn_scatter: q_idx is required (it also names the output rows)");
+  return chunk_attn_impl(ring, q, k_cur, v_cur, q_scale, kcur_scale, vcur_scale, q_idx, n_q_dev, n_q_max,
+                         softmax_scale, o_cache, 1, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+static cca_status chunk_attn_impl(const cca_kv_ring *ring, const void *q, const void *k_cur, const void *v_cur,
+                                  const float *q_scale, const float *kcur_scale, const float *vcur_scale,
+                                  const int32_t *q_idx, const int32_t *n_q_dev, int32_t n_q_max,
+                                  float softmax_scale, void *out, int scatter_out, void *workspace,
+                                  size_t workspace_bytes, cca_stream_t stream) {
   if (!ring) return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: NULL ring");
   const cca_kv_ring_desc &d = ring->d;
   if (n_q_max < 0 || n_q_max > d.chunk_len)
@@ -1122,6 +1158,7 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q, const void *k_
   args.q_idx = q_idx;
   args.n_q_dev = n_q_dev;
   args.out = static_cast<__nv_bfloat16 *>(out);
+  args.scatter_out = scatter_out;
   if (need > 0) {
     args.ws_o = static_cast<float *>(workspace);
     const size_t rows = static_cast<size_t>(2) * p.grid * (kNQ * kBM);
@@ -1145,7 +1182,6 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q, const void *k_
   return launch_attn<64, false>(ring, p, args, q, k_cur, v_cur, st);
 }
 
-}  // extern "C"
 
 // ------------------------------------------------------------------ allocation-free variant
 // Some callers cannot hand this library a scratch buffer: a real-time stream

@@ -175,6 +175,27 @@ cca_status cca_chunk_attn(const cca_kv_ring *ring, const void *q,
                           float softmax_scale, void *out, void *workspace,
                           size_t workspace_bytes, cca_stream_t stream);
 
+/* Active-query attention with the scatter-back fused into its epilogue
+ * ["LiveEdit ...", sections 방법론 and 기술 상세: recompute only where the mask
+ * is 1, reuse the cached self-attention output elsewhere]: exactly
+ * cca_chunk_attn with q_idx, except that the result for query i is written to
+ * row q_idx[i] of o_cache instead of row i of a compact buffer, so no separate
+ * cca_scatter pass (and no compact buffer) is needed.  Rows of o_cache that no
+ * active query names keep their contents.
+ *  q_idx: required, device int32 [n_q_max] (as produced by cca_compact);
+ *      an index outside [0, L) sets CCA_DEV_BAD_INDEX and that row is skipped.
+ *  o_cache: device bf16 [L][H][D].
+ *  Other arguments, workspace and errors: as cca_chunk_attn (same workspace
+ *  size). */
+cca_status cca_chunk_attn_scatter(const cca_kv_ring *ring, const void *q,
+                                  const void *k_cur, const void *v_cur,
+                                  const float *q_scale, const float *kcur_scale,
+                                  const float *vcur_scale, const int32_t *q_idx,
+                                  const int32_t *n_q_dev, int32_t n_q_max,
+                                  float softmax_scale, void *o_cache,
+                                  void *workspace, size_t workspace_bytes,
+                                  cca_stream_t stream);
+
 /* Bytes of device workspace cca_chunk_attn needs for this ring and n_q_max
  * (the split-KV partial results; 0 when no split is used). */
 cca_status cca_chunk_attn_workspace_size(const cca_kv_ring *ring, int32_t n_q_max,

@@ -122,6 +122,8 @@ def test_call_validation_without_device_work(L):
                             0.0, vp(0x1000), None, 0, None) == 1
     assert L.cca_chunk_attn(h, None, None, None, None, None, None, None, None, 0, 0.0, None, None, 0,
                             None) == 0  # nothing to do
+    assert L.cca_chunk_attn_scatter(h, vp(0x1000), vp(0x1000), vp(0x1000), None, None, None, None, None, 16,
+                                    0.0, vp(0x1000), None, 0, None) == 1  # q_idx names the output rows
     # mask / compact / scatter argument checks
     assert L.cca_token_mask_l2(vp(0x1000), vp(0x1000), 10, 6, 1.0, -1.0, vp(0x1000), None, None, None) == 1
     assert L.cca_token_mask_l2(vp(0x1000), vp(0x1000), 10, 16, 1.0, 1.5, vp(0x1000), None, None, None) == 1

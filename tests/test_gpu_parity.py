@@ -377,6 +377,60 @@ def test_mask_cached_chunk_end_to_end(c1, c1_ring, c1_ref):
     assert diff <= 1e-2
 
 
+@pytest.mark.parametrize("ctas", ["auto", "37"])
+def test_fused_scatter_equals_attention_then_scatter(c1, c1_ring, monkeypatch, ctas):
+    """cca_chunk_attn_scatter writes every active query's row straight into the
+    cache: bit-identical to cca_chunk_attn on the compact buffer followed by
+    cca_scatter (split items included), inactive rows untouched."""
+    if ctas != "auto":
+        monkeypatch.setenv("CCA_ATTN_CTAS", ctas)
+    m = synth.mask_chunk()
+    src, edit = torch.from_numpy(m.src).to(dev()), torch.from_numpy(m.edit).to(dev())
+    mask = cca.cca_token_mask_l2(src, edit, prune_quantile=m.prune_quantile)
+    idx, n = cca.cca_compact(mask)
+    q, kc, vc = bf(c1.q[0]), bf(c1.k_cur[0]), bf(c1.v_cur[0])
+    o_c = cca.cca_chunk_attn(c1_ring, q, kc, vc, q_idx=idx, n_q_dev=n, n_q_max=1620)
+    two_pass = bf(m.o_cache)
+    cca.cca_scatter(o_c, idx, n, two_pass, n_max=1620)
+    fused = bf(m.o_cache)
+    cca.cca_chunk_attn_scatter(c1_ring, q, kc, vc, idx, fused, n_q_dev=n, n_q_max=1620)
+    torch.cuda.synchronize()
+    check_status(c1_ring)
+    assert torch.equal(fused, two_pass)
+    m_ref, _, _ = omask.token_mask(m.src, m.edit, prune_quantile=m.prune_quantile)
+    assert np.array_equal(to_np(fused)[m_ref == 0], m.o_cache[m_ref == 0])
+
+
+def test_fused_scatter_fp8_and_empty():
+    s = synth.fp8_720p(n_steps=1)
+    m = synth.mask_chunk()
+    ring = cca.KVRing(s.n_heads, s.head_dim, s.chunk_len, s.window, dtype="e4m3", device=dev())
+    for t in range(s.t):
+        ring.append(bf(s.ring_k[t]), bf(s.ring_v[t]))
+    mask = cca.cca_token_mask_l2(torch.from_numpy(m.src).to(dev()), torch.from_numpy(m.edit).to(dev()),
+                                 prune_quantile=m.prune_quantile)
+    idx, n = cca.cca_compact(mask)
+    q8, qs = cca.cca_quant_e4m3(bf(s.q[0]))
+    k8, ks = cca.cca_quant_e4m3(bf(s.k_cur[0]))
+    v8, vs = cca.cca_quant_e4m3(bf(s.v_cur[0]))
+    o_c = cca.cca_chunk_attn(ring, q8, k8, v8, q_scale=qs, kcur_scale=ks, vcur_scale=vs, q_idx=idx, n_q_dev=n,
+                             n_q_max=s.chunk_len)
+    two_pass = torch.zeros((s.chunk_len, s.n_heads, s.head_dim), dtype=torch.bfloat16, device=dev())
+    cca.cca_scatter(o_c, idx, n, two_pass, n_max=s.chunk_len)
+    fused = torch.zeros_like(two_pass)
+    cca.cca_chunk_attn_scatter(ring, q8, k8, v8, idx, fused, q_scale=qs, kcur_scale=ks, vcur_scale=vs, n_q_dev=n,
+                               n_q_max=s.chunk_len)
+    # empty active set: the cache is left as it is
+    keep = torch.full_like(two_pass, 3.0)
+    n0 = torch.zeros(1, dtype=torch.int32, device=dev())
+    cca.cca_chunk_attn_scatter(ring, q8, k8, v8, idx, keep, q_scale=qs, kcur_scale=ks, vcur_scale=vs, n_q_dev=n0,
+                               n_q_max=s.chunk_len)
+    torch.cuda.synchronize()
+    check_status(ring)
+    assert torch.equal(fused, two_pass)
+    assert (keep == 3.0).all()
+
+
 def test_mask_cached_full_and_empty_masks(c1, c1_ring, c1_ref):
     q = bf(c1.q[0])
     full_idx = torch.arange(1620, dtype=torch.int32, device=dev())
