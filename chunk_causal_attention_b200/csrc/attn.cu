@@ -704,9 +704,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
         // p = 2^(x * scale_log2 - m_new), packed f32x2 FMAs, 4 packed partial sums,
         // 16-bit pairs stored to TMEM over the first 64 columns of S, 16 at a time.
-        // e4m3 + packed fp16 ex2: the V-scale ratio pf enters as log2(pf) in the
-        // exponent, so the fp16 result is P itself; its sum is divided by pf.
-        const float m_off = (kFp8 && kExpMode == 1) ? m_new - __log2f(pf) : m_new;
+        // e4m3: the V-scale ratio pf enters as log2(pf) in the exponent, so the
+        // exponential is already P * pf (the 16-bit PV operand); its sum is
+        // divided by pf.
+        const float m_off = kFp8 ? m_new - __log2f(pf) : m_new;
         const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_off, -m_off);
         // Rescale this row of O when the reference maximum moved (O of the
         // previous tile is complete: S of this tile was committed after it);
@@ -754,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               sums[c & 3] = f2_add(sums[c & 3], f2_pack(e0, e1));
               if constexpr (kFp8)
-                p16[c] = pack_f16x2(e0 * pf, e1 * pf);
+                p16[c] = pack_f16x2(e0, e1);
               else
                 p16[c] = pack_bf16x2(e0, e1);
             }
@@ -763,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float s_lo, s_hi;
         f2_unpack(f2_add(f2_add(sums[0], sums[1]), f2_add(sums[2], sums[3])), s_lo, s_hi);
-        const float tile_sum = (kFp8 && kExpMode == 1) ? (s_lo + s_hi) / pf : (s_lo + s_hi);
+        const float tile_sum = kFp8 ? (s_lo + s_hi) / pf : (s_lo + s_hi);
         l_sum = l_sum * alpha + tile_sum;
         m_ref = m_new;
         tmem_st_wait();
