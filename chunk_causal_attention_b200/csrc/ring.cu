@@ -306,12 +306,20 @@ __global__ void finalize_scale_kernel(unsigned *a, unsigned *b, int n) {
 
 static cca_status bulk_copy_pair(const uint8_t *k_src, const uint8_t *v_src, uint8_t *k_dst, uint8_t *v_dst,
                                  int64_t bytes, int32_t *dev_status, cudaStream_t st) {
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(append_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kBulkStages * kBulkPiece);
-  });
+  // The shared-memory limit is a per-device function attribute: set it once per device.
+  static std::mutex mu;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t attr_err = cudaGetDevice(&dev);
+  if (attr_err == cudaSuccess && (dev < 0 || dev >= 64)) return fail(CCA_ERR_UNSUPPORTED, "append: device %d", dev);
+  if (attr_err == cudaSuccess) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_set[dev]) {
+      attr_err = cudaFuncSetAttribute(append_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kBulkStages * kBulkPiece);
+      attr_set[dev] = attr_err == cudaSuccess;
+    }
+  }
   if (attr_err != cudaSuccess) return fail(CCA_ERR_CUDA, "append: %s", cudaGetErrorString(attr_err));
   const int64_t n_pieces = 2 * ((bytes + kBulkPiece - 1) / kBulkPiece);
   const int grid = static_cast<int>(cca_min64(num_sms(), n_pieces));
