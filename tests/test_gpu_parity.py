@@ -150,6 +150,25 @@ def test_mask_fixed_tau_tiny_bit_exact():
     assert np.allclose(d2.cpu().numpy(), d_ref ** 2, rtol=1e-6)
 
 
+@pytest.mark.parametrize("n_tok,n_ch", [(0, 16), (1, 4), (1621, 4), (777, 64), (300, 256)])
+def test_mask_fixed_tau_channel_counts(n_tok, n_ch):
+    """Fixed-tau mask for every supported channel count class and ragged token
+    counts (0 included), against the oracle, with the ambiguity guard."""
+    g = np.random.default_rng(n_tok * 7 + n_ch)
+    src = g.standard_normal((n_tok, n_ch)).astype(np.float32)
+    edit = (src + g.normal(0.0, 0.5, size=(n_tok, n_ch))).astype(np.float32)
+    tau = float(np.sqrt(0.25 * n_ch)) * 1.01
+    m_ref, d_ref, _ = omask.token_mask(src, edit, tau=tau)
+    if n_tok:
+        _ambiguity_guard(d_ref ** 2, tau ** 2)
+    mask = torch.full((max(n_tok, 1),), 9, dtype=torch.uint8, device=dev())[:n_tok]
+    cca.cca_token_mask_l2(torch.from_numpy(src).to(dev()), torch.from_numpy(edit).to(dev()), tau=tau, mask=mask)
+    idx, n = cca.cca_compact(mask)
+    torch.cuda.synchronize()
+    assert np.array_equal(mask.cpu().numpy(), m_ref)
+    assert n.item() == int(m_ref.sum())
+
+
 def test_mask_identical_latents_all_inactive():
     s = synth.tiny()
     src = torch.from_numpy(s.src).to(dev())
@@ -199,7 +218,7 @@ def test_mask_dynamic_tau_and_compaction_bit_exact():
     assert abs(tau_out.item() - tau) <= 1e-5 * tau
 
 
-@pytest.mark.parametrize("n_tok,p", [(1, 0.5), (17, 0.3), (16384, 0.05), (16385, 0.9), (65536, 0.3),
+@pytest.mark.parametrize("n_tok,p", [(0, 0.5), (1, 0.5), (17, 0.3), (16384, 0.05), (16385, 0.9), (65536, 0.3),
                                      (65537, 0.3), (100000, 0.3), (8192 * 37 + 5, 0.5), (8192 * 1000, 0.0),
                                      (8192 * 1000 + 1, 1.0), ((1 << 22) + 3, 0.01), ((1 << 26) + 17, 0.3)])
 def test_compaction_ragged_sizes(n_tok, p):
@@ -281,10 +300,13 @@ def test_attention_tiny_stream(n_chunks):
         assert_attn_close(outs[t], ref, what=f"tiny chunk {t}")
 
 
-@pytest.mark.parametrize("D,L,H,W", [(64, 200, 3, 2), (128, 300, 2, 1), (128, 129, 1, 0), (64, 1, 2, 3)])
+@pytest.mark.parametrize("D,L,H,W", [(64, 200, 3, 2), (128, 300, 2, 1), (128, 129, 1, 0), (64, 1, 2, 3),
+                                     (64, 72, 2, 15)])
 def test_attention_ragged_shapes(D, L, H, W):
+    """Ragged chunk lengths, both head dims, no window, one-token chunks and the
+    largest window (W = 15, 17 visible chunks) with eviction."""
     g = np.random.default_rng(D * 1000 + L)
-    n = W + 3
+    n = W + 3 if W < 15 else 20
     q = [synth.bf16_round(g.standard_normal((L, H, D)).astype(np.float32)) for _ in range(n)]
     k = [synth.bf16_round(g.standard_normal((L, H, D)).astype(np.float32)) for _ in range(n)]
     v = [synth.bf16_round(g.standard_normal((L, H, D)).astype(np.float32)) for _ in range(n)]
