@@ -660,40 +660,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (lane == 0 && (warp & 3) == 0) CCA_TRACE_EV(10 + 10 * wg, g);
         tc_fence_after();
+        // Scores in two 64-column halves: the second half's TMEM load is in flight
+        // while the first half is masked and reduced.  Row maximum: 8 independent
+        // 3-input max chains, then a short tree.
         float x[128];
+        float mx;
         {
-          uint32_t u0[32], u1[32], u2[32], u3[32];
+          float acc[8];
+          uint32_t u0[32], u1[32];
           tmem_ld32(tS + 0, u0);
           tmem_ld32(tS + 32, u1);
-          tmem_ld32(tS + 64, u2);
-          tmem_ld32(tS + 96, u3);
           tmem_ld_wait32(u0);
           tmem_ld_wait32(u1);
-          tmem_ld_wait32(u2);
-          tmem_ld_wait32(u3);
+          uint32_t u2[32], u3[32];
+          tmem_ld32(tS + 64, u2);
+          tmem_ld32(tS + 96, u3);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             x[c] = __uint_as_float(u0[c]);
             x[32 + c] = __uint_as_float(u1[c]);
-            x[64 + c] = __uint_as_float(u2[c]);
-            x[96 + c] = __uint_as_float(u3[c]);
           }
-        }
-        if (valid < kBN) {
+          if (valid < 64) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= valid) x[c] = -INFINITY;
-        }
-        // Row maximum: 8 independent 3-input max chains, then a short tree.
-        float mx;
-        {
-          float acc[8];
+            for (int c = 0; c < 64; ++c)
+              if (c >= valid) x[c] = -INFINITY;
+          }
 #pragma unroll
           for (int k = 0; k < 8; ++k) acc[k] = x[k];
 #pragma unroll
-          for (int c = 8; c < 128; c += 16) {
+          for (int c = 8; c < 64; c += 16) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = fmax3(acc[k], x[c + k], x[c + 8 + k > 127 ? 127 : c + 8 + k]);
+            for (int k = 0; k < 8; ++k) acc[k] = fmax3(acc[k], x[c + k], x[c + 8 + k > 63 ? 63 : c + 8 + k]);
+          }
+          tmem_ld_wait32(u2);
+          tmem_ld_wait32(u3);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            x[64 + c] = __uint_as_float(u2[c]);
+            x[96 + c] = __uint_as_float(u3[c]);
+          }
+          if (valid < kBN) {
+#pragma unroll
+            for (int c = 64; c < 128; ++c)
+              if (c >= valid) x[c] = -INFINITY;
+          }
+#pragma unroll
+          for (int c = 64; c < 128; c += 16) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = fmax3(acc[k], x[c + k], x[c + 8 + k]);
           }
           mx = fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
         }
