@@ -142,7 +142,22 @@ def test_call_validation_without_device_work(L):
     assert L.cca_quant_e4m3(vp(0x1000), cca.CCA_BF16, 4, 2, 80, vp(0x1000), vp(0x1000), None) == 1
     assert L.cca_kv_append(h, None, vp(0x1000), cca.CCA_BF16, None) == 1
     assert L.cca_kv_append(h, vp(0x1000), vp(0x1000), cca.CCA_E4M3, None) == 1
-    L.cca_kv_ring_destroy(h)
+    # workspace queries and the allocation-free variant: argument errors come first
+    sz = ctypes.c_size_t()
+    assert L.cca_chunk_attn_workspace_size(None, 16, ctypes.byref(sz)) == 1
+    assert L.cca_chunk_attn_workspace_size(h, 17, ctypes.byref(sz)) == 1
+    assert L.cca_chunk_attn_workspace_size(h, 16, None) == 1
+    assert L.cca_chunk_attn_noalloc(None, vp(0x1000), vp(0x1000), vp(0x1000), None, None, None, None, None, 16,
+                                    0.0, vp(0x1000), None) == 1
+    assert L.cca_chunk_attn_noalloc(h, vp(0x1000), vp(0x1000), vp(0x1000), None, None, None, None, None, 17,
+                                    0.0, vp(0x1000), None) == 1
+    assert L.cca_compact_workspace_size(-1, ctypes.byref(sz)) == 1
+    # ring bookkeeping calls reject bad handles and counts
+    assert L.cca_kv_ring_restore(h, -1) == 1
+    assert L.cca_kv_ring_restore(None, 3) == 1
+    assert L.cca_kv_ring_reset(None) == 1
+    assert L.cca_kv_ring_query(None, None, None, None, None) == 1
+    assert L.cca_kv_ring_destroy(h) == 0
 
 
 def test_product_path_has_no_cpu_fallback():
