@@ -13,7 +13,6 @@ small owner of the ring's device buffers around ``cca_kv_ring_*``.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 from typing import Optional
 
@@ -372,7 +371,3 @@ def cca_selftest_bounded_wait(status: torch.Tensor, budget_cycles: int, arrive_f
     """Run the bounded-wait self-test; status (int32[1], device) gets CCA_DEV_*."""
     _check(lib().cca_selftest_bounded_wait(_ptr(status, "status", torch.int32), int(budget_cycles),
                                            1 if arrive_first else 0, _stream(stream)), "cca_selftest_bounded_wait")
-
-
-def default_scale(head_dim: int) -> float:
-    return 1.0 / math.sqrt(head_dim)

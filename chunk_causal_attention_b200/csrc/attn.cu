@@ -654,7 +654,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sl2 = a.scale_log2, pf = 1.f;
         if constexpr (kFp8) {
           sl2 *= s_q * chunk_scale(a.k_scale, a.kcur_scale, slot, a.H, head);
-          pf = chunk_scale(a.v_scale, a.vcur_scale, slot, a.H, head) / s_vmax;
+          // Floored at 2^-100 so that a zero V scale (all values of that chunk
+          // zero) still gives finite exponentials whose sum is the sum of P: their
+          // 16-bit PV operand rounds to zero, which is the chunk's exact share.
+          pf = fmaxf(chunk_scale(a.v_scale, a.vcur_scale, slot, a.H, head) / s_vmax, 0x1p-100f);
         }
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], g & 1, abort_flag, budget));
         if (!ok) break;
@@ -1210,25 +1213,17 @@ namespace cca {
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB per GPU that loads the library
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the scratch array on the current device, looked up once
-// per device.  In host code the array's name is only a stand-in, never a
-// device address, so it must go through cudaGetSymbolAddress.
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a stand-in, never a device address, so it goes
+// through cudaGetSymbolAddress, which allocates nothing.  It is looked up on
+// every call rather than cached: after a device reset the library's device
+// code is loaded again and the array may sit elsewhere.
 static cca_status noalloc_scratch(void **out) {
-  static std::mutex mu;
-  static void *addr[64] = {nullptr};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "cca_chunk_attn_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= 64) return fail(CCA_ERR_UNSUPPORTED, "cca_chunk_attn_noalloc: device index %d", dev);
-  std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(CCA_ERR_CUDA, "cca_chunk_attn_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-    addr[dev] = p;
-  }
-  *out = addr[dev];
+  void *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(CCA_ERR_CUDA, "cca_chunk_attn_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+  *out = p;
   return CCA_OK;
 }
 

@@ -152,7 +152,8 @@ cca_status cca_quant_e4m3(const void *x, cca_dtype src_dtype, int32_t n_tok,
  *
  *  q, k_cur, v_cur: device [L][H][D] in the ring's dtype (BF16, or E4M3 codes
  *      with per-head scales q_scale / kcur_scale / vcur_scale, device [H]
- *      fp32; the scale pointers must be NULL for BF16).
+ *      fp32; the scale pointers must be NULL for BF16).  Scales must be finite
+ *      and >= 0; a zero scale means all values of that head are zero.
  *  q_idx: NULL (queries are rows 0 .. n_q-1 of q) or device int32 row indices
  *      into q (the compacted active tokens of the mask cache).
  *  n_q_dev: NULL (n_q = n_q_max) or device int32 holding n_q <= n_q_max; read
@@ -209,9 +210,12 @@ cca_status cca_chunk_attn_workspace_size(const cca_kv_ring *ring, int32_t n_q_ma
  * workspace: the split-KV partial results go to a 64 MiB array compiled into
  * this library, which every GPU that loads the library holds until the
  * process exits.
- *  - No cudaMalloc, cudaFree or other allocating call is made.  The first call
- *    on each device looks the array's device address up once
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - No cudaMalloc, cudaFree or other allocating call is made.  Every call
+ *    looks the array's device address up with cudaGetSymbolAddress (which
+ *    allocates nothing).  The first call on a device also makes the CUDA
+ *    runtime load this library's device code there, which places the array
+ *    and can stall the stream once: make one warm-up call on each device
+ *    before a real-time loop starts, and before any stream capture.
  *  - All calls share the one array and it keeps the last call's contents
  *    (nothing in it needs to start at zero).  Calls that may overlap on the
  *    GPU (different streams, or different host threads) race on it: serialise

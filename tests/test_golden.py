@@ -1,4 +1,4 @@
-"""The oracle still reproduces its frozen outputs (tests/golden/README.md)."""
+"""The oracle still reproduces the outputs frozen by tests/golden/make_golden.py."""
 import json
 import os
 import sys

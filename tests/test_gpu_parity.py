@@ -50,13 +50,42 @@ def half_ulp_bf16(x):
     return np.ldexp(1.0, e - 1 - 8)
 
 
+_RECORD = None
+
+
+@pytest.fixture(autouse=True)
+def _record_errors(record_property):
+    """Every attention comparison records its raw errors (junit properties, and
+    one JSON line per comparison in $CCA_PARITY_LOG when that is set)."""
+    global _RECORD
+    _RECORD = record_property
+    yield
+    _RECORD = None
+
+
+def _log_errors(what, ma, excess, rl, max_abs, rel_l2):
+    if _RECORD is not None:
+        _RECORD(f"{what}|max_abs", ma)
+        _RECORD(f"{what}|max_abs_beyond_bf16_rounding", excess)
+        _RECORD(f"{what}|rel_l2", rl)
+    path = os.environ.get("CCA_PARITY_LOG")
+    if path:
+        import json
+        with open(path, "a") as f:
+            f.write(json.dumps({"what": what, "max_abs": ma, "max_abs_beyond_bf16_rounding": excess,
+                                "rel_l2": rl, "bar_max_abs": max_abs, "bar_rel_l2": rel_l2}) + "\n")
+
+
 def assert_attn_close(got, ref, max_abs=BF16_MAX_ABS, rel_l2=BF16_REL_L2, what=""):
     """Element-wise |got - ref| <= max_abs on top of the bf16 output rounding
-    (half an ulp of bf16 at |ref|), and relative L2 over the tensor <= rel_l2."""
+    (half an ulp of bf16 at |ref|), and relative L2 over the tensor <= rel_l2.
+    The raw max-abs, the part beyond the output rounding and the relative L2
+    are recorded for every call."""
     got = np.asarray(got, dtype=np.float64)
     d = np.abs(got - ref)
     excess = float((d - half_ulp_bf16(ref)).max())
     ma, rl = err(got, ref)
+    _log_errors(what or "attention", ma, excess, rl, max_abs, rel_l2)
     assert excess <= max_abs and rl <= rel_l2, f"{what}: max_abs={ma:.3e} (beyond bf16 rounding {excess:.3e}) rel_l2={rl:.3e}"
     return ma, rl
 
@@ -551,6 +580,41 @@ def test_attention_fp8_ragged_stream_with_eviction():
         ref = _fp8_stream_ref(k, v, q[t], k[t], v[t], t, W)
         assert_attn_close(to_np(o), ref, FP8_MAX_ABS, FP8_REL_L2, what=f"fp8 ragged t={t}")
         ring.append(bf(k[t]), bf(v[t]))
+    check_status(ring)
+
+
+def test_attention_fp8_zero_and_tiny_v_scales():
+    """Caller-supplied V scales far apart: a zero scale for the current chunk
+    (its values are all zero, its keys still take part in the softmax) and a
+    ring chunk whose V scale is 2^-30 of its own absmax scale.  The result is
+    the dequantised attention, finite everywhere."""
+    g = np.random.default_rng(37)
+    L, H, D, W = 200, 2, 128, 2
+    draw = lambda: synth.bf16_round(g.standard_t(4.0, size=(L, H, D)).astype(np.float32))
+    k = [draw() for _ in range(4)]
+    v = [draw() for _ in range(4)]
+    q = draw()
+    ring = cca.KVRing(H, D, L, W, dtype="e4m3", device=dev())
+    for t in range(3):
+        ring.append(bf(k[t]), bf(v[t]))
+    _, slots, ids = ring.query()
+    assert ids == [0, 1, 2]
+    ring.v_scale[slots[1]] *= 2.0 ** -30
+    q8, qs = cca.cca_quant_e4m3(bf(q))
+    k8, ks = cca.cca_quant_e4m3(bf(k[3]))
+    v8, vs = cca.cca_quant_e4m3(bf(v[3]))
+    o = cca.cca_chunk_attn(ring, q8, k8, v8, q_scale=qs, kcur_scale=ks, vcur_scale=torch.zeros_like(vs))
+
+    def deq(x, f=1.0):
+        codes, sc = ofp8.quantize_per_head(x)
+        return ofp8.dequantize_per_head(codes, sc.astype(np.float64) * f)
+
+    past_k = {c: deq(k[c]) for c in range(3)}
+    past_v = {0: deq(v[0]), 1: deq(v[1], 2.0 ** -30), 2: deq(v[2])}
+    ref = oca.chunk_attention(deq(q), past_k, past_v, 3, W, k_cur=deq(k[3]), v_cur=deq(v[3], 0.0))
+    got = to_np(o)
+    assert np.all(np.isfinite(got))
+    assert_attn_close(got, ref, FP8_MAX_ABS, FP8_REL_L2, what="fp8 zero / tiny V scales")
     check_status(ring)
 
 

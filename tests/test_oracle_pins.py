@@ -320,6 +320,57 @@ def test_head_scales_and_dequant_error():
     assert np.all(np.abs(xh - x)[big] <= np.abs(x)[big] * 2.0 ** -4 * 1.0001)
 
 
+def _absmax_uses_full_range(quantize):
+    """What the e4m3fn format fixes for an absmax scale: in every non-zero head
+    the largest magnitude lands on the largest finite code (0x7E = 448), no code
+    exceeds it, and an all-zero head gives only zero codes.  `quantize` maps
+    x [n, H, D] to (codes, scale)."""
+    g = np.random.default_rng(31)
+    heads = [g.standard_normal((300, 4, 32)), g.standard_t(4.0, size=(300, 4, 32)),
+             g.uniform(-1e-3, 1e-3, size=(300, 4, 32)), g.standard_t(1.5, size=(300, 4, 32)) * 1e3]
+    for x in heads:
+        x = x.astype(np.float32)
+        x[:, 2] = 0.0
+        codes, _ = quantize(x)
+        mag = codes & 0x7F
+        if np.any(mag > 0x7E):
+            return False
+        for h in range(x.shape[1]):
+            xh, ch = np.abs(x[:, h]), mag[:, h]
+            if not xh.any():
+                if np.any(ch != 0):
+                    return False
+                continue
+            if not np.all(ch[xh == xh.max()] == 0x7E):
+                return False
+    return True
+
+
+def test_head_scales_pin_absmax_encodes_to_largest_code():
+    assert _absmax_uses_full_range(fp8.quantize_per_head)
+
+
+def test_planted_scale_divisor_240_is_caught():
+    def planted(x):  # the e4m3fnuz maximum (240) as divisor: the range is left unused
+        amax = np.abs(x).max(axis=(0, 2))
+        s = np.where(amax > 0, (amax / np.float32(240.0)).astype(np.float32), np.float32(1.0)).astype(np.float32)
+        y = (x / s[None, :, None]).astype(np.float32)
+        return fp8.e4m3_encode(y.astype(np.float64)), s
+    assert not _absmax_uses_full_range(planted)
+
+
+def test_head_scale_of_power_of_two_range_is_exact():
+    # absmax = 448 * 2^k gives s = 2^k exactly, and grid values times s come back unchanged
+    grid = fp8.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    for k in (-12, -3, 0, 5):
+        x = np.zeros((grid.size, 1, 2), dtype=np.float32)
+        x[:, 0, 0] = (grid * 2.0 ** k).astype(np.float32)
+        x[:, 0, 1] = -x[:, 0, 0]
+        codes, s = fp8.quantize_per_head(x)
+        assert s[0] == np.float32(2.0 ** k)
+        assert np.array_equal(fp8.dequantize_per_head(codes, s), x.astype(np.float64))
+
+
 # --------------------------------------------------------------- planted mistakes
 def _vis_no_sink(t, window):
     return [c for c in ca.visible_chunks(t, window) if c != 0 or t == 0]
