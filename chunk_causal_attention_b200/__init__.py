@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "CCA_BF16", "CCA_E4M3", "CCA_F32", "CcaError", "KVRing", "lib", "lib_path", "EXPORTED",
     "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc",
-    "cca_chunk_attn_scatter",
+    "cca_chunk_attn_scatter", "cca_attn_workspace_size", "cca_chunk_attn_groups", "cca_block_attn",
     "cca_token_mask_l2", "cca_compact", "cca_compact_workspace_size", "cca_scatter", "cca_selftest_bounded_wait",
     "cca_version",
     "cca_take_launch_count",
@@ -36,7 +36,8 @@ _STATUS = {0: "CCA_OK", 1: "CCA_ERR_INVALID_ARG", 2: "CCA_ERR_UNSUPPORTED", 3: "
 EXPORTED = (
     "cca_kv_ring_create", "cca_kv_ring_destroy", "cca_kv_ring_reset", "cca_kv_ring_query",
     "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn",
-    "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_chunk_attn_scatter", "cca_token_mask_l2", "cca_compact",
+    "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_chunk_attn_scatter", "cca_attn_workspace_size",
+    "cca_chunk_attn_groups", "cca_block_attn", "cca_token_mask_l2", "cca_compact",
     "cca_compact_workspace_size",
     "cca_scatter", "cca_selftest_bounded_wait", "cca_last_error", "cca_version", "cca_take_launch_count",
 )
@@ -52,6 +53,17 @@ class _RingDesc(ctypes.Structure):
     _fields_ = [("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("chunk_len", ctypes.c_int32),
                 ("window", ctypes.c_int32), ("dtype", ctypes.c_int), ("k_slots", ctypes.c_void_p),
                 ("v_slots", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
+                ("dev_status", ctypes.c_void_p)]
+
+
+class _BlockDesc(ctypes.Structure):
+    _fields_ = [("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("chunk_len", ctypes.c_int32),
+                ("n_chunks", ctypes.c_int32), ("window", ctypes.c_int32), ("dtype", ctypes.c_int),
+                ("k_cur", ctypes.c_void_p), ("v_cur", ctypes.c_void_p), ("k_hist", ctypes.c_void_p),
+                ("v_hist", ctypes.c_void_p), ("k_ref", ctypes.c_void_p), ("v_ref", ctypes.c_void_p),
+                ("ref_len", ctypes.c_int32),
+                ("kcur_scale", ctypes.c_void_p), ("vcur_scale", ctypes.c_void_p), ("khist_scale", ctypes.c_void_p),
+                ("vhist_scale", ctypes.c_void_p), ("kref_scale", ctypes.c_void_p), ("vref_scale", ctypes.c_void_p),
                 ("dev_status", ctypes.c_void_p)]
 
 
@@ -85,6 +97,9 @@ def lib() -> ctypes.CDLL:
         "cca_chunk_attn_workspace_size": [vp, i32, ctypes.POINTER(sz)],
         "cca_chunk_attn_noalloc": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp],
         "cca_chunk_attn_scatter": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp],
+        "cca_attn_workspace_size": [i32, ctypes.POINTER(sz)],
+        "cca_chunk_attn_groups": [vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, f32, vp, vp, sz, vp],
+        "cca_block_attn": [ctypes.POINTER(_BlockDesc), vp, vp, f32, vp, vp, sz, vp],
         "cca_token_mask_l2": [vp, vp, i32, i32, f32, f32, vp, vp, vp, vp],
         "cca_compact": [vp, i32, vp, vp, vp, sz, vp],
         "cca_compact_workspace_size": [i32, ctypes.POINTER(sz)],
@@ -311,6 +326,74 @@ def cca_chunk_attn_noalloc(ring: KVRing, q: torch.Tensor, k_cur: torch.Tensor, v
                                         _ptr(n_q_dev, "n_q_dev", torch.int32), int(n_q_max), float(softmax_scale),
                                         _ptr(out, "out", torch.bfloat16), _stream(stream)),
            "cca_chunk_attn_noalloc")
+    return out
+
+
+def cca_attn_workspace_size(head_dim: int) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().cca_attn_workspace_size(int(head_dim), ctypes.byref(out)), "cca_attn_workspace_size")
+    return int(out.value)
+
+
+def _workspace(workspace, head_dim, device):
+    need = cca_attn_workspace_size(head_dim)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def cca_chunk_attn_groups(ring: KVRing, q: torch.Tensor, k_cur: torch.Tensor, v_cur: torch.Tensor,
+                          k_ref: Optional[torch.Tensor] = None, v_ref: Optional[torch.Tensor] = None,
+                          q_scale=None, kcur_scale=None, vcur_scale=None, kref_scale=None, vref_scale=None,
+                          softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One denoising step of the active chunk's token groups (N_t, S_t, C_t packed
+    as the n_cur rows of q / k_cur / v_cur) over R (k_ref / v_ref, optional), the
+    ring's sink and window, and the block itself.  Returns out [n_cur, H, D] bf16."""
+    n_cur = q.shape[0]
+    if tuple(k_cur.shape) != tuple(q.shape) or tuple(v_cur.shape) != tuple(q.shape):
+        raise ValueError("q, k_cur and v_cur must have the same shape [n_cur, H, D]")
+    n_ref = 0 if k_ref is None else k_ref.shape[0]
+    if out is None:
+        out = torch.empty((n_cur, ring.n_heads, ring.head_dim), dtype=torch.bfloat16, device=q.device)
+    workspace, ws_bytes = _workspace(workspace, ring.head_dim, q.device)
+    _check(lib().cca_chunk_attn_groups(ring.handle, _ptr(q, "q"), _ptr(k_cur, "k_cur"), _ptr(v_cur, "v_cur"),
+                                       int(n_cur), _ptr(k_ref, "k_ref"), _ptr(v_ref, "v_ref"), int(n_ref),
+                                       _ptr(q_scale, "q_scale"), _ptr(kcur_scale, "kcur_scale"),
+                                       _ptr(vcur_scale, "vcur_scale"), _ptr(kref_scale, "kref_scale"),
+                                       _ptr(vref_scale, "vref_scale"), float(softmax_scale),
+                                       _ptr(out, "out", torch.bfloat16), _ptr(workspace, "workspace"), ws_bytes,
+                                       _stream(stream)), "cca_chunk_attn_groups")
+    return out
+
+
+def cca_block_attn(q: torch.Tensor, k_cur: torch.Tensor, v_cur: torch.Tensor, window: int,
+                   k_hist: Optional[torch.Tensor] = None, v_hist: Optional[torch.Tensor] = None,
+                   k_ref: Optional[torch.Tensor] = None, v_ref: Optional[torch.Tensor] = None,
+                   q_scale=None, kcur_scale=None, vcur_scale=None, khist_scale=None, vhist_scale=None,
+                   kref_scale=None, vref_scale=None, softmax_scale: float = 0.0,
+                   out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Packed block-causal forward: q / k_cur / v_cur [T, L, H, D]; chunk c attends
+    to R, history chunks {0} U {max(1, c-W) .. c-1} (k_hist / v_hist, default the
+    current tensors) and itself.  Returns out [T, L, H, D] bf16."""
+    T, L, H, D = q.shape
+    fp8 = q.dtype == torch.uint8
+    if k_hist is None:
+        k_hist, v_hist, khist_scale, vhist_scale = k_cur, v_cur, kcur_scale, vcur_scale
+    if out is None:
+        out = torch.empty((T, L, H, D), dtype=torch.bfloat16, device=q.device)
+    workspace, ws_bytes = _workspace(workspace, D, q.device)
+    d = _BlockDesc(H, D, L, T, int(window), CCA_E4M3 if fp8 else CCA_BF16,
+                   _ptr(k_cur, "k_cur"), _ptr(v_cur, "v_cur"), _ptr(k_hist, "k_hist"), _ptr(v_hist, "v_hist"),
+                   _ptr(k_ref, "k_ref"), _ptr(v_ref, "v_ref"), 0 if k_ref is None else int(k_ref.shape[0]),
+                   _ptr(kcur_scale, "kcur_scale"), _ptr(vcur_scale, "vcur_scale"),
+                   _ptr(khist_scale, "khist_scale"), _ptr(vhist_scale, "vhist_scale"),
+                   _ptr(kref_scale, "kref_scale"), _ptr(vref_scale, "vref_scale"),
+                   _ptr(status, "status", torch.int32))
+    _check(lib().cca_block_attn(ctypes.byref(d), _ptr(q, "q"), _ptr(q_scale, "q_scale"), float(softmax_scale),
+                                _ptr(out, "out", torch.bfloat16), _ptr(workspace, "workspace"), ws_bytes,
+                                _stream(stream)), "cca_block_attn")
     return out
 
 

@@ -40,7 +40,10 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
+#include <initializer_list>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "ring.cuh"
@@ -54,7 +57,6 @@ constexpr int kNQ = 2;         // Q tiles per work item
 constexpr int kNSK = 3;        // K pipeline stages
 constexpr int kNSV = 2;        // V pipeline stages
 constexpr int kThreads = 384;  // 12 warps
-constexpr int kMaxVis = kMaxWindow + 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
 // Pairs of score columns whose exponential runs on the FMA pipe (polynomial)
 // instead of the MUFU unit: bit k set = pair k of every 8 pairs (2 of 8 here).
@@ -100,24 +102,47 @@ __device__ unsigned long long g_trace[4 << 14];
   } while (0)
 #endif
 
+// KV sources of one launch: 0 = the ring (or the packed clean history), 1 = the
+// current block (or the packed current chunks), 2 = a globally visible group
+// (the reference tokens R).  Each is a [slots][rows][H][D] tensor.
+constexpr int kMaxSrc = 3;
+constexpr int kMaxProb = 32;   // query blocks ("problems") per launch
+constexpr int kMaxSegs = 192;  // visible KV segments over all problems of a launch
+
+// One block of queries with its own list of visible KV segments.  A segment is
+// one slot of one source, all of its rows.  Items of a problem are (query
+// pair, head); all have the same KV tile count n_kv.  The host lists problems
+// by non-increasing n_kv.
+struct AttnProb {
+  int32_t n_q;        // queries of this problem (problem 0: overridden by *n_q_dev)
+  int16_t q_slot;     // slot of the Q tensor holding them (rows 0 .. n_q-1)
+  int16_t out_slot;   // slot of the output tensor
+  int16_t seg0, n_seg;
+  int32_t n_kv;       // KV tiles per item = sum over its segments
+};
+
 struct AttnArgs {
-  const void *q;           // query rows (gather path): [L][H][D] of the ring's element type
+  const void *q;           // query rows (gather path): [rows][H][D] of the ring's element type
   const int32_t *q_idx;    // NULL: dense rows
-  const int32_t *n_q_dev;  // NULL: n_q = n_q_max
-  __nv_bfloat16 *out;      // [n_q_max][H][D], or [L][H][D] with scatter_out
+  const int32_t *n_q_dev;  // NULL: problem 0 has prob[0].n_q queries
+  __nv_bfloat16 *out;      // [slots][out_rows][H][D], or [out_rows][H][D] rows q_idx[i] with scatter_out
   int scatter_out;         // 1: query i's row goes to out row q_idx[i] (fused scatter-back)
   float *ws_o;             // [2 x grid][256][D] partial O of split items (unnormalised)
   float *ws_ml;            // [2 x grid][256][2] (running max in log2 units, row sum)
   int32_t *dev_status;
-  // e4m3 only: per-head dequantisation scales of Q, of the current chunk's K/V
-  // ([H]) and of the ring slots' K/V ([(1+W)][H]).
-  const float *q_scale, *kcur_scale, *vcur_scale, *k_scale, *v_scale;
-  int n_q_max, L, H;
-  int tiles_per_chunk, n_kv_tiles;
+  // e4m3 only: per-head dequantisation scales, [slots][H] per tensor.
+  const float *q_scale;
+  const float *k_scale[kMaxSrc], *v_scale[kMaxSrc];
+  int out_rows;            // rows per output slot (scatter: rows of the cache)
+  int q_rows;              // rows of the gathered Q tensor (gather path)
+  int H;
   float scale_log2;
   long long wait_budget;
-  int n_vis;               // visible chunks, the current one last
-  uint64_t slots_packed;   // 4-bit ring slot of visible chunk c at bits [4c, 4c+4)
+  int src_len[kMaxSrc];    // rows per slot of each source
+  int n_prob;
+  AttnProb prob[kMaxProb];
+  uint16_t seg[kMaxSegs];     // (source << 12) | slot
+  uint16_t seg_t0[kMaxSegs];  // first KV tile of the segment in its problem's list
 };
 
 // Shared-memory plan.  Q/K/V tiles arrive by TMA as 128-row x 128-byte boxes
@@ -140,74 +165,180 @@ struct AttnSmem {
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
-// KV tile j of the visible list -> (ring slot or -1 for the current chunk, first row).
-__device__ __forceinline__ void kv_tile_coords(const AttnArgs &a, int j, int &slot, int &row0) {
-  const int c = j / a.tiles_per_chunk;
-  row0 = (j - c * a.tiles_per_chunk) * kBN;
-  slot = c == a.n_vis - 1 ? -1 : static_cast<int>((a.slots_packed >> (4 * c)) & 15u);
-}
-
-__device__ __forceinline__ int vis_slot(const AttnArgs &a, int c) {
-  return c == a.n_vis - 1 ? -1 : static_cast<int>((a.slots_packed >> (4 * c)) & 15u);
-}
-
 // ---- work schedule (identical in every role, the combine kernel included)
-// Items are (query pair, head), head-major (so CTAs running together share a
-// head's K/V in L2), for the pairs holding the first n_q queries.  With G CTAs: CTA c takes items c, c + G, ... for q = items / G full
-// rounds; the r = items % G remaining items form a list of r * n_kv KV tiles cut
-// into G near-equal ranges, so CTA c also takes 0, 1 or 2 partial segments.
-// Partial segment k (0 or 1) of CTA c writes workspace slot 2c + k.
+// Items are (problem, query pair, head), problem-major and head-major inside a
+// problem (so CTAs running together share a head's K/V in L2), for the query
+// pairs holding each problem's queries.  With G CTAs, CTA c first takes whole
+// items in rounds, item k*G + c in even rounds and k*G + G-1-c in odd ones
+// (so that rounds of unequal items even out).  When the items left after the
+// full rounds would unbalance the CTAs (one of them more than 1/8 of the
+// average load), their KV tiles are concatenated into one list cut into G
+// near-equal ranges instead: CTA c then takes the pieces of [c*tr/G,
+// (c+1)*tr/G).  A piece that covers only part of its item is "partial": its
+// (O, m, l) go to workspace slot 2c (the piece holding the range's first tile)
+// or 2c+1 (the one holding its last tile), and the combine kernel merges them.
 struct Sched {
-  int n_items, q, r, n_pairs;  // n_pairs: query pairs holding the first n_q queries
-  int64_t tr;                  // KV tiles in the remainder list
+  int n_items, qr;  // items; whole rounds
+  int rem0;         // first item of the split remainder (n_items if none)
+  int64_t tr;       // KV tiles in the remainder list (0: no split)
 };
 struct Seg {
-  int pair, head, j0, j1, slot;  // slot < 0: whole item, direct output
+  int prob, pair, head, j0, j1, slot;  // slot < 0: whole item, direct output
 };
 
-__device__ __forceinline__ Sched make_sched(int n_q, int H, int n_kv, int G) {
+__device__ __forceinline__ int prob_nq(const AttnArgs &a, int p, int n_q0) { return p == 0 ? n_q0 : a.prob[p].n_q; }
+__device__ __forceinline__ int prob_pairs(const AttnArgs &a, int p, int n_q0) {
+  return (prob_nq(a, p, n_q0) + kNQ * kBM - 1) / (kNQ * kBM);
+}
+
+__device__ __forceinline__ Sched make_sched(const AttnArgs &a, int n_q0, int G) {
   Sched s;
-  s.n_pairs = (n_q + kNQ * kBM - 1) / (kNQ * kBM);
-  s.n_items = s.n_pairs * H;
-  s.q = s.n_items / G;
-  s.r = s.n_items % G;
-  s.tr = static_cast<int64_t>(s.r) * n_kv;
+  int n = 0;
+  int64_t total = 0;
+  for (int p = 0; p < a.n_prob; ++p) {
+    const int cnt = prob_pairs(a, p, n_q0) * a.H;
+    n += cnt;
+    total += static_cast<int64_t>(cnt) * a.prob[p].n_kv;
+  }
+  s.n_items = n;
+  const int q = n / G, r = n % G;
+  s.qr = q;
+  s.rem0 = q * G;
+  s.tr = 0;
+  if (r > 0) {
+    // longest remainder item (problems are listed by non-increasing n_kv)
+    int i0 = 0, nkv_first = 0;
+    int64_t tr = 0;
+    for (int p = 0; p < a.n_prob; ++p) {
+      const int cnt = prob_pairs(a, p, n_q0) * a.H, i1 = i0 + cnt;
+      const int b0 = i0 > s.rem0 ? i0 : s.rem0;
+      if (b0 < i1) {
+        if (tr == 0) nkv_first = a.prob[p].n_kv;
+        tr += static_cast<int64_t>(i1 - b0) * a.prob[p].n_kv;
+      }
+      i0 = i1;
+    }
+    if (static_cast<int64_t>(nkv_first) * 8 * G > total) {
+      s.tr = tr;
+    } else {  // the leftover items are short next to a CTA's load: one more round of whole items
+      s.qr = q + 1;
+      s.rem0 = n;
+    }
+  }
   return s;
 }
 
-__device__ __forceinline__ bool get_seg(const Sched &s, int n_kv, int G, int c, int k, Seg &g) {
-  const int P = s.n_pairs > 0 ? s.n_pairs : 1;
-  if (k < s.q) {
-    const int u = c + k * G;
-    g = {u % P, u / P, 0, n_kv, -1};
-    return true;
+// Item u -> (problem, pair, head).
+__device__ __forceinline__ void item_coords(const AttnArgs &a, int n_q0, int u, int &p, int &pair, int &head) {
+  for (p = 0; p + 1 < a.n_prob; ++p) {
+    const int cnt = prob_pairs(a, p, n_q0) * a.H;
+    if (u < cnt) break;
+    u -= cnt;
   }
-  k -= s.q;
-  const int64_t lo = static_cast<int64_t>(c) * s.tr / G, hi = static_cast<int64_t>(c + 1) * s.tr / G;
-  if (lo >= hi || k > 1) return false;
-  const int64_t u0 = lo / n_kv;
-  if (k == 0) {
-    const int u = s.q * G + static_cast<int>(u0);
-    const int64_t e0 = hi < (u0 + 1) * n_kv ? hi : (u0 + 1) * n_kv;
-    g = {u % P, u / P, static_cast<int>(lo - u0 * n_kv), static_cast<int>(e0 - u0 * n_kv), 2 * c};
-    return true;
-  }
-  if (hi <= (u0 + 1) * n_kv) return false;
-  const int u = s.q * G + static_cast<int>(u0) + 1;
-  g = {u % P, u / P, 0, static_cast<int>(hi - (u0 + 1) * n_kv), 2 * c + 1};
-  return true;
+  const int np = max(prob_pairs(a, p, n_q0), 1);
+  pair = u % np;
+  head = u / np;
 }
 
-// Dequantisation scale of chunk (slot) for one head: ring slot or current chunk.
-__device__ __forceinline__ float chunk_scale(const float *ring, const float *cur, int slot, int H, int head) {
-  return slot < 0 ? __ldg(cur + head) : __ldg(ring + slot * H + head);
+// Remainder item holding tile offset t of the remainder list: its index, first
+// tile offset and tile count.
+__device__ __forceinline__ void rem_locate(const AttnArgs &a, int n_q0, const Sched &s, int64_t t, int &u,
+                                           int64_t &ustart, int &ulen) {
+  int i0 = 0;
+  int64_t acc = 0;
+  for (int p = 0; p < a.n_prob; ++p) {
+    const int cnt = prob_pairs(a, p, n_q0) * a.H, i1 = i0 + cnt;
+    const int b0 = i0 > s.rem0 ? i0 : s.rem0;
+    const int nkv = a.prob[p].n_kv;
+    if (b0 < i1) {
+      const int64_t span = static_cast<int64_t>(i1 - b0) * nkv;
+      if (t < acc + span || p == a.n_prob - 1) {
+        const int k = static_cast<int>((t - acc) / nkv);
+        u = b0 + k;
+        ustart = acc + static_cast<int64_t>(k) * nkv;
+        ulen = nkv;
+        return;
+      }
+      acc += span;
+    }
+    i0 = i1;
+  }
+  u = s.n_items;
+  ustart = acc;
+  ulen = 1;
+}
+
+// The k-th segment of work of CTA c (false when there is none).
+__device__ __forceinline__ bool get_seg(const AttnArgs &a, int n_q0, const Sched &s, int G, int c, int k, Seg &g) {
+  if (k < s.qr) {
+    const int u = k * G + ((k & 1) ? G - 1 - c : c);
+    if (u >= s.rem0) return false;  // only in the last round of an unsplit schedule
+    int p, pair, head;
+    item_coords(a, n_q0, u, p, pair, head);
+    g = {p, pair, head, 0, a.prob[p].n_kv, -1};
+    return true;
+  }
+  if (s.tr == 0) return false;
+  k -= s.qr;
+  const int64_t lo = static_cast<int64_t>(c) * s.tr / G, hi = static_cast<int64_t>(c + 1) * s.tr / G;
+  int64_t t = lo;
+  for (int piece = 0; t < hi; ++piece) {
+    int u, ulen;
+    int64_t ustart;
+    rem_locate(a, n_q0, s, t, u, ustart, ulen);
+    const int64_t e = hi < ustart + ulen ? hi : ustart + ulen;
+    if (piece == k) {
+      int p, pair, head;
+      item_coords(a, n_q0, u, p, pair, head);
+      const bool whole = t == ustart && e == ustart + ulen;
+      g = {p, pair, head, static_cast<int>(t - ustart), static_cast<int>(e - ustart),
+           whole ? -1 : (t == lo ? 2 * c : 2 * c + 1)};
+      return true;
+    }
+    t = e;
+  }
+  return false;
+}
+
+// Walks the KV tiles of one item in order: tile j -> segment k (its source
+// and slot are a.seg[k]), first row and valid rows.  Segments are visited in
+// order, so a step costs O(1); the cursor holds three registers.
+struct TileCursor {
+  int k;     // current segment
+  int t1;    // first tile after it
+  int vend;  // 128 * (its first tile) + its rows: valid rows of tile j = vend - 128 j
+};
+__device__ __forceinline__ void cursor_begin(const AttnArgs &a, int p, TileCursor &cu) {
+  cu.k = a.prob[p].seg0 - 1;
+  cu.t1 = 0;
+  cu.vend = 0;
+}
+__device__ __forceinline__ void cursor_at(const AttnArgs &a, int p, TileCursor &cu, int j, int &row0, int &valid) {
+  while (j >= cu.t1) {
+    ++cu.k;
+    const int t0 = a.seg_t0[cu.k];
+    cu.vend = t0 * kBN + a.src_len[a.seg[cu.k] >> 12];
+    const AttnProb &P = a.prob[p];
+    cu.t1 = cu.k + 1 < P.seg0 + P.n_seg ? static_cast<int>(a.seg_t0[cu.k + 1]) : P.n_kv;
+  }
+  const int v = cu.vend - j * kBN;
+  valid = v < kBN ? v : kBN;
+  row0 = a.src_len[a.seg[cu.k] >> 12] - v;
+}
+__device__ __forceinline__ int cursor_src(const AttnArgs &a, const TileCursor &cu) { return a.seg[cu.k] >> 12; }
+__device__ __forceinline__ int cursor_slot(const AttnArgs &a, const TileCursor &cu) { return a.seg[cu.k] & 0xFFF; }
+
+// Dequantisation scale of a K or V segment for one head.
+__device__ __forceinline__ float seg_scale(const float *const *tab, int src, int slot, int H, int head) {
+  return __ldg(tab[src] + slot * H + head);
 }
 
 template <int D, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kr,
-                const __grid_constant__ CUtensorMap tm_vr, const __grid_constant__ CUtensorMap tm_kc,
-                const __grid_constant__ CUtensorMap tm_vc, const AttnArgs a) {
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k0,
+                const __grid_constant__ CUtensorMap tm_v0, const __grid_constant__ CUtensorMap tm_k1,
+                const __grid_constant__ CUtensorMap tm_v1, const __grid_constant__ CUtensorMap tm_k2,
+                const __grid_constant__ CUtensorMap tm_v2, const __grid_constant__ AttnArgs a) {
   using namespace sm100;
   using S = AttnSmem<D, kFp8>;
   static_assert(!kFp8 || D == 128, "e4m3 path is built for head_dim 128");
@@ -238,8 +369,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The combine grid (a programmatic dependent) may be scheduled from now on; it
   // waits for this grid's completion before it reads anything.
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int n_q = a.n_q_dev ? min(max(*a.n_q_dev, 0), a.n_q_max) : a.n_q_max;
-  const Sched sch = make_sched(n_q, a.H, a.n_kv_tiles, gridDim.x);
+  const int n_q0 = a.n_q_dev ? min(max(*a.n_q_dev, 0), a.prob[0].n_q) : a.prob[0].n_q;
+  const Sched sch = make_sched(a, n_q0, gridDim.x);
+  auto kmap = [&](int src) { return src == 0 ? &tm_k0 : src == 1 ? &tm_k1 : &tm_k2; };
+  auto vmap = [&](int src) { return src == 0 ? &tm_v0 : src == 1 ? &tm_v1 : &tm_v2; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -267,10 +400,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     if (!a.q_idx) prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_kr);
-    prefetch_tmap(&tm_vr);
-    prefetch_tmap(&tm_kc);
-    prefetch_tmap(&tm_vc);
+    prefetch_tmap(&tm_k0);
+    prefetch_tmap(&tm_v0);
+    prefetch_tmap(&tm_k1);
+    prefetch_tmap(&tm_v1);
+    if (a.src_len[2] > 0) {
+      prefetch_tmap(&tm_k2);
+      prefetch_tmap(&tm_v2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -294,8 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
-      if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      if (!get_seg(a, n_q0, sch, gridDim.x, blockIdx.x, kseg, sg)) break;
       const int pair = sg.pair, head = sg.head, j0 = sg.j0, j1 = sg.j1;
+      const int q_slot = a.prob[sg.prob].q_slot;
+      const int n_q = prob_nq(a, sg.prob, n_q0);
       for (int i = 0; i < kNQ && ok; ++i) {
         if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[i], (it - 1) & 1, abort_flag, budget));
         if (!ok) break;
@@ -305,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             mbar_arrive_expect_tx(&q_full[i], S::kTile);
             for (uint32_t b = 0; b < S::kNBox; ++b)
-              tma_load_3d(&tm_q, &q_full[i], dstq + b * S::kBox, b * kBoxElems, head, row0);
+              tma_load_4d(&tm_q, &q_full[i], dstq + b * S::kBox, b * kBoxElems, head, row0, q_slot);
           }
         } else {
           // Gather: row r of the tile is query q_idx[row0 + r], copied with
@@ -320,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 4; ++k) {
             const int qr = row0 + lane + 32 * k;
             int sr = qr < n_q ? __ldg(a.q_idx + qr) : -1;
-            if (qr < n_q && (sr < 0 || sr >= a.L)) {
+            if (qr < n_q && (sr < 0 || sr >= a.q_rows)) {
               if (a.dev_status) *a.dev_status = CCA_DEV_BAD_INDEX;  // out-of-range index: row read as zeros
               sr = -1;
             }
@@ -347,10 +486,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       q_armed = it + 1;
+      TileCursor cu;
+      cursor_begin(a, sg.prob, cu);
       for (int j = j0; j < j1; ++j, ++g) {
         const uint32_t stage = g % kNSK, ph = (g / kNSK) & 1;
-        int slot, row0;
-        kv_tile_coords(a, j, slot, row0);
+        int row0, valid;
+        cursor_at(a, sg.prob, cu, j, row0, valid);
+        const int src = cursor_src(a, cu), slot = cursor_slot(a, cu);
         if (g >= kNSK) ok = __all_sync(0xffffffffu, mbar_wait(&k_empty[stage], ph ^ 1, abort_flag, budget));
         if (!ok) break;
         ++gk;
@@ -358,12 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t dst = base + S::kK + stage * S::kTile;
           CCA_TRACE_EV(30, g);
           mbar_arrive_expect_tx(&k_full[stage], S::kTile);
-          for (uint32_t b = 0; b < S::kNBox; ++b) {
-            if (slot < 0)
-              tma_load_3d(&tm_kc, &k_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0);
-            else
-              tma_load_4d(&tm_kr, &k_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
-          }
+          for (uint32_t b = 0; b < S::kNBox; ++b)
+            tma_load_4d(kmap(src), &k_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
         }
         if constexpr (kFp8) {
           // e4m3: V tiles come from this warp too; the expanders free a V slot as
@@ -375,12 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             const uint32_t dst = base + S::kV + vst * S::kTile;
             mbar_arrive_expect_tx(&v_full[vst], S::kTile);
-            for (uint32_t b = 0; b < S::kNBox; ++b) {
-              if (slot < 0)
-                tma_load_3d(&tm_vc, &v_full[vst], dst + b * S::kBox, b * kBoxElems, head, row0);
-              else
-                tma_load_4d(&tm_vr, &v_full[vst], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
-            }
+            for (uint32_t b = 0; b < S::kNBox; ++b)
+              tma_load_4d(vmap(src), &v_full[vst], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
           }
         }
       }
@@ -470,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
-      if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      if (!get_seg(a, n_q0, sch, gridDim.x, blockIdx.x, kseg, sg)) break;
       const int j0 = sg.j0, j1 = sg.j1;
       const int n = j1 - j0;
       ok = wait(&q_full[0], it & 1) && wait(&q_full[1], it & 1);
@@ -538,23 +672,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
-      if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      if (!get_seg(a, n_q0, sch, gridDim.x, blockIdx.x, kseg, sg)) break;
+      TileCursor cu;
+      cursor_begin(a, sg.prob, cu);
       for (int j = sg.j0; j < sg.j1; ++j, ++g) {
         const uint32_t stage = g % kNSV, ph = (g / kNSV) & 1;
-        int slot, row0;
-        kv_tile_coords(a, j, slot, row0);
+        int row0, valid;
+        cursor_at(a, sg.prob, cu, j, row0, valid);
+        const int src = cursor_src(a, cu), slot = cursor_slot(a, cu);
         if (g >= kNSV) ok = __all_sync(0xffffffffu, mbar_wait(&v_empty[stage], ph ^ 1, abort_flag, budget));
         if (!ok) break;
         ++gv;
         if (lane == 0) {
           const uint32_t dst = base + S::kV + stage * S::kTile;
           mbar_arrive_expect_tx(&v_full[stage], S::kTile);
-          for (uint32_t b = 0; b < S::kNBox; ++b) {
-            if (slot < 0)
-              tma_load_3d(&tm_vc, &v_full[stage], dst + b * S::kBox, b * kBoxElems, sg.head, row0);
-            else
-              tma_load_4d(&tm_vr, &v_full[stage], dst + b * S::kBox, b * kBoxElems, sg.head, row0, slot);
-          }
+          for (uint32_t b = 0; b < S::kNBox; ++b)
+            tma_load_4d(vmap(src), &v_full[stage], dst + b * S::kBox, b * kBoxElems, sg.head, row0, slot);
         }
       }
     }
@@ -576,7 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int kseg = 0; ok; ++kseg) {
         Seg sg;
-        if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+        if (!get_seg(a, n_q0, sch, gridDim.x, blockIdx.x, kseg, sg)) break;
         for (int j = sg.j0; j < sg.j1; ++j, ++g) {
           const uint32_t stage = g % kNSV, ph = (g / kNSV) & 1;
           ok = __all_sync(0xffffffffu, mbar_wait(&v_full[stage], ph, abort_flag, budget));
@@ -633,31 +766,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
-      if (!get_seg(sch, a.n_kv_tiles, gridDim.x, blockIdx.x, kseg, sg)) break;
+      if (!get_seg(a, n_q0, sch, gridDim.x, blockIdx.x, kseg, sg)) break;
       const int pair = sg.pair, head = sg.head, j0 = sg.j0, j1 = sg.j1;
+      const AttnProb &P = a.prob[sg.prob];
+      const int n_q = prob_nq(a, sg.prob, n_q0);
       // e4m3: scores carry the factor s_q * s_k(chunk); V's factor s_v(chunk) is
       // folded into P relative to the largest s_v of the visible chunks, which
       // the epilogue multiplies back.
       float s_q = 1.f, s_vmax = 1.f;
       if constexpr (kFp8) {
-        s_q = __ldg(a.q_scale + head);
+        s_q = __ldg(a.q_scale + P.q_slot * a.H + head);
         s_vmax = 0.f;
-        for (int c = 0; c < a.n_vis; ++c)
-          s_vmax = fmaxf(s_vmax, chunk_scale(a.v_scale, a.vcur_scale, vis_slot(a, c), a.H, head));
+        for (int k = P.seg0; k < P.seg0 + P.n_seg; ++k)
+          s_vmax = fmaxf(s_vmax, seg_scale(a.v_scale, a.seg[k] >> 12, a.seg[k] & 0xFFF, a.H, head));
         if (!(s_vmax > 0.f)) s_vmax = 1.f;
       }
       float m_ref = -INFINITY, l_sum = 0.f;
+      TileCursor cu;
+      cursor_begin(a, sg.prob, cu);
       for (int j = j0; j < j1; ++j, ++g) {
-        int slot, row0;
-        kv_tile_coords(a, j, slot, row0);
-        const int valid = min(kBN, a.L - row0);
+        int row0, valid;
+        cursor_at(a, sg.prob, cu, j, row0, valid);
+        (void)row0;
         float sl2 = a.scale_log2, pf = 1.f;
         if constexpr (kFp8) {
-          sl2 *= s_q * chunk_scale(a.k_scale, a.kcur_scale, slot, a.H, head);
+          const int src = cursor_src(a, cu), slot = cursor_slot(a, cu);
+          sl2 *= s_q * seg_scale(a.k_scale, src, slot, a.H, head);
           // Floored at 2^-100 so that a zero V scale (all values of that chunk
           // zero) still gives finite exponentials whose sum is the sum of P: their
           // 16-bit PV operand rounds to zero, which is the chunk's exact share.
-          pf = fmaxf(chunk_scale(a.v_scale, a.vcur_scale, slot, a.H, head) / s_vmax, 0x1p-100f);
+          pf = fmaxf(seg_scale(a.v_scale, src, slot, a.H, head) / s_vmax, 0x1p-100f);
         }
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], g & 1, abort_flag, budget));
         if (!ok) break;
@@ -799,8 +937,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (sg.slot < 0) {
         const float inv = s_vmax / l_sum;
         const int orow = a.scatter_out && row_ok ? __ldg(a.q_idx + row) : row;
-        const bool wr_ok = row_ok && orow >= 0 && orow < (a.scatter_out ? a.L : a.n_q_max);
-        __nv_bfloat16 *dst = a.out + (static_cast<int64_t>(wr_ok ? orow : 0) * a.H + head) * D;
+        const bool wr_ok = row_ok && orow >= 0 && orow < a.out_rows;
+        __nv_bfloat16 *dst =
+            a.out + ((static_cast<int64_t>(P.out_slot) * a.out_rows + (wr_ok ? orow : 0)) * a.H + head) * D;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -856,44 +995,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && *abort_flag && a.dev_status) atomicExch(a.dev_status, CCA_DEV_TIMEOUT);
 }
 
-// Merge of the partial segments of the split items: one warp per (item, row),
+// Merge of the partial pieces of the split items: one warp per (item, row),
 // out[row][head] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s over the CTAs
-// whose KV range meets the item.  The schedule is recomputed from n_q exactly as
-// the attention kernel (launched with G CTAs) computed it.  Lane i examines
-// candidate CTA c_first + i; the O rows of up to 8 found pieces are then loaded
-// by the whole warp at once (lane = D/32 columns) before they are summed, so a
-// row costs about two memory round trips.  Launched as a programmatic dependent
-// of the attention kernel: it is resident before the attention grid ends and
-// waits (griddepcontrol.wait) for that grid's memory before reading.
+// whose KV range meets the item.  The schedule is recomputed exactly as the
+// attention kernel (launched with G CTAs) computed it; items that fell whole
+// inside one CTA's range were written by that CTA and are skipped.  Lane i
+// examines candidate CTA c_first + i; the O rows of up to 8 found pieces are
+// then loaded by the whole warp at once (lane = D/32 columns) before they are
+// summed, so a row costs about two memory round trips.  Launched as a
+// programmatic dependent of the attention kernel: it is resident before the
+// attention grid ends and waits (griddepcontrol.wait) for that grid's memory
+// before reading.
+__device__ __forceinline__ int64_t rem_offset(const AttnArgs &a, int n_q0, const Sched &s, int u) {
+  int i0 = 0;
+  int64_t acc = 0;
+  for (int p = 0; p < a.n_prob; ++p) {
+    const int cnt = prob_pairs(a, p, n_q0) * a.H, i1 = i0 + cnt;
+    const int b0 = i0 > s.rem0 ? i0 : s.rem0;
+    const int e0 = i1 < u ? i1 : u;
+    if (b0 < e0) acc += static_cast<int64_t>(e0 - b0) * a.prob[p].n_kv;
+    i0 = i1;
+  }
+  return acc;
+}
+
 template <int D>
-__global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restrict__ ws_o,
-                                                           const float *__restrict__ ws_ml,
-                                                           const int32_t *__restrict__ n_q_dev, int n_q_max, int H,
-                                                           int n_kv, int G, __nv_bfloat16 *__restrict__ out,
-                                                           const int32_t *__restrict__ out_idx, int n_rows) {
+__global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ AttnArgs a, int G) {
   constexpr int kV = D / 32;  // columns per lane
   constexpr int kBatch = 8;   // pieces loaded at once
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int n_q = n_q_dev ? min(max(*n_q_dev, 0), n_q_max) : n_q_max;
-  const Sched sch = make_sched(n_q, H, n_kv, G);
-  if (sch.r == 0) return;
+  const int n_q0 = a.n_q_dev ? min(max(*a.n_q_dev, 0), a.prob[0].n_q) : a.prob[0].n_q;
+  const Sched sch = make_sched(a, n_q0, G);
+  if (sch.tr == 0) return;
   const int lane = threadIdx.x & 31;
-  const uint32_t tr = static_cast<uint32_t>(sch.tr), uG = static_cast<uint32_t>(G);
-  const int n_work = sch.r * (kNQ * kBM);
+  const int64_t tr = sch.tr;
+  const int n_work = (sch.n_items - sch.rem0) * (kNQ * kBM);
   const int w0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   for (int w = w0; w < n_work; w += nw) {
     const int ur = w / (kNQ * kBM), rr = w % (kNQ * kBM);
-    const int u = sch.q * G + ur, pair = u % sch.n_pairs, head = u / sch.n_pairs;
+    const int u = sch.rem0 + ur;
+    int p, pair, head;
+    item_coords(a, n_q0, u, p, pair, head);
     const int row = pair * (kNQ * kBM) + rr;
-    if (row >= n_q) continue;
-    const uint32_t t0 = static_cast<uint32_t>(ur) * n_kv, t1 = t0 + n_kv;  // the item's tiles in the list
-    const int c_first = static_cast<int>(((t0 + 1) * uG + tr - 1) / tr) - 1;
-    const int c_last = min(G - 1, static_cast<int>((t1 * uG + tr - 1) / tr));
+    if (row >= prob_nq(a, p, n_q0)) continue;
+    const int64_t t0 = rem_offset(a, n_q0, sch, u), t1 = t0 + a.prob[p].n_kv;  // the item's tiles in the list
+    const int c_first = static_cast<int>(((t0 + 1) * G + tr - 1) / tr) - 1;
+    const int c_last = min(G - 1, static_cast<int>((t1 * G + tr - 1) / tr));
+    {  // whole inside one CTA's range: written directly by that CTA
+      const int64_t lo = static_cast<int64_t>(c_first) * tr / G, hi = static_cast<int64_t>(c_first + 1) * tr / G;
+      if (lo <= t0 && hi >= t1) continue;
+    }
     auto probe = [&](int c, int &slot) {
       if (c > c_last) return false;
-      const uint32_t lo = static_cast<uint32_t>(c) * tr / uG, hi = static_cast<uint32_t>(c + 1) * tr / uG;
-      slot = 2 * c + (lo / n_kv == static_cast<uint32_t>(ur) ? 0 : 1);
+      const int64_t lo = static_cast<int64_t>(c) * tr / G, hi = static_cast<int64_t>(c + 1) * tr / G;
+      slot = 2 * c + (lo >= t0 ? 0 : 1);
       return lo < hi && hi > t0 && lo < t1;
     };
     // pass 1: (m, l) of every piece, one lane per candidate
@@ -901,7 +1057,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restri
     for (int cb = c_first; cb <= c_last; cb += 32) {
       int slot;
       if (probe(cb + lane, slot))
-        mmax = fmaxf(mmax, __ldcg(ws_ml + (static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2));
+        mmax = fmaxf(mmax, __ldcg(a.ws_ml + (static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
@@ -913,7 +1069,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restri
       const bool mine = probe(cb + lane, slot);
       float wgt = 0.f;
       if (mine) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(ws_ml + (static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2));
+        const float2 ml =
+            __ldcg(reinterpret_cast<const float2 *>(a.ws_ml + (static_cast<int64_t>(slot) * (kNQ * kBM) + rr) * 2));
         wgt = exp2f(ml.x - mmax);
         den += wgt * ml.y;
       }
@@ -928,7 +1085,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restri
           todo &= todo - 1;
           ws[b] = live ? __shfl_sync(0xffffffffu, wgt, src) : 0.f;
           const int sl = __shfl_sync(0xffffffffu, slot, src);
-          const float *o = ws_o + (static_cast<int64_t>(sl) * (kNQ * kBM) + rr) * D + lane * kV;
+          const float *o = a.ws_o + (static_cast<int64_t>(sl) * (kNQ * kBM) + rr) * D + lane * kV;
           if (live) {
             if constexpr (kV == 4) {
               const float4 v = __ldcg(reinterpret_cast<const float4 *>(o));
@@ -951,9 +1108,10 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float *__restri
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     const float inv = 1.f / den;
-    const int orow = out_idx ? __ldg(out_idx + row) : row;  // fused scatter-back
-    if (orow < 0 || orow >= n_rows) continue;               // bad index (flagged by the gather)
-    __nv_bfloat16 *dst = out + (static_cast<int64_t>(orow) * H + head) * D + lane * kV;
+    const int orow = a.scatter_out ? __ldg(a.q_idx + row) : row;  // fused scatter-back
+    if (orow < 0 || orow >= a.out_rows) continue;                 // bad index (flagged by the gather)
+    __nv_bfloat16 *dst =
+        a.out + ((static_cast<int64_t>(a.prob[p].out_slot) * a.out_rows + orow) * a.H + head) * D + lane * kV;
     if constexpr (kV == 4) {
       *reinterpret_cast<uint2 *>(dst) = make_uint2(sm100::pack_bf16x2(acc[0] * inv, acc[1] * inv),
                                                    sm100::pack_bf16x2(acc[2] * inv, acc[3] * inv));
@@ -977,81 +1135,149 @@ static PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   return fn;
 }
 
-// [rows][H][D] (rank 3) or [slots][rows][H][D] (rank 4) bf16/e4m3 tensor; box =
-// 128 bytes of D x 1 head x 128 rows (x 1 slot), 128-byte swizzle, zero fill.
+// [slots][rows][H][D] bf16/e4m3 tensor as a rank-4 map; box = 128 bytes of D x
+// 1 head x 128 rows x 1 slot, 128-byte swizzle, zero fill past the rows of a
+// slot.  Encoded maps are kept in a small per-thread cache keyed by everything
+// they depend on, so a stream loop that reuses its buffers encodes each once.
 static cca_status make_tmap(CUtensorMap *tm, const void *ptr, CUtensorMapDataType dt, int esize, int D, int H,
                             int rows, int slots) {
+  struct Entry {
+    const void *ptr;
+    int dt, D, H, rows, slots;
+    CUtensorMap map;
+  };
+  constexpr int kCache = 32;
+  thread_local Entry cache[kCache];
+  thread_local int n_cached = 0, next = 0;
+  for (int i = 0; i < n_cached; ++i) {
+    const Entry &e = cache[i];
+    if (e.ptr == ptr && e.dt == static_cast<int>(dt) && e.D == D && e.H == H && e.rows == rows &&
+        e.slots == slots) {
+      *tm = e.map;
+      return CCA_OK;
+    }
+  }
   auto enc = tmap_encoder();
   if (!enc) return fail(CCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  const int rank = slots > 0 ? 4 : 3;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(slots > 0 ? slots : 1)};
+                        static_cast<cuuint64_t>(slots)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * esize, static_cast<cuuint64_t>(H) * D * esize,
                            static_cast<cuuint64_t>(rows) * H * D * esize};
   cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / esize), 1, 128, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(tm, dt, rank, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  CUresult r = enc(tm, dt, 4, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CCA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  Entry &e = n_cached < kCache ? cache[n_cached++] : cache[next++ % kCache];
+  e = {ptr, static_cast<int>(dt), D, H, rows, slots, *tm};
   return CCA_OK;
 }
-
-struct AttnPlan {
-  int grid, tiles_per_chunk, n_kv_tiles, n_vis, max_items;
-  int32_t slots[kMaxVis];
-};
 
 static int env_int(const char *name, int dflt) {
   const char *s = std::getenv(name);
   return s && *s ? std::atoi(s) : dflt;
 }
 
-// Grid: one persistent CTA per SM (CCA_ATTN_CTAS overrides), never more CTAs
-// than KV tiles of work.
-static void plan_attention(const cca_kv_ring *ring, int n_q_max, AttnPlan &p) {
-  const cca_kv_ring_desc &d = ring->d;
-  p.n_vis = ring_visible(ring, p.slots, nullptr) + 1;  // cached chunks + the current chunk
-  p.tiles_per_chunk = (d.chunk_len + kBN - 1) / kBN;
-  p.n_kv_tiles = p.n_vis * p.tiles_per_chunk;
-  p.max_items = ((n_q_max + kNQ * kBM - 1) / (kNQ * kBM)) * d.n_heads;
+// One kernel launch: the arguments plus the tensors behind the maps.
+struct AttnLaunch {
+  AttnArgs args;
+  const void *q;  // Q tensor [q_slots][q_rows][H][D] (dense path)
+  int q_rows_map, q_slots;
+  const void *k[kMaxSrc], *v[kMaxSrc];
+  int src_slots[kMaxSrc];
+  int D;
+  bool fp8;
+  int64_t work;  // upper bound on (item, KV tile) pairs, for the grid size
+};
+
+// Persistent grid: one CTA per SM (CCA_ATTN_CTAS overrides), never more CTAs
+// than (item, KV tile) pairs of work.
+static int attn_grid(int64_t work) {
   int g = env_int("CCA_ATTN_CTAS", 0);
   if (g <= 0) g = num_sms();
-  const int64_t work = static_cast<int64_t>(p.max_items) * p.n_kv_tiles;
   if (work < g) g = static_cast<int>(work > 0 ? work : 1);
-  p.grid = g;
+  return g;
 }
 
-// Partial-segment slots: 2 per CTA, 256 rows each.
-static size_t workspace_bytes_for(const cca_kv_ring *ring, int n_q_max, const AttnPlan &p) {
-  if (n_q_max == 0) return 0;
-  const size_t rows = static_cast<size_t>(2) * p.grid * (kNQ * kBM);
-  return rows * (static_cast<size_t>(ring->d.head_dim) + 2) * sizeof(float) + 256;
+// Partial-piece slots: 2 per CTA, 256 rows each, O (D fp32) plus (m, l).
+static size_t workspace_bytes_for_grid(int grid, int D) {
+  const size_t rows = static_cast<size_t>(2) * grid * (kNQ * kBM);
+  return rows * (static_cast<size_t>(D) + 2) * sizeof(float) + 256;
 }
+
+// Workspace that suffices for every attention launch with this head_dim on
+// the current device (the grid never exceeds CCA_ATTN_CTAS or the SM count).
+static size_t workspace_bytes_any(int D) {
+  int g = env_int("CCA_ATTN_CTAS", 0);
+  if (g <= 0) g = num_sms();
+  return workspace_bytes_for_grid(g, D);
+}
+
+// Host copy of the device schedule's decision: does any item get split?
+static bool host_splits(const AttnArgs &a, int G) {
+  int n = 0;
+  int64_t total = 0;
+  for (int p = 0; p < a.n_prob; ++p) {
+    const int cnt = (a.prob[p].n_q + kNQ * kBM - 1) / (kNQ * kBM) * a.H;
+    n += cnt;
+    total += static_cast<int64_t>(cnt) * a.prob[p].n_kv;
+  }
+  const int q = n / G, r = n % G;
+  if (r == 0) return false;
+  int i0 = 0;
+  for (int p = 0; p < a.n_prob; ++p) {
+    const int cnt = (a.prob[p].n_q + kNQ * kBM - 1) / (kNQ * kBM) * a.H, i1 = i0 + cnt;
+    if (i1 > q * G) return static_cast<int64_t>(a.prob[p].n_kv) * 8 * G > total;
+    i0 = i1;
+  }
+  return false;
+}
+
+static std::mutex g_attr_mu;
 
 template <int D, bool kFp8>
-static cca_status launch_attn(const cca_kv_ring *ring, const AttnPlan &p, const AttnArgs &args, const void *q,
-                              const void *k_cur, const void *v_cur, cudaStream_t st) {
+static cca_status launch_attn(AttnLaunch &L, void *workspace, size_t workspace_bytes, cudaStream_t st) {
   using S = AttnSmem<D, kFp8>;
-  const cca_kv_ring_desc &d = ring->d;
+  AttnArgs &args = L.args;
+  const int H = args.H;
   const CUtensorMapDataType dt = kFp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int es = kFp8 ? 1 : 2;
-  CUtensorMap tq, tkr, tvr, tkc, tvc;
+  const int grid = attn_grid(L.work);
+  const size_t need = workspace_bytes_for_grid(grid, D);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(CCA_ERR_INVALID_ARG, "attention: workspace of %zu bytes (16-byte aligned) required", need);
+  args.ws_o = static_cast<float *>(workspace);
+  args.ws_ml = args.ws_o + static_cast<size_t>(2) * grid * (kNQ * kBM) * D;
+  CUtensorMap tq, tk[kMaxSrc], tv[kMaxSrc];
   std::memset(&tq, 0, sizeof(tq));
-  if (!args.q_idx) CCA_TRY(make_tmap(&tq, q, dt, es, D, d.n_heads, args.n_q_max, 0));
-  CCA_TRY(make_tmap(&tkr, d.k_slots, dt, es, D, d.n_heads, d.chunk_len, 1 + d.window));
-  CCA_TRY(make_tmap(&tvr, d.v_slots, dt, es, D, d.n_heads, d.chunk_len, 1 + d.window));
-  CCA_TRY(make_tmap(&tkc, k_cur, dt, es, D, d.n_heads, d.chunk_len, 0));
-  CCA_TRY(make_tmap(&tvc, v_cur, dt, es, D, d.n_heads, d.chunk_len, 0));
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(S::kAlloc));
-  if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "cca_chunk_attn: %s", cudaGetErrorString(e));
-  attn_kernel<D, kFp8><<<p.grid, kThreads, S::kAlloc, st>>>(tq, tkr, tvr, tkc, tvc, args);
+  if (!args.q_idx) CCA_TRY(make_tmap(&tq, L.q, dt, es, D, H, L.q_rows_map, L.q_slots));
+  for (int s = 0; s < kMaxSrc; ++s) {
+    // An unused source reuses source 1's tensor (never read: no segment names it).
+    const bool used = args.src_len[s] > 0;
+    const void *kp = used ? L.k[s] : L.k[1], *vp = used ? L.v[s] : L.v[1];
+    const int rows = used ? args.src_len[s] : args.src_len[1], slots = used ? L.src_slots[s] : L.src_slots[1];
+    CCA_TRY(make_tmap(&tk[s], kp, dt, es, D, H, rows, slots));
+    CCA_TRY(make_tmap(&tv[s], vp, dt, es, D, H, rows, slots));
+  }
+  {
+    // The shared-memory opt-in is per device and kernel: set it once per device.
+    static bool done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    if (dev < 0 || dev >= 64 || !done[dev]) {
+      const cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(S::kAlloc));
+      if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "attention: %s", cudaGetErrorString(e));
+      if (dev >= 0 && dev < 64) done[dev] = true;
+    }
+  }
+  attn_kernel<D, kFp8><<<grid, kThreads, S::kAlloc, st>>>(tq, tk[0], tv[0], tk[1], tv[1], tk[2], tv[2], args);
   CCA_TRY(launched("attn_kernel"));
-  // Split items exist unless the item count is known on the host and divides
-  // evenly over the grid.
-  const bool maybe_split = args.n_q_dev != nullptr || (p.max_items % p.grid) != 0;
-  if (maybe_split) {
-    const int64_t warps = static_cast<int64_t>(p.grid) * (kNQ * kBM);
+  // Split items exist unless the item count is known on the host and the
+  // schedule gives every item to one CTA.
+  if (args.n_q_dev != nullptr || host_splits(args, grid)) {
+    const int64_t warps = static_cast<int64_t>(grid) * (kNQ * kBM);
     int64_t blocks = (warps + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
@@ -1065,19 +1291,59 @@ static cca_status launch_attn(const cca_kv_ring *ring, const AttnPlan &p, const 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t le = cudaLaunchKernelEx(&cfg, attn_combine_kernel<D>, static_cast<const float *>(args.ws_o),
-                                              static_cast<const float *>(args.ws_ml), args.n_q_dev, args.n_q_max,
-                                              d.n_heads, p.n_kv_tiles, p.grid, args.out,
-                                              args.scatter_out ? args.q_idx : static_cast<const int32_t *>(nullptr),
-                                              args.scatter_out ? args.L : args.n_q_max);
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, attn_combine_kernel<D>, args, grid);
     if (le != cudaSuccess) {
       cudaGetLastError();
-      return fail(CCA_ERR_CUDA, "cca_chunk_attn: combine launch failed: %s", cudaGetErrorString(le));
+      return fail(CCA_ERR_CUDA, "attention: combine launch failed: %s", cudaGetErrorString(le));
     }
     CCA_TRY(launched("attn_combine_kernel"));
   }
   return CCA_OK;
 }
+
+static cca_status run_launch(AttnLaunch &L, void *workspace, size_t workspace_bytes, cudaStream_t st) {
+  if (L.fp8) return launch_attn<128, true>(L, workspace, workspace_bytes, st);
+  if (L.D == 128) return launch_attn<128, false>(L, workspace, workspace_bytes, st);
+  return launch_attn<64, false>(L, workspace, workspace_bytes, st);
+}
+
+// Builder of the problem / segment tables of one launch.
+struct LaunchBuilder {
+  AttnLaunch &L;
+  int n_seg = 0;
+  explicit LaunchBuilder(AttnLaunch &l) : L(l) {}
+  bool fits(int extra_segs) const { return L.args.n_prob < kMaxProb && n_seg + extra_segs <= kMaxSegs; }
+  // Start a problem; segments follow with add_seg.
+  void begin(int n_q, int q_slot, int out_slot) {
+    AttnProb &P = L.args.prob[L.args.n_prob];
+    P.n_q = n_q;
+    P.q_slot = static_cast<int16_t>(q_slot);
+    P.out_slot = static_cast<int16_t>(out_slot);
+    P.seg0 = static_cast<int16_t>(n_seg);
+    P.n_seg = 0;
+    P.n_kv = 0;
+  }
+  void add_seg(int src, int slot) {
+    AttnProb &P = L.args.prob[L.args.n_prob];
+    L.args.seg[n_seg] = static_cast<uint16_t>((src << 12) | slot);
+    L.args.seg_t0[n_seg] = static_cast<uint16_t>(P.n_kv);
+    P.n_kv += (L.args.src_len[src] + kBN - 1) / kBN;
+    ++P.n_seg;
+    ++n_seg;
+  }
+  void end() {
+    const AttnProb &P = L.args.prob[L.args.n_prob];
+    L.work += static_cast<int64_t>((P.n_q + kNQ * kBM - 1) / (kNQ * kBM)) * L.args.H * P.n_kv;
+    ++L.args.n_prob;
+  }
+};
+
+static float scale_log2_of(float softmax_scale, int D) {
+  const double scale = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(D));
+  return static_cast<float>(scale * 1.4426950408889634);  // scale * log2(e)
+}
+
+static long long wait_budget() { return static_cast<long long>(env_int("CCA_WAIT_BUDGET_MCYCLES", 4000)) * 1000000LL; }
 
 }  // namespace cca
 
@@ -1106,9 +1372,14 @@ int cca_debug_trace_read(unsigned long long *host, int max_n) {
 cca_status cca_chunk_attn_workspace_size(const cca_kv_ring *ring, int32_t n_q_max, size_t *bytes) {
   if (!ring || !bytes || n_q_max < 0 || n_q_max > ring->d.chunk_len)
     return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn_workspace_size: bad argument");
-  AttnPlan p;
-  plan_attention(ring, n_q_max, p);
-  *bytes = workspace_bytes_for(ring, n_q_max, p);
+  *bytes = n_q_max == 0 ? 0 : workspace_bytes_any(ring->d.head_dim);
+  return CCA_OK;
+}
+
+cca_status cca_attn_workspace_size(int32_t head_dim, size_t *bytes) {
+  if (!bytes || (head_dim != 64 && head_dim != 128))
+    return fail(CCA_ERR_INVALID_ARG, "cca_attn_workspace_size: head_dim must be 64 or 128");
+  *bytes = workspace_bytes_any(head_dim);
   return CCA_OK;
 }
 
@@ -1133,6 +1404,38 @@ cca_status cca_chunk_attn_scatter(const cca_kv_ring *ring, const void *q, const 
 
 }  // extern "C"
 
+// Common checks of the e4m3 scale pointers (all non-NULL, 4-byte aligned) or
+// their absence for BF16.
+static cca_status check_scales(const char *what, cca_dtype dt, std::initializer_list<const float *> sc) {
+  if (dt == CCA_E4M3) {
+    for (const float *p : sc) {
+      if (!p) return fail(CCA_ERR_INVALID_ARG, "%s: E4M3 needs every per-head scale", what);
+      if (reinterpret_cast<uintptr_t>(p) & 3) return fail(CCA_ERR_INVALID_ARG, "%s: scales must be 4-byte aligned", what);
+    }
+  } else {
+    for (const float *p : sc)
+      if (p) return fail(CCA_ERR_INVALID_ARG, "%s: BF16 takes no scales", what);
+  }
+  return CCA_OK;
+}
+
+// The ring's cached chunks visible from its current chunk, as segments of source 0.
+static void add_ring_segments(const cca_kv_ring *ring, LaunchBuilder &b) {
+  int32_t slots[kMaxWindow + 1];
+  const int n = ring_visible(ring, slots, nullptr);
+  for (int c = 0; c < n; ++c) b.add_seg(0, slots[c]);
+}
+
+static void init_launch(AttnLaunch &L, int H, int D, cca_dtype dt, float softmax_scale, int32_t *dev_status) {
+  std::memset(&L, 0, sizeof(L));
+  L.args.H = H;
+  L.D = D;
+  L.fp8 = dt == CCA_E4M3;
+  L.args.scale_log2 = scale_log2_of(softmax_scale, D);
+  L.args.wait_budget = wait_budget();
+  L.args.dev_status = dev_status;
+}
+
 static cca_status chunk_attn_impl(const cca_kv_ring *ring, const void *q, const void *k_cur, const void *v_cur,
                                   const float *q_scale, const float *kcur_scale, const float *vcur_scale,
                                   const int32_t *q_idx, const int32_t *n_q_dev, int32_t n_q_max,
@@ -1147,59 +1450,189 @@ static cca_status chunk_attn_impl(const cca_kv_ring *ring, const void *q, const 
     return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: q, k_cur, v_cur and out must be non-NULL");
   if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out))
     return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: q, k_cur, v_cur and out must be 16-byte aligned");
-  if (d.dtype == CCA_E4M3) {
-    if (!q_scale || !kcur_scale || !vcur_scale)
-      return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: E4M3 ring needs q/kcur/vcur scales");
-    const uintptr_t m = reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(kcur_scale) |
-                        reinterpret_cast<uintptr_t>(vcur_scale);
-    if (m & 3) return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: scales must be 4-byte aligned");
-    if (d.head_dim != 128)
-      return fail(CCA_ERR_UNSUPPORTED, "cca_chunk_attn: E4M3 attention is built for head_dim 128");
-  } else if (q_scale || kcur_scale || vcur_scale) {
-    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: BF16 ring takes no scales");
-  }
+  CCA_TRY(check_scales("cca_chunk_attn", d.dtype, {q_scale, kcur_scale, vcur_scale}));
+  if (d.dtype == CCA_E4M3 && d.head_dim != 128)
+    return fail(CCA_ERR_UNSUPPORTED, "cca_chunk_attn: E4M3 attention is built for head_dim 128");
   if ((q_idx && (reinterpret_cast<uintptr_t>(q_idx) & 3)) || (n_q_dev && (reinterpret_cast<uintptr_t>(n_q_dev) & 3)))
     return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: q_idx / n_q_dev must be 4-byte aligned");
-  AttnPlan p;
-  plan_attention(ring, n_q_max, p);
-  const size_t need = workspace_bytes_for(ring, n_q_max, p);
-  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
-    return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn: workspace of %zu bytes (16-byte aligned) required", need);
-  AttnArgs args;
-  std::memset(&args, 0, sizeof(args));
-  args.q = q;
-  args.q_scale = q_scale;
-  args.kcur_scale = kcur_scale;
-  args.vcur_scale = vcur_scale;
-  args.k_scale = d.k_scale;
-  args.v_scale = d.v_scale;
-  args.q_idx = q_idx;
-  args.n_q_dev = n_q_dev;
-  args.out = static_cast<__nv_bfloat16 *>(out);
-  args.scatter_out = scatter_out;
-  if (need > 0) {
-    args.ws_o = static_cast<float *>(workspace);
-    const size_t rows = static_cast<size_t>(2) * p.grid * (kNQ * kBM);
-    args.ws_ml = args.ws_o + rows * d.head_dim;
-  }
-  args.dev_status = d.dev_status;
-  args.n_q_max = n_q_max;
-  args.L = d.chunk_len;
-  args.H = d.n_heads;
-  args.tiles_per_chunk = p.tiles_per_chunk;
-  args.n_kv_tiles = p.n_kv_tiles;
-  const double scale = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(d.head_dim));
-  args.scale_log2 = static_cast<float>(scale * 1.4426950408889634);  // scale * log2(e)
-  args.wait_budget = static_cast<long long>(env_int("CCA_WAIT_BUDGET_MCYCLES", 4000)) * 1000000LL;
-  args.n_vis = p.n_vis;
-  args.slots_packed = 0;
-  for (int c = 0; c + 1 < p.n_vis; ++c) args.slots_packed |= static_cast<uint64_t>(p.slots[c] & 15) << (4 * c);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (d.dtype == CCA_E4M3) return launch_attn<128, true>(ring, p, args, q, k_cur, v_cur, st);
-  if (d.head_dim == 128) return launch_attn<128, false>(ring, p, args, q, k_cur, v_cur, st);
-  return launch_attn<64, false>(ring, p, args, q, k_cur, v_cur, st);
+  AttnLaunch L;
+  init_launch(L, d.n_heads, d.head_dim, d.dtype, softmax_scale, d.dev_status);
+  AttnArgs &a = L.args;
+  a.q = q;
+  a.q_idx = q_idx;
+  a.n_q_dev = n_q_dev;
+  a.out = static_cast<__nv_bfloat16 *>(out);
+  a.scatter_out = scatter_out;
+  a.q_scale = q_scale;
+  a.k_scale[0] = d.k_scale;
+  a.v_scale[0] = d.v_scale;
+  a.k_scale[1] = kcur_scale;
+  a.v_scale[1] = vcur_scale;
+  a.out_rows = scatter_out ? d.chunk_len : n_q_max;
+  a.q_rows = d.chunk_len;
+  a.src_len[0] = d.chunk_len;
+  a.src_len[1] = d.chunk_len;
+  L.q = q;
+  L.q_rows_map = n_q_max;
+  L.q_slots = 1;
+  L.k[0] = d.k_slots;
+  L.v[0] = d.v_slots;
+  L.src_slots[0] = 1 + d.window;
+  L.k[1] = k_cur;
+  L.v[1] = v_cur;
+  L.src_slots[1] = 1;
+  LaunchBuilder b(L);
+  b.begin(n_q_max, 0, 0);
+  add_ring_segments(ring, b);
+  b.add_seg(1, 0);
+  b.end();
+  return run_launch(L, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" {
+
+cca_status cca_chunk_attn_groups(const cca_kv_ring *ring, const void *q, const void *k_cur, const void *v_cur,
+                                 int32_t n_cur, const void *k_ref, const void *v_ref, int32_t n_ref,
+                                 const float *q_scale, const float *kcur_scale, const float *vcur_scale,
+                                 const float *kref_scale, const float *vref_scale, float softmax_scale, void *out,
+                                 void *workspace, size_t workspace_bytes, cca_stream_t stream) {
+  const char *what = "cca_chunk_attn_groups";
+  if (!ring) return fail(CCA_ERR_INVALID_ARG, "%s: NULL ring", what);
+  const cca_kv_ring_desc &d = ring->d;
+  if (n_cur < 0 || n_cur > (1 << 24) || n_ref < 0 || n_ref > (1 << 24))
+    return fail(CCA_ERR_INVALID_ARG, "%s: need 0 <= n_cur, n_ref <= 2^24", what);
+  if (n_cur == 0) return CCA_OK;
+  if (!q || !k_cur || !v_cur || !out || (n_ref > 0 && (!k_ref || !v_ref)))
+    return fail(CCA_ERR_INVALID_ARG, "%s: q, k_cur, v_cur, out (and k_ref, v_ref when n_ref > 0) must be non-NULL",
+                what);
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out) ||
+      (n_ref > 0 && (!aligned16(k_ref) || !aligned16(v_ref))))
+    return fail(CCA_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", what);
+  if (d.dtype == CCA_E4M3 && d.head_dim != 128)
+    return fail(CCA_ERR_UNSUPPORTED, "%s: E4M3 attention is built for head_dim 128", what);
+  CCA_TRY(check_scales(what, d.dtype, {q_scale, kcur_scale, vcur_scale}));
+  if (n_ref > 0) CCA_TRY(check_scales(what, d.dtype, {kref_scale, vref_scale}));
+  AttnLaunch L;
+  init_launch(L, d.n_heads, d.head_dim, d.dtype, softmax_scale, d.dev_status);
+  AttnArgs &a = L.args;
+  a.q = q;
+  a.out = static_cast<__nv_bfloat16 *>(out);
+  a.q_scale = q_scale;
+  a.k_scale[0] = d.k_scale;
+  a.v_scale[0] = d.v_scale;
+  a.k_scale[1] = kcur_scale;
+  a.v_scale[1] = vcur_scale;
+  a.k_scale[2] = kref_scale;
+  a.v_scale[2] = vref_scale;
+  a.out_rows = n_cur;
+  a.q_rows = n_cur;
+  a.src_len[0] = d.chunk_len;
+  a.src_len[1] = n_cur;
+  a.src_len[2] = n_ref;
+  L.q = q;
+  L.q_rows_map = n_cur;
+  L.q_slots = 1;
+  L.k[0] = d.k_slots;
+  L.v[0] = d.v_slots;
+  L.src_slots[0] = 1 + d.window;
+  L.k[1] = k_cur;
+  L.v[1] = v_cur;
+  L.src_slots[1] = 1;
+  L.k[2] = k_ref;
+  L.v[2] = v_ref;
+  L.src_slots[2] = 1;
+  LaunchBuilder b(L);
+  b.begin(n_cur, 0, 0);
+  if (n_ref > 0) b.add_seg(2, 0);
+  add_ring_segments(ring, b);
+  b.add_seg(1, 0);
+  b.end();
+  return run_launch(L, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+cca_status cca_block_attn(const cca_block_desc *bd, const void *q, const float *q_scale, float softmax_scale,
+                          void *out, void *workspace, size_t workspace_bytes, cca_stream_t stream) {
+  const char *what = "cca_block_attn";
+  if (!bd) return fail(CCA_ERR_INVALID_ARG, "%s: NULL descriptor", what);
+  const cca_block_desc &d = *bd;
+  const int T = d.n_chunks, Lc = d.chunk_len, W = d.window;
+  if (d.n_heads < 1 || (d.head_dim != 64 && d.head_dim != 128) || Lc < 1 || T < 0 || T > 4095 || W < 0 ||
+      d.ref_len < 0 || d.ref_len > (1 << 24) || (d.dtype != CCA_BF16 && d.dtype != CCA_E4M3) ||
+      static_cast<int64_t>(Lc) * d.n_heads * d.head_dim > (int64_t(1) << 33))
+    return fail(CCA_ERR_INVALID_ARG, "%s: bad dims (H >= 1, D in {64,128}, L >= 1, 0 <= T <= 4095, W >= 0)", what);
+  if (d.dtype == CCA_E4M3 && d.head_dim != 128)
+    return fail(CCA_ERR_UNSUPPORTED, "%s: E4M3 attention is built for head_dim 128", what);
+  if (T == 0) return CCA_OK;
+  if (!q || !out || !d.k_cur || !d.v_cur || !d.k_hist || !d.v_hist || (d.ref_len > 0 && (!d.k_ref || !d.v_ref)))
+    return fail(CCA_ERR_INVALID_ARG, "%s: NULL tensor", what);
+  const void *const tens[6] = {q, out, d.k_cur, d.v_cur, d.k_hist, d.v_hist};
+  for (const void *p : tens)
+    if (!aligned16(p)) return fail(CCA_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", what);
+  if (d.ref_len > 0 && (!aligned16(d.k_ref) || !aligned16(d.v_ref)))
+    return fail(CCA_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", what);
+  CCA_TRY(check_scales(what, d.dtype, {q_scale, d.kcur_scale, d.vcur_scale, d.khist_scale, d.vhist_scale}));
+  if (d.ref_len > 0) CCA_TRY(check_scales(what, d.dtype, {d.kref_scale, d.vref_scale}));
+  AttnLaunch base;
+  init_launch(base, d.n_heads, d.head_dim, d.dtype, softmax_scale, d.dev_status);
+  AttnArgs &a = base.args;
+  a.q = q;
+  a.out = static_cast<__nv_bfloat16 *>(out);
+  a.q_scale = q_scale;
+  a.k_scale[0] = d.khist_scale;
+  a.v_scale[0] = d.vhist_scale;
+  a.k_scale[1] = d.kcur_scale;
+  a.v_scale[1] = d.vcur_scale;
+  a.k_scale[2] = d.kref_scale;
+  a.v_scale[2] = d.vref_scale;
+  a.out_rows = Lc;
+  a.q_rows = Lc;
+  a.src_len[0] = Lc;
+  a.src_len[1] = Lc;
+  a.src_len[2] = d.ref_len;
+  base.q = q;
+  base.q_rows_map = Lc;
+  base.q_slots = T;
+  base.k[0] = d.k_hist;
+  base.v[0] = d.v_hist;
+  base.src_slots[0] = T;
+  base.k[1] = d.k_cur;
+  base.v[1] = d.v_cur;
+  base.src_slots[1] = T;
+  base.k[2] = d.k_ref;
+  base.v[2] = d.v_ref;
+  base.src_slots[2] = 1;
+  // Chunk c sees R, history chunks {0} U {max(1, c-W) .. c-1} and its own
+  // current chunk.  Chunks are listed longest visible list first (the schedule
+  // wants problems by non-increasing KV length) and cut into launches that fit
+  // the argument tables.
+  auto n_hist = [&](int c) { return c == 0 ? 0 : 1 + (c - 1 - (c - W > 1 ? c - W : 1) + 1); };
+  std::vector<int> order(T);
+  for (int c = 0; c < T; ++c) order[c] = c;
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return n_hist(x) > n_hist(y); });
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int i = 0; i < T;) {
+    AttnLaunch L = base;
+    LaunchBuilder b(L);
+    for (; i < T; ++i) {
+      const int c = order[i];
+      const int need = n_hist(c) + 1 + (d.ref_len > 0 ? 1 : 0);
+      if (need > kMaxSegs) return fail(CCA_ERR_UNSUPPORTED, "%s: %d visible segments exceed %d", what, need, kMaxSegs);
+      if (!b.fits(need)) break;
+      b.begin(Lc, c, c);
+      if (d.ref_len > 0) b.add_seg(2, 0);
+      if (c > 0) {
+        b.add_seg(0, 0);
+        for (int h = (c - W > 1 ? c - W : 1); h < c; ++h) b.add_seg(0, h);
+      }
+      b.add_seg(1, c);
+      b.end();
+    }
+    CCA_TRY(run_launch(L, workspace, workspace_bytes, st));
+  }
+  return CCA_OK;
+}
+
+}  // extern "C"
 
 // ------------------------------------------------------------------ allocation-free variant
 // Some callers cannot hand this library a scratch buffer: a real-time stream
@@ -1239,9 +1672,7 @@ cca_status cca_chunk_attn_noalloc(const cca_kv_ring *ring, const void *q, const 
   if (n_q_max < 0 || n_q_max > ring->d.chunk_len)
     return fail(CCA_ERR_INVALID_ARG, "cca_chunk_attn_noalloc: need 0 <= n_q_max <= chunk_len (%d)",
                 ring->d.chunk_len);
-  AttnPlan p;
-  plan_attention(ring, n_q_max, p);
-  const size_t need = workspace_bytes_for(ring, n_q_max, p);
+  const size_t need = n_q_max == 0 ? 0 : workspace_bytes_any(ring->d.head_dim);
   if (need > kNoAllocScratchBytes)
     return fail(CCA_ERR_INVALID_ARG,
                 "cca_chunk_attn_noalloc: this call needs %zu bytes of scratch, more than the %zu-byte built-in "

@@ -230,6 +230,81 @@ cca_status cca_chunk_attn_noalloc(const cca_kv_ring *ring, const void *q,
                                   float softmax_scale, void *out,
                                   cca_stream_t stream);
 
+/* Bytes of device workspace that suffice for every attention call of this
+ * library with the given head_dim (64 or 128) on the current device: the
+ * split-KV partial results of at most one CTA per SM (or CCA_ATTN_CTAS). */
+cca_status cca_attn_workspace_size(int32_t head_dim, size_t *bytes);
+
+/* ------------------------------------------------------------------------ */
+/* Token groups of the active chunk, and the packed block-causal forward      */
+/* ------------------------------------------------------------------------ */
+
+/* Attention of one denoising step with the token groups of the pages' mask
+ * ["JoyAI-Video-Edit 소개", section 세 부품으로 이루어진 아키텍처 (the
+ * attention-mask figure: noisy tokens N_t, global tokens H_0, history tokens
+ * H_{t-1}, MLLM condition tokens C_t, reference VAE tokens R, source VAE
+ * tokens S_t) and section 청크 단위 자기회귀 적응 (the active chunk sees its
+ * own source and condition tokens in both directions, the windowed history
+ * and the global sink causally; future chunks are masked; only R is open to
+ * every query)].
+ *
+ * The active block of chunk t = n_appended -- its groups N_t, S_t and C_t,
+ * concatenated in any order as n_cur rows -- attends with one dense softmax to
+ * the reference group R (n_ref rows; none when n_ref = 0), to the ring's
+ * cached chunks (the sink and the window, exactly as cca_chunk_attn) and to
+ * itself.  No element mask inside that set.  The history chunks of the ring
+ * hold the clean tokens of earlier chunks (chunk_len rows each).
+ *  q, k_cur, v_cur: device [n_cur][H][D] in the ring's dtype; 0 <= n_cur <= 2^24.
+ *  k_ref, v_ref: device [n_ref][H][D] (ring dtype), NULL when n_ref = 0.
+ *  q_scale, kcur_scale, vcur_scale, kref_scale, vref_scale: E4M3 only,
+ *      device [H] fp32 (NULL for BF16; the ref scales also NULL when n_ref = 0).
+ *  out: device [n_cur][H][D] bf16.
+ *  workspace: as cca_chunk_attn, of at least cca_attn_workspace_size(D) bytes.
+ * R's own queries see R only: that is cca_block_attn with one chunk of R and
+ * no history.  Errors: CCA_ERR_INVALID_ARG, CCA_ERR_UNSUPPORTED (E4M3 with
+ * D = 64), CCA_ERR_CUDA. */
+cca_status cca_chunk_attn_groups(const cca_kv_ring *ring, const void *q, const void *k_cur, const void *v_cur,
+                                 int32_t n_cur, const void *k_ref, const void *v_ref, int32_t n_ref,
+                                 const float *q_scale, const float *kcur_scale, const float *vcur_scale,
+                                 const float *kref_scale, const float *vref_scale, float softmax_scale, void *out,
+                                 void *workspace, size_t workspace_bytes, cca_stream_t stream);
+
+/* Packed block-causal forward: every chunk of a sequence in one call, as in
+ * training with teacher forcing ["JoyAI-Video-Edit 소개", section 청크 단위
+ * 자기회귀 적응: the noisy active chunks, their clean history and the other
+ * groups are packed into one sequence under the group mask, each target chunk
+ * with its own noise level].  Chunk c (0 <= c < T) of the "current" tensors
+ * (the noisy chunks) attends to: R (ref_len rows, optional), the history
+ * chunks {0} U {max(1, c-W) .. c-1} of the "history" tensors (the clean
+ * chunks; chunk 0 is the sink) and current chunk c itself.  With the history
+ * tensors equal to the current ones this is plain windowed block-causal
+ * attention (W >= T-1: full block-causal), which also gives the clean
+ * chunks' own outputs.
+ *  k_cur, v_cur, k_hist, v_hist: device [T][L][H][D] (dtype); the history
+ *      tensors may alias the current ones.
+ *  k_ref, v_ref: device [ref_len][H][D] or NULL with ref_len = 0.
+ *  Scales (E4M3 only, else NULL): kcur/vcur/khist/vhist [T][H], kref/vref [H].
+ *  dev_status: device int32 (CCA_DEV_*), may be NULL. */
+typedef struct cca_block_desc {
+  int32_t n_heads;      /* H >= 1                                   */
+  int32_t head_dim;     /* D: 64 or 128 (E4M3: 128)                 */
+  int32_t chunk_len;    /* L >= 1 tokens per chunk                  */
+  int32_t n_chunks;     /* T, 0 <= T <= 4095                        */
+  int32_t window;       /* W >= 0 history chunks besides the sink   */
+  cca_dtype dtype;      /* CCA_BF16 or CCA_E4M3                     */
+  const void *k_cur, *v_cur, *k_hist, *v_hist, *k_ref, *v_ref;
+  int32_t ref_len;
+  const float *kcur_scale, *vcur_scale, *khist_scale, *vhist_scale, *kref_scale, *vref_scale;
+  int32_t *dev_status;
+} cca_block_desc;
+
+/* q: device [T][L][H][D] (dtype); q_scale: E4M3 [T][H] else NULL; out: device
+ * [T][L][H][D] bf16.  workspace: at least cca_attn_workspace_size(D) bytes
+ * (reused by the launches of the call, which run in order on the stream).
+ * Errors: CCA_ERR_INVALID_ARG, CCA_ERR_UNSUPPORTED, CCA_ERR_CUDA. */
+cca_status cca_block_attn(const cca_block_desc *desc, const void *q, const float *q_scale, float softmax_scale,
+                          void *out, void *workspace, size_t workspace_bytes, cca_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* L2 token mask, compaction, scatter (LiveEdit mask cache)                 */
 /* ------------------------------------------------------------------------ */

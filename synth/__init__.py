@@ -24,6 +24,11 @@ Workloads (seed = index):
   4 mask      1620x16 fp32 source/edit latents on the 30x54 grid; 1-4 random
               ellipses covering 30 % +- 2 % get offset N(2,1), background N(0,0.1);
               Q/K/V of workload 1; cached outputs N(0, 0.02^2) bf16
+  5 groups    the 720p chunk t=4 with its token groups: N_t (1620 noisy tokens),
+              S_t (1620 source tokens), C_t (256 condition tokens) and R (1620
+              reference tokens); ring = clean chunks 0..3; per-head RMS 1, bf16
+  6 packed    T=8 chunks of the 720p shape in one sequence (teacher forcing):
+              noisy Q/K/V and clean K/V [T, 1620, 24, 128], per-head RMS 1, bf16
 """
 
 from __future__ import annotations
@@ -204,6 +209,66 @@ def mask_chunk(seed: int = 4, n_ch: int = 16, n_heads: int = 24, head_dim: int =
     edit = (src + np.where(region[:, None], off_in, off_out)).astype(np.float32)
     o_cache = bf16_round(g.normal(0.0, 0.02, size=(n, n_heads, head_dim)).astype(np.float32))
     return MaskChunk(src, edit, region, 0.70, o_cache)
+
+
+# ---------------------------------------------------------------- workload 5
+@dataclasses.dataclass
+class GroupsChunk:
+    n_heads: int
+    head_dim: int
+    chunk_len: int  # tokens of one clean history chunk
+    window: int
+    ring_k: list  # clean chunks 0..t-1
+    ring_v: list
+    t: int
+    groups: dict  # name -> (q, k, v) [n, H, D] for "N", "S", "C" (packed in that order)
+    ref: tuple  # (q, k, v) of R [n_ref, H, D], or None
+
+
+def groups_chunk(seed: int = 5, n_heads: int = 24, head_dim: int = 128, chunk_len: int = TOKENS_720P,
+                 window: int = 3, n_prefill: int = 4, n_src: int = TOKENS_720P, n_cond: int = 256,
+                 n_ref: int = TOKENS_720P) -> GroupsChunk:
+    """Workload 5: one denoising step of chunk t with all token groups present.
+    The MLLM condition tokens count (256) is not on the pages."""
+    g = rng(seed)
+
+    def draw(n):
+        return bf16_round(_head_rms_one(g.standard_normal((n, n_heads, head_dim), dtype=np.float32)))
+
+    ring_k, ring_v = [], []
+    for _ in range(n_prefill):
+        ring_k.append(draw(chunk_len))
+        ring_v.append(draw(chunk_len))
+    groups = {name: (draw(n), draw(n), draw(n)) for name, n in (("N", chunk_len), ("S", n_src), ("C", n_cond))
+              if n > 0}
+    ref = (draw(n_ref), draw(n_ref), draw(n_ref)) if n_ref > 0 else None
+    return GroupsChunk(n_heads, head_dim, chunk_len, window, ring_k, ring_v, n_prefill, groups, ref)
+
+
+# ---------------------------------------------------------------- workload 6
+@dataclasses.dataclass
+class PackedSequence:
+    window: int
+    q: np.ndarray  # [T, L, H, D] queries of the noisy chunks
+    k_cur: np.ndarray
+    v_cur: np.ndarray
+    k_hist: np.ndarray  # clean chunks
+    v_hist: np.ndarray
+
+
+def packed_sequence(seed: int = 6, n_chunks: int = 8, n_heads: int = 24, head_dim: int = 128,
+                    chunk_len: int = TOKENS_720P, window: int = 3, heavy_tailed: bool = False) -> PackedSequence:
+    """Workload 6: a training-time packed sequence of T chunks."""
+    g = rng(seed)
+    shape = (n_chunks, chunk_len, n_heads, head_dim)
+
+    def draw():
+        if heavy_tailed:
+            return bf16_round(g.standard_t(4.0, size=shape).astype(np.float32))
+        x = g.standard_normal(shape, dtype=np.float32)
+        return bf16_round(np.stack([_head_rms_one(c) for c in x]))
+
+    return PackedSequence(window, draw(), draw(), draw(), draw(), draw())
 
 
 def as_torch_bf16(x: np.ndarray, device="cpu") -> torch.Tensor:

@@ -152,6 +152,36 @@ def test_call_validation_without_device_work(L):
     assert L.cca_chunk_attn_noalloc(h, vp(0x1000), vp(0x1000), vp(0x1000), None, None, None, None, None, 17,
                                     0.0, vp(0x1000), None) == 1
     assert L.cca_compact_workspace_size(-1, ctypes.byref(sz)) == 1
+    assert L.cca_attn_workspace_size(96, ctypes.byref(sz)) == 1
+    assert L.cca_attn_workspace_size(128, None) == 1
+    # token groups: NULL ring / tensors, sizes out of range, misalignment, scales on BF16
+    g = L.cca_chunk_attn_groups
+    assert g(None, vp(0x1000), vp(0x1000), vp(0x1000), 8, None, None, 0, None, None, None, None, None, 0.0,
+             vp(0x1000), None, 0, None) == 1
+    assert g(h, vp(0x1000), vp(0x1000), vp(0x1000), -1, None, None, 0, None, None, None, None, None, 0.0,
+             vp(0x1000), None, 0, None) == 1
+    assert g(h, vp(0x1000), vp(0x1000), vp(0x1000), 8, None, None, 4, None, None, None, None, None, 0.0,
+             vp(0x1000), None, 0, None) == 1  # n_ref > 0 without k_ref / v_ref
+    assert g(h, vp(0x1004), vp(0x1000), vp(0x1000), 8, None, None, 0, None, None, None, None, None, 0.0,
+             vp(0x1000), None, 0, None) == 1
+    assert g(h, vp(0x1000), vp(0x1000), vp(0x1000), 8, None, None, 0, vp(0x2000), None, None, None, None, 0.0,
+             vp(0x1000), None, 0, None) == 1
+    assert g(h, None, None, None, 0, None, None, 0, None, None, None, None, None, 0.0, None, None, 0, None) == 0
+    # packed block-causal forward: descriptor checks
+    def bd(**kw):
+        d = dict(n_heads=2, head_dim=64, chunk_len=16, n_chunks=3, window=1, dtype=cca.CCA_BF16,
+                 k_cur=0x1000, v_cur=0x2000, k_hist=0x1000, v_hist=0x2000, k_ref=None, v_ref=None, ref_len=0,
+                 kcur_scale=None, vcur_scale=None, khist_scale=None, vhist_scale=None, kref_scale=None,
+                 vref_scale=None, dev_status=None)
+        d.update(kw)
+        return cca._BlockDesc(**d)
+    b = L.cca_block_attn
+    assert b(None, vp(0x1000), None, 0.0, vp(0x1000), None, 0, None) == 1
+    for bad in (dict(head_dim=96), dict(n_heads=0), dict(chunk_len=0), dict(window=-1), dict(n_chunks=4096),
+                dict(k_hist=None), dict(v_cur=0x2008), dict(ref_len=5), dict(dtype=cca.CCA_E4M3),
+                dict(kcur_scale=0x3000), dict(dtype=9)):
+        assert b(ctypes.byref(bd(**bad)), vp(0x1000), None, 0.0, vp(0x1000), None, 0, None) != 0, bad
+    assert b(ctypes.byref(bd(n_chunks=0)), None, None, 0.0, None, None, 0, None) == 0  # nothing to do
     # ring bookkeeping calls reject bad handles and counts
     assert L.cca_kv_ring_restore(h, -1) == 1
     assert L.cca_kv_ring_restore(None, 3) == 1
