@@ -22,6 +22,7 @@ __all__ = [
     "CCA_BF16", "CCA_E4M3", "CCA_F32", "CcaError", "KVRing", "lib", "lib_path", "EXPORTED",
     "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc",
     "cca_chunk_attn_scatter", "cca_attn_workspace_size", "cca_chunk_attn_groups", "cca_block_attn",
+    "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope",
     "cca_token_mask_l2", "cca_compact", "cca_compact_workspace_size", "cca_scatter", "cca_selftest_bounded_wait",
     "cca_version",
     "cca_take_launch_count",
@@ -37,7 +38,8 @@ EXPORTED = (
     "cca_kv_ring_create", "cca_kv_ring_destroy", "cca_kv_ring_reset", "cca_kv_ring_query",
     "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn",
     "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_chunk_attn_scatter", "cca_attn_workspace_size",
-    "cca_chunk_attn_groups", "cca_block_attn", "cca_token_mask_l2", "cca_compact",
+    "cca_chunk_attn_groups", "cca_block_attn", "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope",
+    "cca_token_mask_l2", "cca_compact",
     "cca_compact_workspace_size",
     "cca_scatter", "cca_selftest_bounded_wait", "cca_last_error", "cca_version", "cca_take_launch_count",
 )
@@ -98,6 +100,9 @@ def lib() -> ctypes.CDLL:
         "cca_chunk_attn_noalloc": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp],
         "cca_chunk_attn_scatter": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp],
         "cca_attn_workspace_size": [i32, ctypes.POINTER(sz)],
+        "cca_mrope_freqs": [i32, i32, i32, i32, f32, vp],
+        "cca_rope_qk": [vp, vp, ctypes.c_int, i32, i32, i32, vp, vp, vp, vp, vp],
+        "cca_kv_append_rope": [vp, vp, vp, ctypes.c_int, vp, vp, vp],
         "cca_chunk_attn_groups": [vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, f32, vp, vp, sz, vp],
         "cca_block_attn": [ctypes.POINTER(_BlockDesc), vp, vp, f32, vp, vp, sz, vp],
         "cca_token_mask_l2": [vp, vp, i32, i32, f32, f32, vp, vp, vp, vp],
@@ -234,6 +239,43 @@ def cca_kv_append(ring: KVRing, k_new: torch.Tensor, v_new: torch.Tensor, stream
         raise ValueError("k_new and v_new must share a dtype")
     _check(lib().cca_kv_append(ring.handle, _ptr(k_new, "k_new"), _ptr(v_new, "v_new"), _src_dtype(k_new),
                                _stream(stream)), "cca_kv_append")
+
+
+def cca_mrope_freqs(head_dim: int, sections=None, base: float = 10000.0, device=None) -> torch.Tensor:
+    """Default [4, D/2] fp32 frequency table (t, h, w sections, then the 1D source row)."""
+    if sections is None:
+        p = head_dim // 2
+        sections = (p - 2 * (p // 3), p // 3, p // 3)
+    buf = (ctypes.c_float * (2 * head_dim))()
+    _check(lib().cca_mrope_freqs(int(head_dim), int(sections[0]), int(sections[1]), int(sections[2]),
+                                 float(base), buf), "cca_mrope_freqs")
+    t = torch.tensor(list(buf), dtype=torch.float32).reshape(4, head_dim // 2)
+    return t if device is None else t.to(device)
+
+
+def cca_rope_qk(q: Optional[torch.Tensor], k: Optional[torch.Tensor], pos: torch.Tensor, freq: torch.Tensor,
+                q_out: Optional[torch.Tensor] = None, k_out: Optional[torch.Tensor] = None, stream=None):
+    """(rope(q), rope(k)) as bf16 [n, H, D]; pos int32 [n, 4], freq fp32 [4, D/2] on the device."""
+    x = q if q is not None else k
+    n, h, d = x.shape
+    if q is not None and q_out is None:
+        q_out = torch.empty((n, h, d), dtype=torch.bfloat16, device=x.device)
+    if k is not None and k_out is None:
+        k_out = torch.empty((n, h, d), dtype=torch.bfloat16, device=x.device)
+    _check(lib().cca_rope_qk(_ptr(q, "q"), _ptr(k, "k"), _src_dtype(x), n, h, d, _ptr(pos, "pos", torch.int32),
+                             _ptr(freq, "freq", torch.float32), _ptr(q_out, "q_out", torch.bfloat16),
+                             _ptr(k_out, "k_out", torch.bfloat16), _stream(stream)), "cca_rope_qk")
+    return q_out, k_out
+
+
+def cca_kv_append_rope(ring: KVRing, k_new: torch.Tensor, v_new: torch.Tensor, pos: torch.Tensor,
+                       freq: torch.Tensor, stream=None) -> None:
+    shape = (ring.chunk_len, ring.n_heads, ring.head_dim)
+    if tuple(k_new.shape) != shape or tuple(v_new.shape) != shape or k_new.dtype != v_new.dtype:
+        raise ValueError(f"k_new/v_new must be {shape} of one dtype")
+    _check(lib().cca_kv_append_rope(ring.handle, _ptr(k_new, "k_new"), _ptr(v_new, "v_new"), _src_dtype(k_new),
+                                    _ptr(pos, "pos", torch.int32), _ptr(freq, "freq", torch.float32),
+                                    _stream(stream)), "cca_kv_append_rope")
 
 
 def cca_quant_e4m3(x: torch.Tensor, x8: Optional[torch.Tensor] = None, scale: Optional[torch.Tensor] = None,

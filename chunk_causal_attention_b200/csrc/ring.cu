@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "ring.cuh"
+#include "rope.cuh"
 #include "sm100.cuh"
 
 namespace cca {
@@ -91,14 +92,35 @@ constexpr int kAppendUnroll = 10;
 constexpr int64_t kMaxChunkElems = int64_t(1) << 33;  // keeps 16-byte vector indices below 2^30
 constexpr int kAppendUnrollF32 = 4;  // fp32 sources: two 16-byte loads per output
 
-template <bool kF32>
+// With kRope, K (blockIdx.y == 0) is rotated on the way (rope.cuh): its 16-byte
+// vectors are expanded to fp32, turned and rounded to bf16 once.
+__device__ __forceinline__ uint4 rope_bf16x8(const RopeArgs &r, uint4 u, int64_t tok, int d0, int D) {
+  float x[8];
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    x[2 * j] = __uint_as_float(w[j] << 16);
+    x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+  }
+  rope8(r, tok, d0, D, x);
+  return to_bf16x8(make_float4(x[0], x[1], x[2], x[3]), make_float4(x[4], x[5], x[6], x[7]));
+}
+__device__ __forceinline__ uint4 rope_f32x8(const RopeArgs &r, float4 a, float4 b, int64_t tok, int d0, int D) {
+  float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  rope8(r, tok, d0, D, x);
+  return to_bf16x8(make_float4(x[0], x[1], x[2], x[3]), make_float4(x[4], x[5], x[6], x[7]));
+}
+
+template <bool kF32, bool kRope>
 __global__ void __launch_bounds__(256, 4) append_bf16_kernel(const void *__restrict__ k_src,
                                                              const void *__restrict__ v_src,
                                                              uint4 *__restrict__ k_dst,
-                                                             uint4 *__restrict__ v_dst, int n_vec) {
+                                                             uint4 *__restrict__ v_dst, int n_vec, RopeArgs rk,
+                                                             int vec_per_tok, int D) {
   constexpr int kU = kF32 ? kAppendUnrollF32 : kAppendUnroll;
   const void *src = blockIdx.y == 0 ? k_src : v_src;
   uint4 *dst = blockIdx.y == 0 ? k_dst : v_dst;
+  const bool rot = kRope && blockIdx.y == 0;
   const int stride = gridDim.x * blockDim.x;  // n_vec < 2^31 is checked on the host
   for (int i0 = blockIdx.x * blockDim.x + threadIdx.x; i0 < n_vec; i0 += kU * stride) {
     uint4 v[kU];
@@ -108,9 +130,12 @@ __global__ void __launch_bounds__(256, 4) append_bf16_kernel(const void *__restr
       if (i < static_cast<unsigned>(n_vec)) {
         if constexpr (!kF32) {
           v[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + i);
+          if (rot) v[u] = rope_bf16x8(rk, v[u], i / vec_per_tok, static_cast<int>((static_cast<int64_t>(i) * 8) % D), D);
         } else {
-          v[u] = to_bf16x8(__ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i)),
-                           __ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i) + 1));
+          const float4 a = __ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i));
+          const float4 b = __ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i) + 1);
+          v[u] = rot ? rope_f32x8(rk, a, b, i / vec_per_tok, static_cast<int>((static_cast<int64_t>(i) * 8) % D), D)
+                     : to_bf16x8(a, b);
         }
       }
     }
@@ -223,7 +248,8 @@ __device__ __forceinline__ void load8(const void *base, int64_t elem, float (&x)
 template <bool kF32>
 __global__ void __launch_bounds__(256) absmax_kernel(const void *__restrict__ x0, const void *__restrict__ x1,
                                                      unsigned *amax0, unsigned *amax1, int n_tok, int H,
-                                                     int D) {
+                                                     int D, RopeArgs rope0) {
+  const bool rot = blockIdx.z == 0 && rope0.pos != nullptr;  // x0 rotated before it is measured
   const void *x = blockIdx.z == 0 ? x0 : x1;
   unsigned *amax = blockIdx.z == 0 ? amax0 : amax1;
   const int h = blockIdx.y;
@@ -235,6 +261,7 @@ __global__ void __launch_bounds__(256) absmax_kernel(const void *__restrict__ x0
     for (int l = blockIdx.x * rows_per_iter + r0; l < n_tok; l += gridDim.x * rows_per_iter) {
       float v[8];
       load8<kF32>(x, (static_cast<int64_t>(l) * H + h) * D + c * 8, v);
+      if (rot) rope8(rope0, l, c * 8, D, v);
 #pragma unroll
       for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
     }
@@ -262,7 +289,8 @@ template <bool kF32>
 __global__ void __launch_bounds__(256) quant_e4m3_kernel(const void *__restrict__ x0, const void *__restrict__ x1,
                                                          const unsigned *amax0, const unsigned *amax1,
                                                          uint8_t *__restrict__ y0, uint8_t *__restrict__ y1,
-                                                         int n_tok, int H, int D) {
+                                                         int n_tok, int H, int D, RopeArgs rope0) {
+  const bool rot = blockIdx.z == 0 && rope0.pos != nullptr;
   const void *x = blockIdx.z == 0 ? x0 : x1;
   const unsigned *amax = blockIdx.z == 0 ? amax0 : amax1;
   uint8_t *y = blockIdx.z == 0 ? y0 : y1;
@@ -277,6 +305,7 @@ __global__ void __launch_bounds__(256) quant_e4m3_kernel(const void *__restrict_
     const int64_t e = (static_cast<int64_t>(l) * H + h) * D + c * 8;
     float v[8];
     load8<kF32>(x, e, v);
+    if (rot) rope8(rope0, l, c * 8, D, v);  // same rotation as the absmax pass
     uint32_t w[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -329,7 +358,8 @@ static cca_status bulk_copy_pair(const uint8_t *k_src, const uint8_t *v_src, uin
 
 // Quantise one or two [n_tok][H][D] tensors; scale arrays are [H] each.
 static cca_status quantize_pair(const void *x0, const void *x1, cca_dtype src, int n_tok, int H, int D,
-                                uint8_t *y0, uint8_t *y1, float *s0, float *s1, cudaStream_t st) {
+                                uint8_t *y0, uint8_t *y1, float *s0, float *s1, cudaStream_t st,
+                                RopeArgs r0 = RopeArgs{nullptr, nullptr}) {
   const int nt = x1 ? 2 : 1;
   unsigned *a0 = reinterpret_cast<unsigned *>(s0), *a1 = reinterpret_cast<unsigned *>(s1);
   zero_u32_kernel<<<1, 256, 0, st>>>(a0, x1 ? a1 : nullptr, H);
@@ -341,13 +371,13 @@ static cca_status quantize_pair(const void *x0, const void *x1, cca_dtype src, i
     if (bx > target) bx = target > 0 ? target : 1;
     dim3 grid(bx, H, nt);
     if (src == CCA_F32) {
-      absmax_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D);
+      absmax_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D, r0);
       CCA_TRY(launched("absmax_kernel"));
-      quant_e4m3_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D);
+      quant_e4m3_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D, r0);
     } else {
-      absmax_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D);
+      absmax_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D, r0);
       CCA_TRY(launched("absmax_kernel"));
-      quant_e4m3_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D);
+      quant_e4m3_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D, r0);
     }
     CCA_TRY(launched("quant_e4m3_kernel"));
   }
@@ -412,8 +442,10 @@ cca_status cca_kv_ring_restore(cca_kv_ring *ring, int64_t n_appended) {
   return CCA_OK;
 }
 
-cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new, cca_dtype src_dtype,
-                         cca_stream_t stream) {
+}  // extern "C"
+
+static cca_status kv_append_impl(cca_kv_ring *ring, const void *k_new, const void *v_new, cca_dtype src_dtype,
+                                 RopeArgs rk, cca_stream_t stream) {
   if (!ring || !k_new || !v_new) return fail(CCA_ERR_INVALID_ARG, "cca_kv_append: NULL argument");
   if (!aligned16(k_new) || !aligned16(v_new))
     return fail(CCA_ERR_INVALID_ARG, "cca_kv_append: k_new/v_new must be 16-byte aligned");
@@ -437,8 +469,18 @@ cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new
     const int64_t cap = static_cast<int64_t>(num_sms()) * 2;  // x2 tensors: 4 blocks of 256 per SM
     if (blocks > cap) blocks = cap;
     dim3 grid(static_cast<unsigned>(blocks), 2);
-    if (src_dtype == CCA_F32) {
-      append_bf16_kernel<true><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, static_cast<int>(n_vec));
+    const int vpt = d.n_heads * d.head_dim / 8;
+    if (rk.pos) {  // K rotated on the way into the ring
+      if (src_dtype == CCA_F32)
+        append_bf16_kernel<true, true><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, static_cast<int>(n_vec), rk, vpt,
+                                                             d.head_dim);
+      else
+        append_bf16_kernel<false, true><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, static_cast<int>(n_vec), rk,
+                                                              vpt, d.head_dim);
+      CCA_TRY(launched("append_bf16_kernel"));
+    } else if (src_dtype == CCA_F32) {
+      append_bf16_kernel<true, false><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, static_cast<int>(n_vec), rk, vpt,
+                                                            d.head_dim);
       CCA_TRY(launched("append_bf16_kernel"));
     } else {
       CCA_TRY(bulk_copy_pair(static_cast<const uint8_t *>(k_new), static_cast<const uint8_t *>(v_new),
@@ -449,10 +491,24 @@ cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new
     uint8_t *kd = static_cast<uint8_t *>(d.k_slots) + slot * n_elem;
     uint8_t *vd = static_cast<uint8_t *>(d.v_slots) + slot * n_elem;
     CCA_TRY(quantize_pair(k_new, v_new, src_dtype, d.chunk_len, d.n_heads, d.head_dim, kd, vd,
-                          d.k_scale + slot * d.n_heads, d.v_scale + slot * d.n_heads, st));
+                          d.k_scale + slot * d.n_heads, d.v_scale + slot * d.n_heads, st, rk));
   }
   ring->n_appended = t + 1;
   return CCA_OK;
+}
+
+extern "C" {
+
+cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new, cca_dtype src_dtype,
+                         cca_stream_t stream) {
+  return kv_append_impl(ring, k_new, v_new, src_dtype, RopeArgs{nullptr, nullptr}, stream);
+}
+
+cca_status cca_kv_append_rope(cca_kv_ring *ring, const void *k_new, const void *v_new, cca_dtype src_dtype,
+                              const int32_t *pos, const float *freq, cca_stream_t stream) {
+  if (!pos || !freq || !aligned16(pos) || (reinterpret_cast<uintptr_t>(freq) & 3))
+    return fail(CCA_ERR_INVALID_ARG, "cca_kv_append_rope: pos (16-byte aligned) and freq (4-byte aligned) required");
+  return kv_append_impl(ring, k_new, v_new, src_dtype, RopeArgs{pos, freq}, stream);
 }
 
 cca_status cca_quant_e4m3(const void *x, cca_dtype src_dtype, int32_t n_tok, int32_t n_heads, int32_t head_dim,

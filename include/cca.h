@@ -129,6 +129,46 @@ cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new
                          cca_dtype src_dtype, cca_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Rotary position encoding (fused 3D + 1D angle)                            */
+/* ------------------------------------------------------------------------ */
+
+/* ["JoyAI-Video-Edit 소개", section 세 부품으로 이루어진 아키텍처: positions are
+ * encoded by a rotation whose angle fuses a 3D spatio-temporal RoPE with a 1D
+ * source RoPE, so source and generated tokens of one sequence differ.]  The
+ * formula is not on the pages; this library's reading: each token carries
+ * integer coordinates pos = (t, h, w, s) -- latent frame, row, column and a
+ * source index -- and pair i (elements 2i, 2i+1 of every head) is rotated by
+ *     theta_i = t F[0][i] + h F[1][i] + w F[2][i] + s F[3][i]
+ * (x'_{2i} = x_{2i} cos - x_{2i+1} sin, x'_{2i+1} = x_{2i} sin + x_{2i+1} cos):
+ * the 3D rotation and the 1D source rotation act in the same plane, so their
+ * angles add.  pos: device int32 [n_tok][4], 16-byte aligned.  F ("freq"):
+ * device fp32 [4][D/2]. */
+
+/* Default table into host memory freq[4][D/2]: coordinate a in {t, h, w}
+ * turns the sec_a pairs of its section (t first, then h, then w; sec_t +
+ * sec_h + sec_w = D/2) at frequencies base^(-j / sec_a), j = 0 .. sec_a-1, and
+ * 0 elsewhere; the source index turns every pair i at base^(-2i / D).
+ * Errors: CCA_ERR_INVALID_ARG. */
+cca_status cca_mrope_freqs(int32_t head_dim, int32_t sec_t, int32_t sec_h, int32_t sec_w, float base,
+                           float *freq);
+
+/* Rotate the current chunk's queries and keys in one launch: q_out = rope(q),
+ * k_out = rope(k), all [n_tok][H][D]; inputs CCA_BF16 or CCA_F32 (fp32
+ * rotation, one rounding to the bf16 outputs).  Either q or k may be NULL (its
+ * output is then ignored); outputs may alias their inputs for BF16 input.
+ * Errors: CCA_ERR_INVALID_ARG, CCA_ERR_CUDA. */
+cca_status cca_rope_qk(const void *q, const void *k, cca_dtype src_dtype, int32_t n_tok, int32_t n_heads,
+                       int32_t head_dim, const int32_t *pos, const float *freq, void *q_out, void *k_out,
+                       cca_stream_t stream);
+
+/* cca_kv_append with the rotation applied to K as it is stored (V is stored
+ * as given): the clean chunk's keys enter the cache already encoded.  For an
+ * E4M3 ring the rotated keys are what the absmax scale and the codes are taken
+ * from.  pos: [L][4] of the chunk being appended.  Errors: as cca_kv_append. */
+cca_status cca_kv_append_rope(cca_kv_ring *ring, const void *k_new, const void *v_new, cca_dtype src_dtype,
+                              const int32_t *pos, const float *freq, cca_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* FP8 quantiser                                                             */
 /* ------------------------------------------------------------------------ */
 

@@ -271,6 +271,14 @@ def packed_sequence(seed: int = 6, n_chunks: int = 8, n_heads: int = 24, head_di
     return PackedSequence(window, draw(), draw(), draw(), draw(), draw())
 
 
+def grid_positions(t: int, source: int = 0, grid=(GRID_H, GRID_W), n_frames: int = 1) -> np.ndarray:
+    """Integer token coordinates (t, h, w, s) of the latent frames t .. t+n_frames-1
+    of a chunk on the latent grid, frame-major then row-major: int32 [n, 4]."""
+    f, r, c = np.meshgrid(np.arange(n_frames), np.arange(grid[0]), np.arange(grid[1]), indexing="ij")
+    n = f.size
+    return np.stack([t + f.reshape(n), r.reshape(n), c.reshape(n), np.full(n, source)], axis=1).astype(np.int32)
+
+
 def as_torch_bf16(x: np.ndarray, device="cpu") -> torch.Tensor:
     """float32 array of bf16 values -> contiguous bf16 tensor (exact)."""
     return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16).to(device)

@@ -190,6 +190,30 @@ def test_call_validation_without_device_work(L):
     assert L.cca_kv_ring_destroy(h) == 0
 
 
+def test_library_rope_table_follows_the_stated_recipe(L):
+    """cca_mrope_freqs is host code: its table equals the oracle's fp64 table
+    rounded to fp32 (within an ulp of the pow), and bad sections are refused."""
+    import numpy as np
+    from oracle import rope as orope
+    for D, sec in ((128, (22, 21, 21)), (64, (12, 10, 10)), (128, (64, 0, 0))):
+        buf = (ctypes.c_float * (2 * D))()
+        assert L.cca_mrope_freqs(D, *sec, ctypes.c_float(10000.0), buf) == 0
+        got = np.array(list(buf), dtype=np.float64).reshape(4, D // 2)
+        want = orope.frequencies(D, sections=sec)
+        assert np.all(np.abs(got - want) <= 2.0 ** -23 * np.abs(want))
+    buf = (ctypes.c_float * 256)()
+    assert L.cca_mrope_freqs(128, 22, 21, 20, ctypes.c_float(10000.0), buf) == 1
+    assert L.cca_mrope_freqs(96, 16, 16, 16, ctypes.c_float(10000.0), buf) == 1
+    assert L.cca_mrope_freqs(128, 22, 21, 21, ctypes.c_float(1.0), buf) == 1
+    vp = ctypes.c_void_p
+    assert L.cca_rope_qk(vp(0x1000), None, cca.CCA_BF16, 10, 2, 64, None, vp(0x2000), vp(0x1000), None, None) == 1
+    assert L.cca_rope_qk(vp(0x1000), None, cca.CCA_E4M3, 10, 2, 64, vp(0x3000), vp(0x2000), vp(0x1000), None,
+                         None) == 1
+    assert L.cca_rope_qk(vp(0x1008), None, cca.CCA_BF16, 10, 2, 64, vp(0x3000), vp(0x2000), vp(0x1000), None,
+                         None) == 1
+    assert L.cca_rope_qk(None, None, cca.CCA_BF16, 10, 2, 64, None, None, None, None, None) == 0
+
+
 def test_product_path_has_no_cpu_fallback():
     import torch
     with pytest.raises((ValueError, RuntimeError)):
