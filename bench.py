@@ -71,6 +71,59 @@ def job_value(world: int, flop_per_rank_step: float, ms_per_step_max: float) -> 
 
 
 # ------------------------------------------------------------------ clocks
+class NvmlClockSampler:
+    """SM clock and throttle reasons sampled through NVML every ``period_s``
+    during the timed region (dense enough for a region of a few ms)."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, gpu_index: int, period_s: float = 0.002):
+        import pynvml
+        pynvml.nvmlInit()
+        self.nv = pynvml
+        self.h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+        self.period = period_s
+        self.rows = []
+        self.stop_flag = False
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.rows.append((float(mhz), float(mx), int(rs)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        time.sleep(0.02)
+
+    def stop(self, n_skip: int = 0):
+        time.sleep(0.01)
+        self.stop_flag = True
+        self.thread.join(timeout=2)
+        rows = self.rows[n_skip:] or self.rows
+        if not rows:
+            return None
+        reasons = sorted({n for _, _, r in rows for n, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_min_mhz": min(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons, "samples": len(rows),
+                "sampler": f"NVML every {self.period * 1e3:.0f} ms"}
+
+
+def clock_sampler(gpu_index: int):
+    try:
+        return NvmlClockSampler(gpu_index)
+    except Exception:
+        return ClockSampler(gpu_index)
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -153,10 +206,35 @@ def blas_threads():
 
 
 def cpu_baseline():
-    flop, dt = oracle_sample(L, H)  # one full 720p attention call
+    """The fp64 oracle on the host cores: the 720p call (the line's value), plus
+    the tiny stream and the 486-query mask-cached call, each the median of 3 runs."""
+    import synth
+    from oracle import chunk_attention as oca
+    runs = [oracle_sample(L, H) for _ in range(3)]  # one full 720p attention call each
+    flop = runs[0][0]
+    dt = statistics.median(r[1] for r in runs)
+    # tiny stream: 4 chunks of 16 tokens, H=1, D=64, W=2 (all four chunk calls)
+    s0 = synth.tiny()
+    t0s = []
+    for _ in range(3):
+        t0 = time.perf_counter()
+        for t in range(4):
+            oca.chunk_attention(s0.q[t], s0.k, s0.v, t, s0.window)
+        t0s.append(time.perf_counter() - t0)
+    flop0 = sum(4.0 * 16 * (16 * len(oca.visible_chunks(t, 2))) * 64 for t in range(4))
+    # mask-cached call: 486 active queries of the 720p call
+    t4s = [oracle_sample(486, H)[1] for _ in range(3)]
+    flop4 = 4.0 * 486 * LK * H * D
     return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"fp64 numpy oracle, one full 720p attention call (1620 queries x 24 heads x 8100 keys), "
-                      f"{dt:.2f} s"}
+                      f"median of 3 runs: {dt:.2f} s",
+            "workloads": {
+                "720p_call": {"s_median": dt, "s_runs": [r[1] for r in runs], "tflops": flop / dt / 1e12},
+                "tiny_stream_4_chunks": {"ms_median": statistics.median(t0s) * 1e3,
+                                         "ms_runs": [x * 1e3 for x in t0s],
+                                         "gflops": flop0 / statistics.median(t0s) / 1e9},
+                "mask_cached_486_queries": {"s_median": statistics.median(t4s), "s_runs": t4s,
+                                            "tflops": flop4 / statistics.median(t4s) / 1e12}}}
 
 
 def run_reference(args, rank, world):
@@ -390,6 +468,143 @@ def extra_workloads(dev, stream, peak_tf, peak_gbs):
     return out
 
 
+def extra_rows(dev, stream, peak_tf, peak_gbs):
+    """The other hot-path rows at their workload sizes: the clean-pass call, the
+    token-group step, the packed block-causal forward, the LiveEdit-shaped chunk,
+    the rotary encoding and the e4m3 append.  Inputs are drawn on the device
+    (timing only; parity is the tests' job)."""
+    import torch
+    import chunk_causal_attention_b200 as cca
+    out = {}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    rnd = lambda *sh: torch.randn(*sh, generator=gen, device=dev).to(torch.bfloat16)
+    med_us = lambda ts: float(np.median(ts)) * 1e3
+
+    def ring_with(n_tok, window, n_prefill, dtype="bf16"):
+        r = cca.KVRing(H, D, n_tok, window, dtype=dtype, device=dev)
+        for _ in range(n_prefill):
+            r.append(rnd(n_tok, H, D), rnd(n_tok, H, D))
+        return r
+
+    # ---- clean pass: the third attention call of a chunk (same shape as a denoising call)
+    rings = [ring_with(L, W, 4) for _ in range(3)]
+    qkv = [(rnd(L, H, D), rnd(L, H, D), rnd(L, H, D)) for _ in range(3)]
+    o = torch.empty((L, H, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(cca.cca_attn_workspace_size(D), dtype=torch.uint8, device=dev)
+    it = [0]
+
+    def clean_call():
+        i = it[0] % 3
+        it[0] += 1
+        cca.cca_chunk_attn(rings[i], *qkv[i], out=o, workspace=ws)
+    us = med_us(_timed(clean_call, 60, stream))
+    out["clean_pass_720p"] = {"us": us, "tflops": FLOP_PER_CALL / (us * 1e-6) / 1e12,
+                              "frac_of_bf16_peak": FLOP_PER_CALL / (us * 1e-6) / 1e12 / peak_tf}
+    del qkv
+
+    # ---- token groups: N_t (1620) + S_t (1620) + C_t (256) over R (1620), sink + 3 window chunks, themselves
+    n_cur, n_ref = L + L + 256, L
+    qg, kg, vg = rnd(n_cur, H, D), rnd(n_cur, H, D), rnd(n_cur, H, D)
+    kr, vr = rnd(n_ref, H, D), rnd(n_ref, H, D)
+    og = torch.empty((n_cur, H, D), dtype=torch.bfloat16, device=dev)
+    us = med_us(_timed(lambda: cca.cca_chunk_attn_groups(rings[0], qg, kg, vg, k_ref=kr, v_ref=vr, out=og,
+                                                         workspace=ws), 30, stream))
+    lk = n_ref + 4 * L + n_cur
+    fl = 4.0 * n_cur * lk * H * D
+    out["groups_720p"] = {"us": us, "q_tokens": n_cur, "kv_tokens": lk, "tflops": fl / (us * 1e-6) / 1e12,
+                          "frac_of_bf16_peak": fl / (us * 1e-6) / 1e12 / peak_tf}
+    del qg, kg, vg, kr, vr, og
+
+    # ---- packed block-causal forward: T = 8 chunks of the 720p shape, window 3
+    T = 8
+    qp, kp, vp, kh, vh = (rnd(T, L, H, D) for _ in range(5))
+    op = torch.empty((T, L, H, D), dtype=torch.bfloat16, device=dev)
+    us = med_us(_timed(lambda: cca.cca_block_attn(qp, kp, vp, W, k_hist=kh, v_hist=vh, out=op, workspace=ws),
+                       10, stream))
+    n_vis = sum(1 + (0 if c == 0 else 1 + (c - max(1, c - W))) for c in range(T))
+    fl = 4.0 * L * (n_vis * L) * H * D
+    out["block_causal_720p_T8"] = {"us": us, "chunks": T, "window": W, "tflops": fl / (us * 1e-6) / 1e12,
+                                   "frac_of_bf16_peak": fl / (us * 1e-6) / 1e12 / peak_tf}
+    del qp, kp, vp, kh, vh, op
+
+    # ---- LiveEdit-shaped chunk: 3 latent frames (4860 tokens), sink + 2-chunk window, 4 denoising
+    # steps on the active tokens of the 3-frame mask (fused scatter-back), the clean pass, the append
+    F_, Wl = 3, 2
+    Ll = F_ * L
+    rl = ring_with(Ll, Wl, 3)
+    ql = [rnd(Ll, H, D) for _ in range(4)]
+    kl = [rnd(Ll, H, D) for _ in range(4)]
+    vl = [rnd(Ll, H, D) for _ in range(4)]
+    caches = [rnd(Ll, H, D) for _ in range(4)]
+    ol = torch.empty((Ll, H, D), dtype=torch.bfloat16, device=dev)
+    src = torch.randn((F_, L, 16), generator=gen, device=dev)
+    region = (torch.rand(L, generator=gen, device=dev) < 0.3).float()[None, :, None]
+    edit = src + region * (2.0 + torch.randn((F_, L, 16), generator=gen, device=dev)) + \
+        (1 - region) * 0.1 * torch.randn((F_, L, 16), generator=gen, device=dev)
+    maskl = torch.empty(Ll, dtype=torch.uint8, device=dev)
+    idxl = torch.empty(Ll, dtype=torch.int32, device=dev)
+    nl = torch.empty(1, dtype=torch.int32, device=dev)
+
+    def liveedit_chunk(append=True):
+        cca.cca_token_mask_l2_frames(src, edit, prune_quantile=0.7, mask=maskl)
+        cca.cca_compact(maskl, idxl, nl)
+        for st in range(4):
+            cca.cca_chunk_attn_scatter(rl, ql[st], kl[st], vl[st], idxl, caches[st], n_q_dev=nl, n_q_max=Ll,
+                                       workspace=ws)
+        cca.cca_chunk_attn(rl, ql[0], kl[0], vl[0], out=ol, workspace=ws)  # clean pass
+        if append:
+            n0 = rl.n_appended
+            rl.append(kl[0], vl[0])
+            rl.restore(n0)  # keep the visible set fixed across reps
+    ms = float(np.median(_timed(liveedit_chunk, 10, stream)))
+    n_act = int(nl.item())
+    lkl = (1 + Wl + 1) * Ll
+    us_full = med_us(_timed(lambda: cca.cca_chunk_attn(rl, ql[1], kl[1], vl[1], out=ol, workspace=ws), 10, stream))
+    us_act = med_us(_timed(lambda: cca.cca_chunk_attn_scatter(rl, ql[1], kl[1], vl[1], idxl, caches[1], n_q_dev=nl,
+                                                              n_q_max=Ll, workspace=ws), 10, stream))
+    fl_full, fl_act = 4.0 * Ll * lkl * H * D, 4.0 * n_act * lkl * H * D
+    out["liveedit_3frame_chunk"] = {
+        "ms_per_chunk": ms, "tokens_per_chunk": Ll, "kv_tokens": lkl, "active_tokens": n_act, "steps": 4,
+        "full_call_us": us_full, "full_call_tflops": fl_full / (us_full * 1e-6) / 1e12,
+        "full_call_frac_of_bf16_peak": fl_full / (us_full * 1e-6) / 1e12 / peak_tf,
+        "active_call_us": us_act, "active_call_tflops": fl_act / (us_act * 1e-6) / 1e12,
+        "step": "3-frame mask + compaction + 4 active-token attention calls (fused scatter) + clean pass + append"}
+    del rl, ql, kl, vl, caches, ol
+
+    # ---- rotary encoding: Q and K of a 720p chunk in one launch; the rotating append
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def bw(fn, nbytes, reps=20):
+        ts = []
+        for _ in range(reps):
+            flush.sum()
+            torch.cuda._sleep(200000)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        t = float(np.median(ts)) * 1e-3
+        return {"us": t * 1e6, "gbs": nbytes / t / 1e9, "frac_of_hbm": nbytes / t / 1e9 / peak_gbs}
+    import synth
+    pos = torch.from_numpy(synth.grid_positions(4)).to(dev)
+    freq = cca.cca_mrope_freqs(D, device=dev)
+    qr, kr_ = rnd(L, H, D), rnd(L, H, D)
+    qo, ko = torch.empty_like(qr), torch.empty_like(kr_)
+    nbytes = 4 * L * H * D * 2
+    out["rope_qk_720p"] = bw(lambda: cca.cca_rope_qk(qr, kr_, pos, freq, q_out=qo, k_out=ko), nbytes)
+    ra = cca.KVRing(H, D, L, W, device=dev)
+    out["append_rope_720p"] = bw(lambda: cca.cca_kv_append_rope(ra, qr, kr_, pos, freq), nbytes)
+    r8 = cca.KVRing(H, D, L, W, dtype="e4m3", device=dev)
+    e8 = bw(lambda: r8.append(qr, kr_), 2 * L * H * D * 2 + 2 * L * H * D)
+    e8["note"] = ("algorithmic bytes: read bf16 K and V once, write their e4m3 codes; the absmax and quantise passes "
+                  "read them twice")
+    out["append_e4m3_720p"] = e8
+    return out
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args, rank, world, local_rank):
     import torch
@@ -433,7 +648,7 @@ def run_gpu(args, rank, world, local_rank):
         step(reps[i % 3])
     torch.cuda.synchronize()
 
-    sampler = ClockSampler(local_rank) if rank == 0 else None
+    sampler = clock_sampler(local_rank) if rank == 0 else None
     if sampler:
         sampler.start()
     attn_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * CALLS_PER_STEP)] for _ in range(args.steps)]
@@ -563,11 +778,50 @@ def run_gpu(args, rank, world, local_rank):
     }
     if args.extras:
         peak_tf_, peak_gbs_, _ = peaks()
-        line["extra"] = extra_workloads(torch.device("cuda", local_rank), torch.cuda.current_stream(), peak_tf_,
-                                        peak_gbs_)
+        dev0 = torch.device("cuda", local_rank)
+        ex = extra_workloads(dev0, torch.cuda.current_stream(), peak_tf_, peak_gbs_)
+        ex.update(extra_rows(dev0, torch.cuda.current_stream(), peak_tf_, peak_gbs_))
+        line["rows"] = row_summary(line, ex)
+        line["extra"] = ex
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
+
+
+def row_summary(line, ex):
+    """One compact figure per hot-path row, ahead of the long "extra" block."""
+    g = lambda *ks: _dig(ex, ks)
+    mhz = (line.get("clocks") or {}).get("sm_mhz")
+    r = {
+        "a1_append_720p_us": g("append_720p", "us"), "a1_append_stream_frac_hbm": g("append_720p_stream", "frac_of_hbm"),
+        "a2_append_e4m3_720p_us": g("append_e4m3_720p", "us"),
+        "a3_bf16_call_us": line["attn_us_per_call"], "a3_bf16_frac": line["roofline"]["frac"],
+        "a3_bf16_call_us_at_1965mhz": line["attn_us_per_call"] * mhz / 1965.0 if mhz else None,
+        "a3_clean_pass_us": g("clean_pass_720p", "us"),
+        "a3_fp8_call_us": g("fp8_720p", "attn_us_per_call"), "a3_fp8_frac": g("fp8_720p", "frac_of_fp8_peak"),
+        "a4_mask_dynamic_us": g("mask_dynamic_720p_us"), "a4_mask_sweep_2^26_frac_hbm":
+            g("sweep_mask_fixed_log2_tokens", 26, "frac_of_hbm"),
+        "a5_compact_sweep_2^26_frac_hbm": g("sweep_compact_log2_tokens", 26, "frac_of_hbm"),
+        "a6_active_486_attn_us": g("mask_cached_720p", "attn_us"),
+        "a7_scatter_sweep_2^18_frac_hbm": g("sweep_scatter_log2_active_rows", 18, "frac_of_hbm"),
+        "c2_drift_pct": g("long_stream_225", "drift_pct"),
+        "f1_groups_us": g("groups_720p", "us"), "f1_groups_frac": g("groups_720p", "frac_of_bf16_peak"),
+        "f2_rope_qk_frac_hbm": g("rope_qk_720p", "frac_of_hbm"),
+        "f2_append_rope_frac_hbm": g("append_rope_720p", "frac_of_hbm"),
+        "f3_liveedit_ms_per_chunk": g("liveedit_3frame_chunk", "ms_per_chunk"),
+        "f3_liveedit_full_call_frac": g("liveedit_3frame_chunk", "full_call_frac_of_bf16_peak"),
+        "f4_block_T8_us": g("block_causal_720p_T8", "us"),
+        "f4_block_T8_frac": g("block_causal_720p_T8", "frac_of_bf16_peak"),
+    }
+    return r
+
+
+def _dig(d, ks):
+    for k in ks:
+        if not isinstance(d, dict):
+            return None
+        d = d.get(k, d.get(str(k)))
+    return d
 
 
 # ------------------------------------------------------------------ profiling cases

@@ -22,7 +22,7 @@ __all__ = [
     "CCA_BF16", "CCA_E4M3", "CCA_F32", "CcaError", "KVRing", "lib", "lib_path", "EXPORTED",
     "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc",
     "cca_chunk_attn_scatter", "cca_attn_workspace_size", "cca_chunk_attn_groups", "cca_block_attn",
-    "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope",
+    "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope", "cca_token_mask_l2_frames",
     "cca_token_mask_l2", "cca_compact", "cca_compact_workspace_size", "cca_scatter", "cca_selftest_bounded_wait",
     "cca_version",
     "cca_take_launch_count",
@@ -39,7 +39,7 @@ EXPORTED = (
     "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn",
     "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_chunk_attn_scatter", "cca_attn_workspace_size",
     "cca_chunk_attn_groups", "cca_block_attn", "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope",
-    "cca_token_mask_l2", "cca_compact",
+    "cca_token_mask_l2", "cca_token_mask_l2_frames", "cca_compact",
     "cca_compact_workspace_size",
     "cca_scatter", "cca_selftest_bounded_wait", "cca_last_error", "cca_version", "cca_take_launch_count",
 )
@@ -106,6 +106,7 @@ def lib() -> ctypes.CDLL:
         "cca_chunk_attn_groups": [vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, f32, vp, vp, sz, vp],
         "cca_block_attn": [ctypes.POINTER(_BlockDesc), vp, vp, f32, vp, vp, sz, vp],
         "cca_token_mask_l2": [vp, vp, i32, i32, f32, f32, vp, vp, vp, vp],
+        "cca_token_mask_l2_frames": [vp, vp, i32, i32, i32, f32, f32, vp, vp, vp, vp],
         "cca_compact": [vp, i32, vp, vp, vp, sz, vp],
         "cca_compact_workspace_size": [i32, ctypes.POINTER(sz)],
         "cca_scatter": [vp, vp, vp, i32, i32, vp, vp],
@@ -450,6 +451,22 @@ def cca_token_mask_l2(src: torch.Tensor, edit: torch.Tensor, tau: float = 0.0, p
                                    float(tau), float(prune_quantile), _ptr(mask, "mask", torch.uint8),
                                    _ptr(dist2, "dist2", torch.float32), _ptr(tau_out, "tau_out", torch.float32),
                                    _stream(stream)), "cca_token_mask_l2")
+    return mask
+
+
+def cca_token_mask_l2_frames(src: torch.Tensor, edit: torch.Tensor, tau: float = 0.0, prune_quantile: float = -1.0,
+                             mask: Optional[torch.Tensor] = None, dist2: Optional[torch.Tensor] = None,
+                             tau_out: Optional[torch.Tensor] = None, stream=None):
+    """Mask of a multi-frame chunk: src / edit [F, N, C]; one decision per position
+    from the norm over all frames and channels, written for every frame: [F * N] uint8."""
+    f, n, c = src.shape
+    if mask is None:
+        mask = torch.empty(f * n, dtype=torch.uint8, device=src.device)
+    _check(lib().cca_token_mask_l2_frames(_ptr(src, "src", torch.float32), _ptr(edit, "edit", torch.float32), f, n,
+                                          c, float(tau), float(prune_quantile), _ptr(mask, "mask", torch.uint8),
+                                          _ptr(dist2, "dist2", torch.float32),
+                                          _ptr(tau_out, "tau_out", torch.float32), _stream(stream)),
+           "cca_token_mask_l2_frames")
     return mask
 
 

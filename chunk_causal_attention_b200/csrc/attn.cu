@@ -172,14 +172,20 @@ struct AttnSmem {
 // items in rounds, item k*G + c in even rounds and k*G + G-1-c in odd ones
 // (so that rounds of unequal items even out).  When the items left after the
 // full rounds would unbalance the CTAs (one of them more than 1/8 of the
-// average load), their KV tiles are concatenated into one list cut into G
-// near-equal ranges instead: CTA c then takes the pieces of [c*tr/G,
-// (c+1)*tr/G).  A piece that covers only part of its item is "partial": its
-// (O, m, l) go to workspace slot 2c (the piece holding the range's first tile)
-// or 2c+1 (the one holding its last tile), and the combine kernel merges them.
+// average load), they are split along their KV tiles instead, in one of two
+// ways.  Aligned: with r leftover items and s = G / r >= 2, item i is cut into
+// s near-equal pieces taken by CTAs i*s .. i*s+s-1, one piece per CTA (each
+// piece pays one Q load, one pipeline fill and one partial write).  Ranges,
+// when aligned pieces would be much longer than an even share: the leftover
+// items' KV tiles are concatenated into one list cut into G near-equal ranges
+// [c*tr/G, (c+1)*tr/G), so a CTA may take two pieces.  A piece that covers
+// only part of its item is "partial": its (O, m, l) go to workspace slot 2c
+// (aligned pieces, and the piece holding a range's first tile) or 2c+1 (the
+// one holding its last tile), and the combine kernel merges them.
 struct Sched {
   int n_items, qr;  // items; whole rounds
   int rem0;         // first item of the split remainder (n_items if none)
+  int s;            // aligned mode: pieces per leftover item (0: ranges)
   int64_t tr;       // KV tiles in the remainder list (0: no split)
 };
 struct Seg {
@@ -204,6 +210,7 @@ __device__ __forceinline__ Sched make_sched(const AttnArgs &a, int n_q0, int G) 
   const int q = n / G, r = n % G;
   s.qr = q;
   s.rem0 = q * G;
+  s.s = 0;
   s.tr = 0;
   if (r > 0) {
     // longest remainder item (problems are listed by non-increasing n_kv)
@@ -220,6 +227,9 @@ __device__ __forceinline__ Sched make_sched(const AttnArgs &a, int n_q0, int G) 
     }
     if (static_cast<int64_t>(nkv_first) * 8 * G > total) {
       s.tr = tr;
+      const int pieces = G / r;  // aligned pieces per leftover item
+      const int64_t even = (tr + G - 1) / G;
+      if (pieces >= 2 && (nkv_first + pieces - 1) / pieces <= even + 2) s.s = pieces;
     } else {  // the leftover items are short next to a CTA's load: one more round of whole items
       s.qr = q + 1;
       s.rem0 = n;
@@ -280,6 +290,17 @@ __device__ __forceinline__ bool get_seg(const AttnArgs &a, int n_q0, const Sched
   }
   if (s.tr == 0) return false;
   k -= s.qr;
+  if (s.s > 0) {  // aligned: one piece of item rem0 + c / s
+    const int u = s.rem0 + c / s.s, j = c % s.s;
+    if (k > 0 || u >= s.n_items) return false;
+    int p, pair, head;
+    item_coords(a, n_q0, u, p, pair, head);
+    const int n = a.prob[p].n_kv;
+    const int j0 = j * n / s.s, j1 = (j + 1) * n / s.s;
+    if (j0 >= j1) return false;
+    g = {p, pair, head, j0, j1, 2 * c};
+    return true;
+  }
   const int64_t lo = static_cast<int64_t>(c) * s.tr / G, hi = static_cast<int64_t>(c + 1) * s.tr / G;
   int64_t t = lo;
   for (int piece = 0; t < hi; ++piece) {
@@ -1029,6 +1050,19 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
   if (sch.tr == 0) return;
   const int lane = threadIdx.x & 31;
   const int64_t tr = sch.tr;
+  // Range bounds floor(c * tr / G) and ceil(x * G / tr) in 32-bit arithmetic when
+  // every product fits (always at the sizes of one chunk), else in 64-bit.
+  const bool small = (tr + 1) * (G + 1) < (int64_t(1) << 32);
+  auto bound = [&](int64_t c) -> int64_t {
+    if (small) return static_cast<uint32_t>(c) * static_cast<uint32_t>(tr) / static_cast<uint32_t>(G);
+    return c * tr / G;
+  };
+  auto ceil_div = [&](int64_t x) -> int64_t {
+    if (small)
+      return (static_cast<uint32_t>(x) * static_cast<uint32_t>(G) + static_cast<uint32_t>(tr) - 1u) /
+             static_cast<uint32_t>(tr);
+    return (x * G + tr - 1) / tr;
+  };
   const int n_work = (sch.n_items - sch.rem0) * (kNQ * kBM);
   const int w0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -1039,16 +1073,30 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
     item_coords(a, n_q0, u, p, pair, head);
     const int row = pair * (kNQ * kBM) + rr;
     if (row >= prob_nq(a, p, n_q0)) continue;
-    const int64_t t0 = rem_offset(a, n_q0, sch, u), t1 = t0 + a.prob[p].n_kv;  // the item's tiles in the list
-    const int c_first = static_cast<int>(((t0 + 1) * G + tr - 1) / tr) - 1;
-    const int c_last = min(G - 1, static_cast<int>((t1 * G + tr - 1) / tr));
-    {  // whole inside one CTA's range: written directly by that CTA
-      const int64_t lo = static_cast<int64_t>(c_first) * tr / G, hi = static_cast<int64_t>(c_first + 1) * tr / G;
-      if (lo <= t0 && hi >= t1) continue;
+    // candidate CTAs c_first .. c_last; probe(c) says whether c holds a piece
+    // of this item and in which workspace slot
+    int c_first, c_last;
+    int64_t t0 = 0, t1 = 0;
+    const int n_kv = a.prob[p].n_kv;
+    if (sch.s > 0) {
+      c_first = ur * sch.s;
+      c_last = c_first + sch.s - 1;
+    } else {
+      t0 = rem_offset(a, n_q0, sch, u);  // the item's tiles in the list
+      t1 = t0 + n_kv;
+      c_first = static_cast<int>(ceil_div(t0 + 1)) - 1;
+      c_last = min(G - 1, static_cast<int>(ceil_div(t1)));
+      const int64_t lo = bound(c_first), hi = bound(c_first + 1);
+      if (lo <= t0 && hi >= t1) continue;  // whole inside one CTA's range: written directly by that CTA
     }
     auto probe = [&](int c, int &slot) {
       if (c > c_last) return false;
-      const int64_t lo = static_cast<int64_t>(c) * tr / G, hi = static_cast<int64_t>(c + 1) * tr / G;
+      if (sch.s > 0) {
+        const int j = c - c_first;
+        slot = 2 * c;
+        return j * n_kv / sch.s < (j + 1) * n_kv / sch.s;
+      }
+      const int64_t lo = bound(c), hi = bound(c + 1);
       slot = 2 * c + (lo >= t0 ? 0 : 1);
       return lo < hi && hi > t0 && lo < t1;
     };

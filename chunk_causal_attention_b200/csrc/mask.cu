@@ -22,31 +22,40 @@ constexpr int kMaskThreads = 256;
 constexpr int kSelectThreads = 1024;
 constexpr int kMaxSelectTokens = 32768;
 
+// Squared distance of position u over the channels of every latent frame of
+// the chunk (frames fstride elements apart; one frame for a one-frame chunk).
 __device__ __forceinline__ float token_dist2(const float *__restrict__ src, const float *__restrict__ edit,
-                                             int64_t u, int n_ch) {
-  const float4 *s = reinterpret_cast<const float4 *>(src + u * n_ch);
-  const float4 *e = reinterpret_cast<const float4 *>(edit + u * n_ch);
+                                             int64_t u, int n_ch, int n_frames, int64_t fstride) {
   float acc = 0.f;
-  for (int c = 0; c < n_ch / 4; ++c) {
-    const float4 a = __ldg(s + c), b = __ldg(e + c);
-    const float d0 = b.x - a.x, d1 = b.y - a.y, d2 = b.z - a.z, d3 = b.w - a.w;
-    acc = fmaf(d0, d0, acc);
-    acc = fmaf(d1, d1, acc);
-    acc = fmaf(d2, d2, acc);
-    acc = fmaf(d3, d3, acc);
+  for (int f = 0; f < n_frames; ++f) {
+    const float4 *s = reinterpret_cast<const float4 *>(src + f * fstride + u * n_ch);
+    const float4 *e = reinterpret_cast<const float4 *>(edit + f * fstride + u * n_ch);
+    for (int c = 0; c < n_ch / 4; ++c) {
+      const float4 a = __ldg(s + c), b = __ldg(e + c);
+      const float d0 = b.x - a.x, d1 = b.y - a.y, d2 = b.z - a.z, d3 = b.w - a.w;
+      acc = fmaf(d0, d0, acc);
+      acc = fmaf(d1, d1, acc);
+      acc = fmaf(d2, d2, acc);
+      acc = fmaf(d3, d3, acc);
+    }
   }
   return acc;
 }
 
 // Fixed threshold: one thread per token, grid-stride.
+// With n_frames > 1 the decision of position u is written for every frame:
+// mask[f * n_tok + u].
 __global__ void __launch_bounds__(kMaskThreads) mask_fixed_kernel(const float *__restrict__ src,
                                                                   const float *__restrict__ edit, int n_tok,
                                                                   int n_ch, float tau2, uint8_t *__restrict__ mask,
-                                                                  float *__restrict__ dist2, float *tau_out) {
+                                                                  float *__restrict__ dist2, float *tau_out,
+                                                                  int n_frames) {
   const int stride = gridDim.x * blockDim.x;
+  const int64_t fstride = static_cast<int64_t>(n_tok) * n_ch;
   for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < n_tok; u += stride) {
-    const float d2 = token_dist2(src, edit, u, n_ch);
-    mask[u] = d2 > tau2 ? 1 : 0;
+    const float d2 = token_dist2(src, edit, u, n_ch, n_frames, fstride);
+    const uint8_t m = d2 > tau2 ? 1 : 0;
+    for (int f = 0; f < n_frames; ++f) mask[static_cast<int64_t>(f) * n_tok + u] = m;
     if (dist2) dist2[u] = d2;
   }
   if (tau_out && blockIdx.x == 0 && threadIdx.x == 0) *tau_out = sqrtf(tau2);
@@ -57,12 +66,14 @@ __global__ void __launch_bounds__(kMaskThreads) mask_fixed_kernel(const float *_
 __global__ void __launch_bounds__(kSelectThreads) mask_select_kernel(const float *__restrict__ src,
                                                                      const float *__restrict__ edit, int n_tok,
                                                                      int n_ch, int k, uint8_t *__restrict__ mask,
-                                                                     float *__restrict__ dist2, float *tau_out) {
+                                                                     float *__restrict__ dist2, float *tau_out,
+                                                                     int n_frames) {
+  const int64_t fstride = static_cast<int64_t>(n_tok) * n_ch;
   extern __shared__ unsigned s_bits[];  // n_tok entries
   __shared__ unsigned hist[256];
   __shared__ unsigned s_prefix, s_rank;
   for (int u = threadIdx.x; u < n_tok; u += blockDim.x) {
-    const float d2 = token_dist2(src, edit, u, n_ch);
+    const float d2 = token_dist2(src, edit, u, n_ch, n_frames, fstride);
     s_bits[u] = __float_as_uint(d2);
     if (dist2) dist2[u] = d2;
   }
@@ -110,7 +121,10 @@ __global__ void __launch_bounds__(kSelectThreads) mask_select_kernel(const float
     __syncthreads();
   }
   const float tau2 = __uint_as_float(s_prefix);
-  for (int u = threadIdx.x; u < n_tok; u += blockDim.x) mask[u] = __uint_as_float(s_bits[u]) > tau2 ? 1 : 0;
+  for (int u = threadIdx.x; u < n_tok; u += blockDim.x) {
+    const uint8_t m = __uint_as_float(s_bits[u]) > tau2 ? 1 : 0;
+    for (int f = 0; f < n_frames; ++f) mask[static_cast<int64_t>(f) * n_tok + u] = m;
+  }
   if (tau_out && threadIdx.x == 0) *tau_out = sqrtf(tau2);
 }
 
@@ -448,11 +462,11 @@ __global__ void __launch_bounds__(256) scatter_kernel(const uint4 *__restrict__ 
 
 using namespace cca;
 
-extern "C" {
-
-cca_status cca_token_mask_l2(const float *src, const float *edit, int32_t n_tok, int32_t n_ch, float tau,
-                             float prune_quantile, uint8_t *mask, float *dist2_out, float *tau_out,
-                             cca_stream_t stream) {
+static cca_status token_mask_impl(const float *src, const float *edit, int32_t n_frames, int32_t n_tok,
+                                  int32_t n_ch, float tau, float prune_quantile, uint8_t *mask, float *dist2_out,
+                                  float *tau_out, cca_stream_t stream) {
+  if (n_frames < 1 || n_frames > 64 || static_cast<int64_t>(n_frames) * n_tok > (int64_t(1) << 31) - 1)
+    return fail(CCA_ERR_INVALID_ARG, "cca_token_mask_l2: need 1 <= n_frames <= 64 and n_frames * n_pos < 2^31");
   if (n_tok < 0 || n_ch < 4 || n_ch > 256 || (n_ch & 3))
     return fail(CCA_ERR_INVALID_ARG, "cca_token_mask_l2: need n_tok >= 0 and n_ch a multiple of 4 in [4, 256]");
   if (n_tok > 0 && (!src || !edit || !mask || !aligned16(src) || !aligned16(edit)))
@@ -467,7 +481,8 @@ cca_status cca_token_mask_l2(const float *src, const float *edit, int32_t n_tok,
     int blocks = (n_tok + kMaskThreads - 1) / kMaskThreads;
     const int cap = num_sms() * 8;
     if (blocks > cap) blocks = cap;
-    mask_fixed_kernel<<<blocks, kMaskThreads, 0, st>>>(src, edit, n_tok, n_ch, tau * tau, mask, dist2_out, tau_out);
+    mask_fixed_kernel<<<blocks, kMaskThreads, 0, st>>>(src, edit, n_tok, n_ch, tau * tau, mask, dist2_out, tau_out,
+                                                       n_frames);
     return launched("mask_fixed_kernel");
   }
   if (!(prune_quantile > 0.f && prune_quantile <= 1.f))
@@ -483,8 +498,22 @@ cca_status cca_token_mask_l2(const float *src, const float *edit, int32_t n_tok,
     if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "cca_token_mask_l2: %s", cudaGetErrorString(e));
   }
   mask_select_kernel<<<1, kSelectThreads, smem, st>>>(src, edit, n_tok, n_ch, k < 1 ? 1 : k, mask, dist2_out,
-                                                       tau_out);
+                                                       tau_out, n_frames);
   return launched("mask_select_kernel");
+}
+
+extern "C" {
+
+cca_status cca_token_mask_l2(const float *src, const float *edit, int32_t n_tok, int32_t n_ch, float tau,
+                             float prune_quantile, uint8_t *mask, float *dist2_out, float *tau_out,
+                             cca_stream_t stream) {
+  return token_mask_impl(src, edit, 1, n_tok, n_ch, tau, prune_quantile, mask, dist2_out, tau_out, stream);
+}
+
+cca_status cca_token_mask_l2_frames(const float *src, const float *edit, int32_t n_frames, int32_t n_pos,
+                                    int32_t n_ch, float tau, float prune_quantile, uint8_t *mask, float *dist2_out,
+                                    float *tau_out, cca_stream_t stream) {
+  return token_mask_impl(src, edit, n_frames, n_pos, n_ch, tau, prune_quantile, mask, dist2_out, tau_out, stream);
 }
 
 static size_t seg_workspace_bytes() { return static_cast<size_t>(kMaxSegCtas) * 8 + 16; }

@@ -366,6 +366,22 @@ cca_status cca_token_mask_l2(const float *src, const float *edit, int32_t n_tok,
                              uint8_t *mask, float *dist2_out, float *tau_out,
                              cca_stream_t stream);
 
+/* The mask over a chunk of several latent frames ["LiveEdit ...", section 기술
+ * 상세: inference runs chunks of 3 latent frames; the mask M^k_{u,v} is
+ * indexed by spatial position only].  Reading: one decision per position p,
+ * from the L2 norm over the channels of every frame of chunk k-1 at p, applied
+ * to the tokens of all frames of chunk k at p.
+ *  src, edit: device [n_frames][n_pos][n_ch] fp32 (frame-major, 16-byte aligned).
+ *  mask: device uint8 [n_frames][n_pos]; mask[f][p] = [d2(p) > tau2] for every f.
+ *  dist2_out: device fp32 [n_pos] or NULL; tau_out as cca_token_mask_l2.
+ *  Dynamic tau: the k-th smallest d2 over the n_pos positions, k = ceil(q n_pos)
+ *  (n_pos <= 32768).  1 <= n_frames <= 64; n_frames = 1 is cca_token_mask_l2.
+ *  Compacting the mask (cca_compact over n_frames * n_pos tokens) lists the
+ *  active tokens frame by frame, ascending.  Errors: as cca_token_mask_l2. */
+cca_status cca_token_mask_l2_frames(const float *src, const float *edit, int32_t n_frames, int32_t n_pos,
+                                    int32_t n_ch, float tau, float prune_quantile, uint8_t *mask, float *dist2_out,
+                                    float *tau_out, cca_stream_t stream);
+
 /* idx[0 .. n) = ascending positions u with mask[u] != 0; *n_active_dev = n.
  *  mask: device uint8 [n_tok]; idx: device int32 [n_tok] (entries >= n are not
  *  written); n_active_dev: device int32.

@@ -26,7 +26,8 @@ Readings where the pages are open:
 * compaction lists active positions in ascending order; scatter writes the
   recomputed rows back into the cache, leaving inactive rows untouched.
 
-Pins: the mask equals thresholding ``numpy.linalg.norm`` (a library routine);
+Pins: the mask equals thresholding ``numpy.linalg.norm`` (a library routine),
+also for multi-frame chunks (norm over frames and channels of a position);
 with dynamic tau the active count is ``N - k``; ``compact`` equals
 ``numpy.flatnonzero``; scatter leaves inactive rows bit-identical.
 """
@@ -71,6 +72,30 @@ def token_mask(src: np.ndarray, edit: np.ndarray, tau: float | None = None,
     if tau is None:
         raise ValueError("give tau or prune_quantile")
     return (d > tau).astype(np.uint8), d, float(tau)
+
+
+def token_mask_frames(src: np.ndarray, edit: np.ndarray, tau: float | None = None,
+                      prune_quantile: float | None = None):
+    """Mask of a chunk of several latent frames, src/edit [F, N, C].
+
+    The formula is indexed by spatial position (u, v) only while a chunk holds
+    3 latent frames ["LiveEdit ...", section 기술 상세]; the reading used: the
+    norm of position p runs over the channels of every frame, and its decision
+    applies to the tokens of all frames at p.  Returns (mask uint8 [F * N],
+    frame-major; d fp64 [N]; tau).
+    """
+    src = np.asarray(src, dtype=np.float64)
+    edit = np.asarray(edit, dtype=np.float64)
+    if src.shape != edit.shape or src.ndim != 3:
+        raise ValueError("src/edit must both be [F, N, C]")
+    diff = edit - src
+    d = np.sqrt(np.sum(diff * diff, axis=(0, 2)))
+    if prune_quantile is not None:
+        tau = dynamic_tau(d, prune_quantile)
+    if tau is None:
+        raise ValueError("give tau or prune_quantile")
+    m = (d > tau).astype(np.uint8)
+    return np.tile(m, src.shape[0]), d, float(tau)
 
 
 def compact(mask: np.ndarray) -> tuple[np.ndarray, int]:

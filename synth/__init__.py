@@ -29,6 +29,10 @@ Workloads (seed = index):
               reference tokens); ring = clean chunks 0..3; per-head RMS 1, bf16
   6 packed    T=8 chunks of the 720p shape in one sequence (teacher forcing):
               noisy Q/K/V and clean K/V [T, 1620, 24, 128], per-head RMS 1, bf16
+  7 liveedit  LiveEdit-shaped chunk: 3 latent frames of the 30x54 grid = 4860
+              tokens, 24 heads x 128, sink + 2-chunk window, current t=3, 4
+              denoising steps; mask latents [3, 1620, 16] with the workload-4
+              ellipse recipe (the region held over the 3 frames), dynamic tau 70 %
 """
 
 from __future__ import annotations
@@ -277,6 +281,71 @@ def grid_positions(t: int, source: int = 0, grid=(GRID_H, GRID_W), n_frames: int
     f, r, c = np.meshgrid(np.arange(n_frames), np.arange(grid[0]), np.arange(grid[1]), indexing="ij")
     n = f.size
     return np.stack([t + f.reshape(n), r.reshape(n), c.reshape(n), np.full(n, source)], axis=1).astype(np.int32)
+
+
+# ---------------------------------------------------------------- workload 7
+@dataclasses.dataclass
+class LiveEditChunk:
+    n_heads: int
+    head_dim: int
+    n_frames: int
+    chunk_len: int  # n_frames * 1620
+    window: int
+    ring_k: list
+    ring_v: list
+    t: int
+    q: list  # per denoising step [L, H, D]
+    k_cur: list
+    v_cur: list
+    src: np.ndarray  # [F, 1620, 16] fp32 latents of chunk k-1
+    edit: np.ndarray
+    prune_quantile: float
+    o_cache: np.ndarray  # [L, H, D] bf16 values
+
+
+def liveedit_chunk(seed: int = 7, n_frames: int = 3, n_steps: int = 4, n_heads: int = 24, head_dim: int = 128,
+                   window: int = 2, n_prefill: int = 3, n_ch: int = 16, coverage: float = 0.30,
+                   tol: float = 0.02) -> LiveEditChunk:
+    """Workload 7.  Chunk size (3 latent frames) and step count (4) are the
+    LiveEdit page's; grid, heads, head size, window and channel count are not
+    on that page and follow the other workloads."""
+    g = rng(seed)
+    L = n_frames * TOKENS_720P
+    shape = (L, n_heads, head_dim)
+
+    def draw():
+        return bf16_round(_head_rms_one(g.standard_normal(shape, dtype=np.float32)))
+
+    ring_k, ring_v = [], []
+    for _ in range(n_prefill):
+        ring_k.append(draw())
+        ring_v.append(draw())
+    q, kc, vc = [], [], []
+    for _ in range(n_steps):
+        q.append(draw())
+        kc.append(draw())
+        vc.append(draw())
+    n = TOKENS_720P
+    src = g.standard_normal((n_frames, n, n_ch), dtype=np.float32)
+    n_ell = int(g.integers(1, 5))
+    centres = np.stack([g.uniform(0, GRID_H, n_ell), g.uniform(0, GRID_W, n_ell)], axis=1)
+    axes = np.stack([g.uniform(0.3, 1.0, n_ell) * GRID_W / 4, g.uniform(0.3, 1.0, n_ell) * GRID_H / 4], axis=1)
+    angles = g.uniform(0, np.pi, n_ell)
+    lo, hi = 0.0, 8.0
+    region = _ellipse_union(centres, axes, angles, hi)
+    for _ in range(60):
+        mid = 0.5 * (lo + hi)
+        region = _ellipse_union(centres, axes, angles, mid)
+        cov = region.mean()
+        if abs(cov - coverage) <= tol:
+            break
+        lo, hi = (mid, hi) if cov < coverage else (lo, mid)
+    off_in = g.normal(2.0, 1.0, size=(n_frames, n, n_ch))
+    off_out = g.normal(0.0, 0.1, size=(n_frames, n, n_ch))
+    edit = (src + np.where(region[None, :, None], off_in, off_out)).astype(np.float32)
+    o_cache = bf16_round(g.normal(0.0, 0.02, size=shape).astype(np.float32))
+    return LiveEditChunk(n_heads, head_dim, n_frames, L, window, ring_k, ring_v, n_prefill, q, kc, vc, src, edit,
+                         0.70, o_cache)
 
 
 def as_torch_bf16(x: np.ndarray, device="cpu") -> torch.Tensor:

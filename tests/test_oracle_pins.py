@@ -421,3 +421,21 @@ def test_planted_round_half_away_is_caught():
         return np.copysign(np.floor(a / qn + 0.5) * qn, x)
     tie = np.array([1.0625])
     assert enc_half_away(tie)[0] != fp8.e4m3_decode(fp8.e4m3_encode(tie))[0]
+
+
+def test_mask_frames_is_thresholded_norm_over_frames_and_channels():
+    g = np.random.default_rng(41)
+    F, N, C = 3, 200, 16
+    src = g.standard_normal((F, N, C)).astype(np.float32)
+    edit = (src + g.normal(0, 1, (F, N, C))).astype(np.float32)
+    m, d, tau = mc.token_mask_frames(src, edit, tau=5.0)
+    # library routine on the position-major layout [N, F * C]
+    ref = np.linalg.norm((edit.astype(np.float64) - src).transpose(1, 0, 2).reshape(N, F * C), axis=1)
+    assert np.allclose(d, ref, rtol=1e-14, atol=0)
+    assert np.array_equal(m, np.tile((ref > 5.0).astype(np.uint8), F))
+    m2, _, tau2 = mc.token_mask_frames(src, edit, prune_quantile=0.7)
+    assert m2.reshape(F, N).sum(axis=1).tolist() == [N - math.ceil(0.7 * N)] * F
+    # a one-frame chunk is the per-token mask
+    m1, d1, _ = mc.token_mask_frames(src[:1], edit[:1], tau=3.0)
+    t1, e1, _ = mc.token_mask(src[0], edit[0], tau=3.0)
+    assert np.array_equal(m1, t1) and np.allclose(d1, e1, rtol=1e-15, atol=0)
