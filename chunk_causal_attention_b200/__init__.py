@@ -22,7 +22,7 @@ __all__ = [
     "CCA_BF16", "CCA_E4M3", "CCA_F32", "CcaError", "KVRing", "lib", "lib_path", "EXPORTED",
     "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc",
     "cca_chunk_attn_scatter", "cca_attn_workspace_size", "cca_chunk_attn_groups", "cca_block_attn",
-    "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope", "cca_token_mask_l2_frames",
+    "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope", "cca_token_mask_l2_frames", "cca_quant_e4m3_f16",
     "cca_token_mask_l2", "cca_compact", "cca_compact_workspace_size", "cca_scatter", "cca_selftest_bounded_wait",
     "cca_version",
     "cca_take_launch_count",
@@ -36,7 +36,7 @@ _STATUS = {0: "CCA_OK", 1: "CCA_ERR_INVALID_ARG", 2: "CCA_ERR_UNSUPPORTED", 3: "
 # Every entry point declared in include/cca.h.
 EXPORTED = (
     "cca_kv_ring_create", "cca_kv_ring_destroy", "cca_kv_ring_reset", "cca_kv_ring_query",
-    "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn",
+    "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_quant_e4m3_f16", "cca_chunk_attn",
     "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_chunk_attn_scatter", "cca_attn_workspace_size",
     "cca_chunk_attn_groups", "cca_block_attn", "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope",
     "cca_token_mask_l2", "cca_token_mask_l2_frames", "cca_compact",
@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
         "cca_kv_ring_restore": [vp, i64],
         "cca_kv_append": [vp, vp, vp, ctypes.c_int, vp],
         "cca_quant_e4m3": [vp, ctypes.c_int, i32, i32, i32, vp, vp, vp],
+        "cca_quant_e4m3_f16": [vp, ctypes.c_int, i32, i32, i32, vp, vp, vp],
         "cca_chunk_attn": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp],
         "cca_chunk_attn_workspace_size": [vp, i32, ctypes.POINTER(sz)],
         "cca_chunk_attn_noalloc": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp],
@@ -167,7 +168,8 @@ class KVRing:
     """Bounded KV cache: sink slot + W window slots per tensor, on one device.
 
     Owns the device buffers (allocated with torch) and the C handle.
-    k_slots / v_slots: [(1+W), L, H, D] (bf16 or uint8 e4m3 codes);
+    k_slots / v_slots: [(1+W), L, H, D] (bf16; e4m3: uint8 codes for K and
+    fp16-widened e4m3 values for V);
     k_scale / v_scale: [(1+W), H] fp32 (e4m3 only); status: int32[1].
     """
 
@@ -186,7 +188,7 @@ class KVRing:
             cdt = CCA_BF16
         elif dtype == "e4m3":
             self.k_slots = torch.empty(shape, dtype=torch.uint8, device=device)
-            self.v_slots = torch.empty(shape, dtype=torch.uint8, device=device)
+            self.v_slots = torch.empty(shape, dtype=torch.float16, device=device)  # widened e4m3 values
             self.k_scale = torch.ones((1 + window, n_heads), dtype=torch.float32, device=device)
             self.v_scale = torch.ones((1 + window, n_heads), dtype=torch.float32, device=device)
             cdt = CCA_E4M3
@@ -290,6 +292,20 @@ def cca_quant_e4m3(x: torch.Tensor, x8: Optional[torch.Tensor] = None, scale: Op
     _check(lib().cca_quant_e4m3(_ptr(x, "x"), _src_dtype(x), n, h, d, _ptr(x8, "x8", torch.uint8),
                                 _ptr(scale, "scale", torch.float32), _stream(stream)), "cca_quant_e4m3")
     return x8, scale
+
+
+def cca_quant_e4m3_f16(x: torch.Tensor, x16: Optional[torch.Tensor] = None, scale: Optional[torch.Tensor] = None,
+                       stream=None):
+    """Per-head absmax e4m3 quantisation of x [n, H, D] returning the codes' values
+    widened to fp16 (the V-side form of E4M3 attention) and the scales."""
+    n, h, d = x.shape
+    if x16 is None:
+        x16 = torch.empty((n, h, d), dtype=torch.float16, device=x.device)
+    if scale is None:
+        scale = torch.empty(h, dtype=torch.float32, device=x.device)
+    _check(lib().cca_quant_e4m3_f16(_ptr(x, "x"), _src_dtype(x), n, h, d, _ptr(x16, "x16", torch.float16),
+                                    _ptr(scale, "scale", torch.float32), _stream(stream)), "cca_quant_e4m3_f16")
+    return x16, scale
 
 
 def cca_chunk_attn_workspace_size(ring: KVRing, n_q_max: int) -> int:
@@ -421,7 +437,7 @@ def cca_block_attn(q: torch.Tensor, k_cur: torch.Tensor, v_cur: torch.Tensor, wi
     to R, history chunks {0} U {max(1, c-W) .. c-1} (k_hist / v_hist, default the
     current tensors) and itself.  Returns out [T, L, H, D] bf16."""
     T, L, H, D = q.shape
-    fp8 = q.dtype == torch.uint8
+    fp8 = q.dtype == torch.uint8  # e4m3: q/k codes, v fp16-widened values
     if k_hist is None:
         k_hist, v_hist, khist_scale, vhist_scale = k_cur, v_cur, kcur_scale, vcur_scale
     if out is None:

@@ -13,9 +13,8 @@
 //  * one work item = two 128-row Q tiles (256 queries) of one head x a range
 //    of 128-row KV tiles; both Q tiles share every K/V tile loaded into shared
 //    memory, halving L2->SM traffic per FLOP;
-//  * warp 0 = TMA producer of Q (once per item) and K (3-stage ring); bf16:
-//    warp 2 = TMA producer of V (2 stages), warp 3 idle; e4m3: warp 0 loads V
-//    too and warps 2-3 expand each e4m3 V tile to fp16 (64 rows each);
+//  * warp 0 = TMA producer of Q (once per item) and K (3-stage ring); warp 2 =
+//    TMA producer of V (2 stages; for e4m3 the fp16-widened values); warp 3 idle;
 //    warp 1 = TMEM allocator and the single thread issuing tcgen05.mma;
 //    warps 4-7 / 8-11 = softmax warpgroups, one per Q tile, one row per thread;
 //  * TMEM (512 columns): S0 | S1 | O0 | O1.  S = Q K^T lands in TMEM; the
@@ -41,6 +40,8 @@
 #include <cstdlib>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <initializer_list>
 #include <mutex>
 #include <vector>
@@ -129,6 +130,9 @@ struct AttnArgs {
   int scatter_out;         // 1: query i's row goes to out row q_idx[i] (fused scatter-back)
   float *ws_o;             // [2 x grid][256][D] partial O of split items (unnormalised)
   float *ws_ml;            // [2 x grid][256][2] (running max in log2 units, row sum)
+  unsigned long long *ws_flag;  // [grid] piece-done flags of the in-kernel merge
+  unsigned long long token;     // value this launch writes into the flags (unique per launch)
+  int merge_in_kernel;     // 1: launched cooperatively; aligned pieces are merged by their CTAs
   int32_t *dev_status;
   // e4m3 only: per-head dequantisation scales, [slots][H] per tensor.
   const float *q_scale;
@@ -146,21 +150,22 @@ struct AttnArgs {
 };
 
 // Shared-memory plan.  Q/K/V tiles arrive by TMA as 128-row x 128-byte boxes
-// with the 128-byte swizzle (two boxes per tile for bf16 D=128).  For e4m3, V
-// tiles are expanded to fp16 in a separate buffer for the 16-bit PV MMA.
+// with the 128-byte swizzle (two boxes per tile for 16-bit D=128).  V is
+// always 16-bit: bf16, or for e4m3 the e4m3 values widened to fp16 (the PV
+// product keeps P in 16 bits, so its B operand is 16-bit too).
 template <int D, bool kFp8>
 struct AttnSmem {
-  static constexpr uint32_t kEsz = kFp8 ? 1 : 2;             // bytes per Q/K/V element
+  static constexpr uint32_t kEsz = kFp8 ? 1 : 2;             // bytes per Q/K element
   static constexpr uint32_t kBox = 128 * 128;                // 128 rows x 128 bytes
-  static constexpr uint32_t kNBox = D * kEsz / 128;          // boxes per 128-row tile
-  static constexpr uint32_t kTile = kBox * kNBox;            // bytes of one loaded Q/K/V tile
-  static constexpr uint32_t kV16Tile = kFp8 ? 128 * D * 2 : 0;
+  static constexpr uint32_t kNBox = D * kEsz / 128;          // boxes per 128-row Q/K tile
+  static constexpr uint32_t kTile = kBox * kNBox;            // bytes of one loaded Q/K tile
+  static constexpr uint32_t kNBoxV = D * 2 / 128;            // boxes per 128-row V tile
+  static constexpr uint32_t kVTile = kBox * kNBoxV;          // bytes of one loaded V tile
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + kNQ * kTile;
   static constexpr uint32_t kV = kK + kNSK * kTile;
-  static constexpr uint32_t kV16 = kV + kNSV * kTile;
-  static constexpr uint32_t kBar = kV16 + kNSV * kV16Tile;
-  static constexpr uint32_t kNumBars = 4 + 2 * kNSK + 4 * kNSV + 8 + 1 + 2;
+  static constexpr uint32_t kBar = kV + kNSV * kVTile;
+  static constexpr uint32_t kNumBars = 4 + 2 * kNSK + 2 * kNSV + 8 + 1 + 2;
   static constexpr uint32_t kBytes = kBar + kNumBars * 8 + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
@@ -375,9 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *k_empty = k_full + kNSK;     // [kNSK]
   uint64_t *v_full = k_empty + kNSK;     // [kNSV] V tile landed
   uint64_t *v_empty = v_full + kNSV;     // [kNSV] V tile consumed (MMA, or the e4m3 expander)
-  uint64_t *v16_full = v_empty + kNSV;   // [kNSV] e4m3: fp16 V ready
-  uint64_t *v16_empty = v16_full + kNSV; // [kNSV] e4m3: fp16 V consumed by the MMAs
-  uint64_t *s_full = v16_empty + kNSV;   // [2] MMA -> softmax: S ready
+  uint64_t *s_full = v_empty + kNSV;     // [2] MMA -> softmax: S ready
   uint64_t *p_full = s_full + 2;        // [2] softmax -> MMA: P ready (and O rescaled)
   uint64_t *o_full = p_full + 2;        // [2] MMA -> softmax: O final for the item
   uint64_t *o_empty = o_full + 2;       // [2] softmax -> MMA: O read out
@@ -411,9 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kNSV; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], kFp8 ? 2 : 1);  // released by the MMA (bf16) or both e4m3 expander warps
-      mbar_init(&v16_full[s], kFp8 ? 2 : 1);
-      mbar_init(&v16_empty[s], 1);
+      mbar_init(&v_empty[s], 1);  // released by the MMA
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -446,7 +447,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     CCA_TRACE_ROLE(0);
     uint32_t g = 0;   // KV tiles handled by this CTA
     uint32_t gk = 0;  // K tile loads armed
-    uint32_t gvk = 0; // e4m3: V tile loads armed
     int it = 0;       // items handled by this CTA
     int q_armed = 0;  // Q phases armed (per tile, identical for both)
     bool ok = true;
@@ -524,20 +524,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (uint32_t b = 0; b < S::kNBox; ++b)
             tma_load_4d(kmap(src), &k_full[stage], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
         }
-        if constexpr (kFp8) {
-          // e4m3: V tiles come from this warp too; the expanders free a V slot as
-          // soon as it is converted, so it never holds back the K loads for long.
-          const uint32_t vst = g % kNSV, vph = (g / kNSV) & 1;
-          if (g >= kNSV) ok = __all_sync(0xffffffffu, mbar_wait(&v_empty[vst], vph ^ 1, abort_flag, budget));
-          if (!ok) break;
-          ++gvk;
-          if (lane == 0) {
-            const uint32_t dst = base + S::kV + vst * S::kTile;
-            mbar_arrive_expect_tx(&v_full[vst], S::kTile);
-            for (uint32_t b = 0; b < S::kNBox; ++b)
-              tma_load_4d(vmap(src), &v_full[vst], dst + b * S::kBox, b * kBoxElems, head, row0, slot);
-          }
-        }
       }
       ++it;
     }
@@ -550,10 +536,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (q_armed > 0)
         for (int i = 0; i < kNQ; ++i) mbar_drain(&q_full[i], (q_armed - 1) & 1, budget);
-      for (uint32_t k = 0; k < kNSV && k < gvk; ++k) {
-        const uint32_t gg = gvk - 1 - k;
-        mbar_drain(&v_full[gg % kNSV], (gg / kNSV) & 1, budget);
-      }
     }
   }
   // ================================================================ MMA issuer
@@ -572,10 +554,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // an add to the (address >> 4) field.
     const uint64_t dQ0 = sdesc_sw128(base + S::kQ, 16, 1024);
     const uint64_t dK0 = sdesc_sw128(base + S::kK, 16, 1024);
-    const uint64_t dV0 = kFp8 ? sdesc_sw128(base + S::kV16, 128 * 128, 1024) : sdesc_sw128(base + S::kV, S::kBox, 1024);
-    constexpr uint32_t kVStageBytes = kFp8 ? S::kV16Tile : S::kTile;
-    uint64_t *pv_full = kFp8 ? v16_full : v_full;
-    uint64_t *pv_empty = kFp8 ? v16_empty : v_empty;
+    const uint64_t dV0 = sdesc_sw128(base + S::kV, S::kBox, 1024);
+    constexpr uint32_t kVStageBytes = S::kVTile;
+    uint64_t *pv_full = v_full;
+    uint64_t *pv_empty = v_empty;
     auto issue_qk = [=](int i, uint32_t stage) {
       const uint64_t qa = dQ0 + ((i * S::kTile) >> 4), kb = dK0 + ((stage * S::kTile) >> 4);
       const uint32_t d = tm + i * 128u;
@@ -685,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
   // ================================================================ V producer
-  else if (warp == 2 && !kFp8) {
+  else if (warp == 2) {
     if (kUseSetMaxNReg) regs_dec<88>();
     // V tiles run on their own warp so a V slot that frees late (after the PV
     // MMAs) never holds back the next K loads.
@@ -705,10 +687,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ++gv;
         if (lane == 0) {
-          const uint32_t dst = base + S::kV + stage * S::kTile;
-          mbar_arrive_expect_tx(&v_full[stage], S::kTile);
-          for (uint32_t b = 0; b < S::kNBox; ++b)
-            tma_load_4d(vmap(src), &v_full[stage], dst + b * S::kBox, b * kBoxElems, sg.head, row0, slot);
+          const uint32_t dst = base + S::kV + stage * S::kVTile;
+          mbar_arrive_expect_tx(&v_full[stage], S::kVTile);
+          for (uint32_t b = 0; b < S::kNBoxV; ++b)
+            tma_load_4d(vmap(src), &v_full[stage], dst + b * S::kBox, b * 64, sg.head, row0, slot);
         }
       }
     }
@@ -718,60 +700,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_drain(&v_full[gg % kNSV], (gg / kNSV) & 1, budget);
       }
   }
-  // ================================================================ e4m3 V expanders
-  else if (warp < 4) {
+  // ================================================================ idle
+  else if (warp == 3) {
     if (kUseSetMaxNReg) regs_dec<88>();
-    if constexpr (kFp8) {
-      // Warps 2 and 3 turn each landed e4m3 V tile (128 rows x 128 bytes,
-      // swizzled) into an fp16 tile (two 128 x 64 boxes, swizzled) for the PV
-      // MMA, 64 rows each.  The conversion is exact: every e4m3 value is an
-      // fp16 value.
-      uint32_t g = 0;
-      bool ok = true;
-      for (int kseg = 0; ok; ++kseg) {
-        Seg sg;
-        if (!get_seg(a, n_q0, sch, gridDim.x, blockIdx.x, kseg, sg)) break;
-        for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-          const uint32_t stage = g % kNSV, ph = (g / kNSV) & 1;
-          ok = __all_sync(0xffffffffu, mbar_wait(&v_full[stage], ph, abort_flag, budget));
-          if (ok && g >= kNSV) ok = __all_sync(0xffffffffu, mbar_wait(&v16_empty[stage], ph ^ 1, abort_flag, budget));
-          if (!ok) break;
-          const uint32_t src = base + S::kV + stage * S::kTile;
-          const uint32_t dst = base + S::kV16 + stage * S::kV16Tile;
-#pragma unroll 4
-          for (int e = (warp - 2) * 512 + lane; e < (warp - 1) * 512; e += 32) {  // 16-byte source chunks
-            const int r = e >> 3, c = e & 7;
-            uint32_t w[4];
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                         : "r"(src + r * 128 + ((c ^ (r & 7)) << 4)));
-            uint32_t h[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[k] & 0xffffu), __NV_E4M3);
-              const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[k] >> 16), __NV_E4M3);
-              h[2 * k] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
-              h[2 * k + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
-            }
-            // elements 16c .. 16c+15 -> box (c >> 2), 16-byte chunks 2(c&3) and 2(c&3)+1
-            const uint32_t ob = dst + (c >> 2) * (128 * 128) + r * 128;
-            const uint32_t c0 = (2 * (c & 3)) ^ (r & 7), c1 = (2 * (c & 3) + 1) ^ (r & 7);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ob + (c0 << 4)), "r"(h[0]), "r"(h[1]),
-                         "r"(h[2]), "r"(h[3])
-                         : "memory");
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ob + (c1 << 4)), "r"(h[4]), "r"(h[5]),
-                         "r"(h[6]), "r"(h[7])
-                         : "memory");
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&v16_full[stage]);
-            mbar_arrive(&v_empty[stage]);
-          }
-        }
-      }
-    }
   }
   // ================================================================ softmax
   else {
@@ -1013,6 +944,88 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // Aligned pieces of a leftover item are merged by the CTAs that computed them
+  // (all resident: cooperative launch): each publishes its piece with the
+  // launch's token, waits (bounded) for the other pieces of its item, then the
+  // softmax warps merge its share of the item's 256 rows.
+  if (a.merge_in_kernel && sch.s > 0 && sch.tr > 0 && !*abort_flag) {
+    const int G = gridDim.x, c = blockIdx.x;
+    const int u = sch.rem0 + c / sch.s;
+    if (u < sch.n_items) {
+      const int c_first = c - c % sch.s, j_me = c % sch.s;
+      int p, pair, head;
+      item_coords(a, n_q0, u, p, pair, head);
+      const int n_kv = a.prob[p].n_kv;
+      if (threadIdx.x == 0) {
+        __threadfence();
+        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(a.ws_flag + c), "l"(a.token) : "memory");
+      }
+      __shared__ int s_ok;
+      if (threadIdx.x == 32) {  // warp 1, lane 0: wait for every non-empty piece of the item
+        int ok = 1;
+        const long long t0 = clock64();
+        for (int j = 0; j < sch.s && ok; ++j) {
+          if (j * n_kv / sch.s >= (j + 1) * n_kv / sch.s) continue;  // empty piece: nothing published
+          while (true) {
+            unsigned long long f;
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(f) : "l"(a.ws_flag + c_first + j) : "memory");
+            if (f == a.token) break;
+            if (clock64() - t0 > budget) {
+              ok = 0;
+              break;
+            }
+          }
+        }
+        s_ok = ok;
+        if (!ok && a.dev_status) atomicExch(a.dev_status, CCA_DEV_TIMEOUT);
+      }
+      __syncthreads();
+      (void)G;
+      if (s_ok && warp >= 4) {
+        constexpr int kV = D / 32;
+        const int n_q = prob_nq(a, p, n_q0);
+        const int r0 = j_me * (kNQ * kBM) / sch.s, r1 = (j_me + 1) * (kNQ * kBM) / sch.s;
+        for (int rr = r0 + (warp - 4); rr < r1; rr += 8) {
+          const int row = pair * (kNQ * kBM) + rr;
+          if (row >= n_q) break;
+          float mmax = -INFINITY;
+          for (int j = 0; j < sch.s; ++j) {
+            if (j * n_kv / sch.s >= (j + 1) * n_kv / sch.s) continue;
+            mmax = fmaxf(mmax, __ldcg(a.ws_ml + (static_cast<int64_t>(2 * (c_first + j)) * (kNQ * kBM) + rr) * 2));
+          }
+          float den = 0.f, acc[kV];
+#pragma unroll
+          for (int k = 0; k < kV; ++k) acc[k] = 0.f;
+          for (int j = 0; j < sch.s; ++j) {
+            if (j * n_kv / sch.s >= (j + 1) * n_kv / sch.s) continue;
+            const int64_t prow = static_cast<int64_t>(2 * (c_first + j)) * (kNQ * kBM) + rr;
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(a.ws_ml + prow * 2));
+            const float w = exp2f(ml.x - mmax);
+            den += w * ml.y;
+            const float *o = a.ws_o + prow * D + lane * kV;
+            if constexpr (kV == 4) {
+              const float4 v = __ldcg(reinterpret_cast<const float4 *>(o));
+              acc[0] += w * v.x, acc[1] += w * v.y, acc[2] += w * v.z, acc[3] += w * v.w;
+            } else {
+              const float2 v = __ldcg(reinterpret_cast<const float2 *>(o));
+              acc[0] += w * v.x, acc[1] += w * v.y;
+            }
+          }
+          const float inv = 1.f / den;
+          const int orow = a.scatter_out ? __ldg(a.q_idx + row) : row;
+          if (orow < 0 || orow >= a.out_rows) continue;
+          __nv_bfloat16 *dst =
+              a.out + ((static_cast<int64_t>(a.prob[p].out_slot) * a.out_rows + orow) * a.H + head) * D + lane * kV;
+          if constexpr (kV == 4) {
+            *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
+                                                         pack_bf16x2(acc[2] * inv, acc[3] * inv));
+          } else {
+            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+          }
+        }
+      }
+    }
+  }
   if (threadIdx.x == 0 && *abort_flag && a.dev_status) atomicExch(a.dev_status, CCA_DEV_TIMEOUT);
 }
 
@@ -1047,7 +1060,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n_q0 = a.n_q_dev ? min(max(*a.n_q_dev, 0), a.prob[0].n_q) : a.prob[0].n_q;
   const Sched sch = make_sched(a, n_q0, G);
-  if (sch.tr == 0) return;
+  if (sch.tr == 0 || (sch.s > 0 && a.merge_in_kernel)) return;  // nothing split, or merged in the attention kernel
   const int lane = threadIdx.x & 31;
   const int64_t tr = sch.tr;
   // Range bounds floor(c * tr / G) and ceil(x * G / tr) in 32-bit arithmetic when
@@ -1247,10 +1260,11 @@ static int attn_grid(int64_t work) {
   return g;
 }
 
-// Partial-piece slots: 2 per CTA, 256 rows each, O (D fp32) plus (m, l).
+// Partial-piece slots: 2 per CTA, 256 rows each, O (D fp32) plus (m, l); then
+// one 8-byte merge flag per CTA.
 static size_t workspace_bytes_for_grid(int grid, int D) {
   const size_t rows = static_cast<size_t>(2) * grid * (kNQ * kBM);
-  return rows * (static_cast<size_t>(D) + 2) * sizeof(float) + 256;
+  return rows * (static_cast<size_t>(D) + 2) * sizeof(float) + static_cast<size_t>(grid) * 8 + 256;
 }
 
 // Workspace that suffices for every attention launch with this head_dim on
@@ -1261,8 +1275,9 @@ static size_t workspace_bytes_any(int D) {
   return workspace_bytes_for_grid(g, D);
 }
 
-// Host copy of the device schedule's decision: does any item get split?
-static bool host_splits(const AttnArgs &a, int G) {
+// Host copy of the device schedule's decision (make_sched with every
+// problem's n_q): 0 = no item split, 1 = ranges, 2 = aligned pieces.
+static int host_split_mode(const AttnArgs &a, int G) {
   int n = 0;
   int64_t total = 0;
   for (int p = 0; p < a.n_prob; ++p) {
@@ -1271,14 +1286,30 @@ static bool host_splits(const AttnArgs &a, int G) {
     total += static_cast<int64_t>(cnt) * a.prob[p].n_kv;
   }
   const int q = n / G, r = n % G;
-  if (r == 0) return false;
-  int i0 = 0;
+  if (r == 0) return 0;
+  int i0 = 0, nkv_first = 0;
+  int64_t tr = 0;
   for (int p = 0; p < a.n_prob; ++p) {
     const int cnt = (a.prob[p].n_q + kNQ * kBM - 1) / (kNQ * kBM) * a.H, i1 = i0 + cnt;
-    if (i1 > q * G) return static_cast<int64_t>(a.prob[p].n_kv) * 8 * G > total;
+    const int b0 = i0 > q * G ? i0 : q * G;
+    if (b0 < i1) {
+      if (tr == 0) nkv_first = a.prob[p].n_kv;
+      tr += static_cast<int64_t>(i1 - b0) * a.prob[p].n_kv;
+    }
     i0 = i1;
   }
-  return false;
+  if (static_cast<int64_t>(nkv_first) * 8 * G <= total) return 0;
+  const int pieces = G / r;
+  const int64_t even = (tr + G - 1) / G;
+  return pieces >= 2 && (nkv_first + pieces - 1) / pieces <= even + 2 ? 2 : 1;
+}
+
+// Unique value per launch for the merge flags (a per-process counter above a
+// seed from the clock, so stale flags of earlier launches never match).
+static unsigned long long next_token() {
+  static std::atomic<unsigned long long> ctr{
+      (static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count()) << 20) | 1ull};
+  return ctr.fetch_add(1ull);
 }
 
 static std::mutex g_attr_mu;
@@ -1289,6 +1320,8 @@ static cca_status launch_attn(AttnLaunch &L, void *workspace, size_t workspace_b
   AttnArgs &args = L.args;
   const int H = args.H;
   const CUtensorMapDataType dt = kFp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // V is 16-bit in both modes: bf16, or the e4m3 values widened to fp16
+  const CUtensorMapDataType dt_v = kFp8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int es = kFp8 ? 1 : 2;
   const int grid = attn_grid(L.work);
   const size_t need = workspace_bytes_for_grid(grid, D);
@@ -1296,6 +1329,9 @@ static cca_status launch_attn(AttnLaunch &L, void *workspace, size_t workspace_b
     return fail(CCA_ERR_INVALID_ARG, "attention: workspace of %zu bytes (16-byte aligned) required", need);
   args.ws_o = static_cast<float *>(workspace);
   args.ws_ml = args.ws_o + static_cast<size_t>(2) * grid * (kNQ * kBM) * D;
+  args.ws_flag = reinterpret_cast<unsigned long long *>(
+      (reinterpret_cast<uintptr_t>(args.ws_ml + static_cast<size_t>(2) * grid * (kNQ * kBM) * 2) + 15) & ~uintptr_t(15));
+  args.token = next_token();
   CUtensorMap tq, tk[kMaxSrc], tv[kMaxSrc];
   std::memset(&tq, 0, sizeof(tq));
   if (!args.q_idx) CCA_TRY(make_tmap(&tq, L.q, dt, es, D, H, L.q_rows_map, L.q_slots));
@@ -1305,26 +1341,62 @@ static cca_status launch_attn(AttnLaunch &L, void *workspace, size_t workspace_b
     const void *kp = used ? L.k[s] : L.k[1], *vp = used ? L.v[s] : L.v[1];
     const int rows = used ? args.src_len[s] : args.src_len[1], slots = used ? L.src_slots[s] : L.src_slots[1];
     CCA_TRY(make_tmap(&tk[s], kp, dt, es, D, H, rows, slots));
-    CCA_TRY(make_tmap(&tv[s], vp, dt, es, D, H, rows, slots));
+    CCA_TRY(make_tmap(&tv[s], vp, dt_v, 2, D, H, rows, slots));
   }
+  int resident = 0;  // co-resident CTAs on this device (1 per SM at this shared-memory size)
   {
     // The shared-memory opt-in is per device and kernel: set it once per device.
     static bool done[64] = {false};
+    static int max_blocks[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lk(g_attr_mu);
     if (dev < 0 || dev >= 64 || !done[dev]) {
-      const cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(S::kAlloc));
+      cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(S::kAlloc));
       if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "attention: %s", cudaGetErrorString(e));
-      if (dev >= 0 && dev < 64) done[dev] = true;
+      int per_sm = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_kernel<D, kFp8>, kThreads, S::kAlloc);
+      if (e != cudaSuccess) per_sm = 0;
+      if (dev >= 0 && dev < 64) {
+        done[dev] = true;
+        max_blocks[dev] = per_sm * num_sms();
+      } else {
+        resident = per_sm * num_sms();
+      }
     }
+    if (dev >= 0 && dev < 64) resident = max_blocks[dev];
   }
-  attn_kernel<D, kFp8><<<grid, kThreads, S::kAlloc, st>>>(tq, tk[0], tv[0], tk[1], tv[1], tk[2], tv[2], args);
-  CCA_TRY(launched("attn_kernel"));
-  // Split items exist unless the item count is known on the host and the
-  // schedule gives every item to one CTA.
-  if (args.n_q_dev != nullptr || host_splits(args, grid)) {
+  // Aligned pieces are merged inside the attention kernel when every CTA is
+  // resident at once (a cooperative launch guarantees it); otherwise by the
+  // combine kernel.
+  const int mode = host_split_mode(args, grid);
+  const bool maybe_aligned = args.n_q_dev != nullptr || mode == 2;
+  args.merge_in_kernel = maybe_aligned && grid <= resident && env_int("CCA_MERGE_IN_KERNEL", 1) != 0;
+  {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = S::kAlloc;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = args.merge_in_kernel ? 1 : 0;
+    const cudaError_t le =
+        cudaLaunchKernelEx(&cfg, attn_kernel<D, kFp8>, tq, tk[0], tv[0], tk[1], tv[1], tk[2], tv[2], args);
+    if (le != cudaSuccess) {
+      cudaGetLastError();
+      return fail(CCA_ERR_CUDA, "attention: launch failed: %s", cudaGetErrorString(le));
+    }
+    CCA_TRY(launched("attn_kernel"));
+  }
+  // The combine kernel runs unless the host knows the schedule splits nothing,
+  // or splits in aligned pieces that the attention kernel merges itself.
+  const bool need_combine = args.n_q_dev != nullptr || mode == 1 || (mode == 2 && !args.merge_in_kernel);
+  if (need_combine) {
     const int64_t warps = static_cast<int64_t>(grid) * (kNQ * kBM);
     int64_t blocks = (warps + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;

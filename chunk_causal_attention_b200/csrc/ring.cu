@@ -92,35 +92,14 @@ constexpr int kAppendUnroll = 10;
 constexpr int64_t kMaxChunkElems = int64_t(1) << 33;  // keeps 16-byte vector indices below 2^30
 constexpr int kAppendUnrollF32 = 4;  // fp32 sources: two 16-byte loads per output
 
-// With kRope, K (blockIdx.y == 0) is rotated on the way (rope.cuh): its 16-byte
-// vectors are expanded to fp32, turned and rounded to bf16 once.
-__device__ __forceinline__ uint4 rope_bf16x8(const RopeArgs &r, uint4 u, int64_t tok, int d0, int D) {
-  float x[8];
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    x[2 * j] = __uint_as_float(w[j] << 16);
-    x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-  }
-  rope8(r, tok, d0, D, x);
-  return to_bf16x8(make_float4(x[0], x[1], x[2], x[3]), make_float4(x[4], x[5], x[6], x[7]));
-}
-__device__ __forceinline__ uint4 rope_f32x8(const RopeArgs &r, float4 a, float4 b, int64_t tok, int d0, int D) {
-  float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-  rope8(r, tok, d0, D, x);
-  return to_bf16x8(make_float4(x[0], x[1], x[2], x[3]), make_float4(x[4], x[5], x[6], x[7]));
-}
-
-template <bool kF32, bool kRope>
+template <bool kF32>
 __global__ void __launch_bounds__(256, 4) append_bf16_kernel(const void *__restrict__ k_src,
                                                              const void *__restrict__ v_src,
                                                              uint4 *__restrict__ k_dst,
-                                                             uint4 *__restrict__ v_dst, int n_vec, RopeArgs rk,
-                                                             int vec_per_tok, int D) {
+                                                             uint4 *__restrict__ v_dst, int n_vec) {
   constexpr int kU = kF32 ? kAppendUnrollF32 : kAppendUnroll;
   const void *src = blockIdx.y == 0 ? k_src : v_src;
   uint4 *dst = blockIdx.y == 0 ? k_dst : v_dst;
-  const bool rot = kRope && blockIdx.y == 0;
   const int stride = gridDim.x * blockDim.x;  // n_vec < 2^31 is checked on the host
   for (int i0 = blockIdx.x * blockDim.x + threadIdx.x; i0 < n_vec; i0 += kU * stride) {
     uint4 v[kU];
@@ -130,12 +109,9 @@ __global__ void __launch_bounds__(256, 4) append_bf16_kernel(const void *__restr
       if (i < static_cast<unsigned>(n_vec)) {
         if constexpr (!kF32) {
           v[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + i);
-          if (rot) v[u] = rope_bf16x8(rk, v[u], i / vec_per_tok, static_cast<int>((static_cast<int64_t>(i) * 8) % D), D);
         } else {
-          const float4 a = __ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i));
-          const float4 b = __ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i) + 1);
-          v[u] = rot ? rope_f32x8(rk, a, b, i / vec_per_tok, static_cast<int>((static_cast<int64_t>(i) * 8) % D), D)
-                     : to_bf16x8(a, b);
+          v[u] = to_bf16x8(__ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i)),
+                           __ldcs(reinterpret_cast<const float4 *>(src) + 2 * static_cast<size_t>(i) + 1));
         }
       }
     }
@@ -285,15 +261,19 @@ __global__ void zero_u32_kernel(unsigned *a, unsigned *b, int n) {
 }
 
 // code = e4m3_rn_satfinite(x / s), s = absmax / 448 (fp32 IEEE divisions).
+// A tensor whose wide flag is set gets the codes' values widened to fp16
+// (exact: every e4m3 value is an fp16 value) instead of the codes.
 template <bool kF32>
 __global__ void __launch_bounds__(256) quant_e4m3_kernel(const void *__restrict__ x0, const void *__restrict__ x1,
                                                          const unsigned *amax0, const unsigned *amax1,
-                                                         uint8_t *__restrict__ y0, uint8_t *__restrict__ y1,
-                                                         int n_tok, int H, int D, RopeArgs rope0) {
+                                                         void *__restrict__ y0, void *__restrict__ y1,
+                                                         int n_tok, int H, int D, RopeArgs rope0, int wide0,
+                                                         int wide1) {
   const bool rot = blockIdx.z == 0 && rope0.pos != nullptr;
   const void *x = blockIdx.z == 0 ? x0 : x1;
   const unsigned *amax = blockIdx.z == 0 ? amax0 : amax1;
-  uint8_t *y = blockIdx.z == 0 ? y0 : y1;
+  void *y = blockIdx.z == 0 ? y0 : y1;
+  const bool wide = (blockIdx.z == 0 ? wide0 : wide1) != 0;
   const int h = blockIdx.y;
   const float a = __uint_as_float(amax[h]);
   const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
@@ -317,7 +297,18 @@ __global__ void __launch_bounds__(256) quant_e4m3_kernel(const void *__restrict_
                                    __NV_SATFINITE, __NV_E4M3);
       w[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
     }
-    *reinterpret_cast<uint2 *>(y + e) = make_uint2(w[0], w[1]);
+    if (!wide) {
+      *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(y) + e) = make_uint2(w[0], w[1]);
+    } else {
+      uint32_t h[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2_raw p2 = __nv_cvt_fp8x2_to_halfraw2(
+            static_cast<__nv_fp8x2_storage_t>((w[j >> 1] >> (16 * (j & 1))) & 0xffffu), __NV_E4M3);
+        h[j] = static_cast<uint32_t>(p2.x) | (static_cast<uint32_t>(p2.y) << 16);
+      }
+      *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(y) + e) = make_uint4(h[0], h[1], h[2], h[3]);
+    }
   }
 }
 
@@ -358,8 +349,8 @@ static cca_status bulk_copy_pair(const uint8_t *k_src, const uint8_t *v_src, uin
 
 // Quantise one or two [n_tok][H][D] tensors; scale arrays are [H] each.
 static cca_status quantize_pair(const void *x0, const void *x1, cca_dtype src, int n_tok, int H, int D,
-                                uint8_t *y0, uint8_t *y1, float *s0, float *s1, cudaStream_t st,
-                                RopeArgs r0 = RopeArgs{nullptr, nullptr}) {
+                                void *y0, void *y1, float *s0, float *s1, cudaStream_t st,
+                                RopeArgs r0 = RopeArgs{nullptr, nullptr}, int wide0 = 0, int wide1 = 0) {
   const int nt = x1 ? 2 : 1;
   unsigned *a0 = reinterpret_cast<unsigned *>(s0), *a1 = reinterpret_cast<unsigned *>(s1);
   zero_u32_kernel<<<1, 256, 0, st>>>(a0, x1 ? a1 : nullptr, H);
@@ -373,11 +364,11 @@ static cca_status quantize_pair(const void *x0, const void *x1, cca_dtype src, i
     if (src == CCA_F32) {
       absmax_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D, r0);
       CCA_TRY(launched("absmax_kernel"));
-      quant_e4m3_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D, r0);
+      quant_e4m3_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D, r0, wide0, wide1);
     } else {
       absmax_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D, r0);
       CCA_TRY(launched("absmax_kernel"));
-      quant_e4m3_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D, r0);
+      quant_e4m3_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D, r0, wide0, wide1);
     }
     CCA_TRY(launched("quant_e4m3_kernel"));
   }
@@ -469,18 +460,11 @@ static cca_status kv_append_impl(cca_kv_ring *ring, const void *k_new, const voi
     const int64_t cap = static_cast<int64_t>(num_sms()) * 2;  // x2 tensors: 4 blocks of 256 per SM
     if (blocks > cap) blocks = cap;
     dim3 grid(static_cast<unsigned>(blocks), 2);
-    const int vpt = d.n_heads * d.head_dim / 8;
-    if (rk.pos) {  // K rotated on the way into the ring
-      if (src_dtype == CCA_F32)
-        append_bf16_kernel<true, true><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, static_cast<int>(n_vec), rk, vpt,
-                                                             d.head_dim);
-      else
-        append_bf16_kernel<false, true><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, static_cast<int>(n_vec), rk,
-                                                              vpt, d.head_dim);
-      CCA_TRY(launched("append_bf16_kernel"));
+    if (rk.pos) {  // K rotated on the way into the ring, V copied
+      CCA_TRY(launch_rope_rows(k_new, v_new, kd, vd, true, false, src_dtype == CCA_F32, rk, d.chunk_len, d.n_heads,
+                               d.head_dim, st));
     } else if (src_dtype == CCA_F32) {
-      append_bf16_kernel<true, false><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, static_cast<int>(n_vec), rk, vpt,
-                                                            d.head_dim);
+      append_bf16_kernel<true><<<grid, 256, 0, st>>>(k_new, v_new, kd, vd, static_cast<int>(n_vec));
       CCA_TRY(launched("append_bf16_kernel"));
     } else {
       CCA_TRY(bulk_copy_pair(static_cast<const uint8_t *>(k_new), static_cast<const uint8_t *>(v_new),
@@ -489,9 +473,9 @@ static cca_status kv_append_impl(cca_kv_ring *ring, const void *k_new, const voi
     }
   } else {
     uint8_t *kd = static_cast<uint8_t *>(d.k_slots) + slot * n_elem;
-    uint8_t *vd = static_cast<uint8_t *>(d.v_slots) + slot * n_elem;
+    uint16_t *vd = static_cast<uint16_t *>(d.v_slots) + slot * n_elem;  // e4m3 values widened to fp16
     CCA_TRY(quantize_pair(k_new, v_new, src_dtype, d.chunk_len, d.n_heads, d.head_dim, kd, vd,
-                          d.k_scale + slot * d.n_heads, d.v_scale + slot * d.n_heads, st, rk));
+                          d.k_scale + slot * d.n_heads, d.v_scale + slot * d.n_heads, st, rk, 0, 1));
   }
   ring->n_appended = t + 1;
   return CCA_OK;
@@ -525,6 +509,22 @@ cca_status cca_quant_e4m3(const void *x, cca_dtype src_dtype, int32_t n_tok, int
     return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3: scale must be 4-byte aligned");
   return quantize_pair(x, nullptr, src_dtype, n_tok, n_heads, head_dim, x8, nullptr, scale, nullptr,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+cca_status cca_quant_e4m3_f16(const void *x, cca_dtype src_dtype, int32_t n_tok, int32_t n_heads, int32_t head_dim,
+                              void *x16, float *scale, cca_stream_t stream) {
+  if (!scale || (n_tok > 0 && (!x || !x16)))
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_f16: NULL argument");
+  if (n_tok < 0 || n_heads < 1 || (head_dim != 64 && head_dim != 128))
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_f16: need n_tok >= 0, H >= 1, D in {64,128}");
+  if (src_dtype != CCA_BF16 && src_dtype != CCA_F32)
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_f16: src_dtype must be CCA_BF16 or CCA_F32");
+  if (n_tok > 0 && (!aligned16(x) || !aligned16(x16)))
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_f16: x/x16 must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_f16: scale must be 4-byte aligned");
+  return quantize_pair(x, nullptr, src_dtype, n_tok, n_heads, head_dim, x16, nullptr, scale, nullptr,
+                       reinterpret_cast<cudaStream_t>(stream), RopeArgs{nullptr, nullptr}, 1, 0);
 }
 
 const char *cca_last_error(void) { return last_error().c_str(); }

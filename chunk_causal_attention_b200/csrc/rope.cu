@@ -4,8 +4,8 @@
 // (ring.cu).
 //
 // HBM-bound: per element one read (bf16 or fp32) and one bf16 write.  Both
-// tensors go through one launch (blockIdx.y picks Q or K); every thread keeps
-// kRopeUnroll 16-byte vectors of loads in flight and the grid is one wave.
+// tensors go through one launch; the angles of a token are computed once and
+// shared by all of its heads.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -14,8 +14,6 @@
 #include "rope.cuh"
 
 namespace cca {
-
-constexpr int kRopeUnroll = 4;
 
 template <bool kF32>
 __device__ __forceinline__ void load8f(const void *base, int64_t elem, float (&x)[8]) {
@@ -44,35 +42,89 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&x)[8]) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// y = rope(x) for tensor blockIdx.y (0: q, 1: k), both [n_tok][H][D].
+// Rows kernel: a block takes kRopeTok tokens at a time.  It first fills a
+// shared table of (cos, sin) for their D/2 planes -- one sincosf per plane and
+// token, shared by all heads -- then streams both tensors' 16-byte vectors of
+// those tokens: rotated (rot0 / rot1) or only copied, rounded to bf16.
+constexpr int kRopeTok = 4;
+constexpr int kRopeThreads = 256;
+
 template <bool kF32>
-__global__ void __launch_bounds__(256) rope_qk_kernel(const void *__restrict__ q, const void *__restrict__ k,
-                                                      uint4 *__restrict__ q_out, uint4 *__restrict__ k_out,
-                                                      RopeArgs r, int H, int D, int64_t n_vec) {
-  const void *x = blockIdx.y == 0 ? q : k;
-  uint4 *y = blockIdx.y == 0 ? q_out : k_out;
-  if (!x) return;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int vec_per_tok = H * D / 8;
-  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < n_vec;
-       i0 += kRopeUnroll * stride) {
-    float v[kRopeUnroll][8];
-#pragma unroll
-    for (int u = 0; u < kRopeUnroll; ++u) {
-      const int64_t i = i0 + u * stride;
-      if (i < n_vec) load8f<kF32>(x, i * 8, v[u]);
+__global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(const void *__restrict__ x0,
+                                                                 const void *__restrict__ x1, uint4 *__restrict__ y0,
+                                                                 uint4 *__restrict__ y1, int rot0, int rot1,
+                                                                 RopeArgs r, int n_tok, int H, int D) {
+  __shared__ float2 cs[kRopeTok][64];  // (cos, sin) per token and plane, D/2 <= 64
+  const int P = D / 2;
+  const int vpt = H * D / 8;  // 16-byte vectors (8 elements) per token and tensor
+  for (int t0 = blockIdx.x * kRopeTok; t0 < n_tok; t0 += gridDim.x * kRopeTok) {
+    const int nt = min(kRopeTok, n_tok - t0);
+    if (rot0 | rot1) {
+      for (int e = threadIdx.x; e < nt * P; e += kRopeThreads) {
+        const int tt = e / P, i = e - tt * P;
+        const int4 p = __ldg(reinterpret_cast<const int4 *>(r.pos) + t0 + tt);
+        const float th = fmaf(static_cast<float>(p.w), __ldg(r.freq + 3 * P + i),
+                              fmaf(static_cast<float>(p.z), __ldg(r.freq + 2 * P + i),
+                                   fmaf(static_cast<float>(p.y), __ldg(r.freq + P + i),
+                                        static_cast<float>(p.x) * __ldg(r.freq + i))));
+        float sn, c;
+        sincosf(th, &sn, &c);
+        cs[tt][i] = make_float2(c, sn);
+      }
+      __syncthreads();
     }
+    const int nv = nt * vpt;
+    for (int tensor = 0; tensor < 2; ++tensor) {
+      const void *x = tensor == 0 ? x0 : x1;
+      uint4 *y = tensor == 0 ? y0 : y1;
+      const bool rot = (tensor == 0 ? rot0 : rot1) != 0;
+      if (!x) continue;
+      const int64_t v0 = static_cast<int64_t>(t0) * vpt;
+      constexpr int kU = 6;  // vectors in flight per thread
+      for (int b = threadIdx.x; b < nv; b += kU * kRopeThreads) {
+        float v[kU][8];
 #pragma unroll
-    for (int u = 0; u < kRopeUnroll; ++u) {
-      const int64_t i = i0 + u * stride;
-      if (i < n_vec) {
-        const int64_t tok = i / vec_per_tok;
-        const int d0 = static_cast<int>((i * 8) % D);
-        rope8(r, tok, d0, D, v[u]);
-        y[i] = pack8_bf16(v[u]);
+        for (int u = 0; u < kU; ++u) {
+          const int i = b + u * kRopeThreads;
+          if (i < nv) load8f<kF32>(x, (v0 + i) * 8, v[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int i = b + u * kRopeThreads;
+          if (i >= nv) continue;
+          if (rot) {
+            const int tt = i / vpt;
+            const int pl = ((i - tt * vpt) * 4) % P;  // first plane of the vector: (8 elements / 2) per vector
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 c = cs[tt][pl + j];
+              const float a = v[u][2 * j], bb = v[u][2 * j + 1];
+              v[u][2 * j] = fmaf(a, c.x, -bb * c.y);
+              v[u][2 * j + 1] = fmaf(a, c.y, bb * c.x);
+            }
+          }
+          y[v0 + i] = pack8_bf16(v[u]);
+        }
       }
     }
+    __syncthreads();
   }
+}
+
+// Launcher shared with the clean-KV append (ring.cu).
+cca_status launch_rope_rows(const void *x0, const void *x1, void *y0, void *y1, bool rot0, bool rot1, bool f32,
+                            RopeArgs r, int n_tok, int H, int D, cudaStream_t st) {
+  int blocks = (n_tok + kRopeTok - 1) / kRopeTok;
+  const int cap = num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) return CCA_OK;
+  if (f32)
+    rope_rows_kernel<true><<<blocks, kRopeThreads, 0, st>>>(x0, x1, static_cast<uint4 *>(y0), static_cast<uint4 *>(y1),
+                                                           rot0, rot1, r, n_tok, H, D);
+  else
+    rope_rows_kernel<false><<<blocks, kRopeThreads, 0, st>>>(x0, x1, static_cast<uint4 *>(y0),
+                                                            static_cast<uint4 *>(y1), rot0, rot1, r, n_tok, H, D);
+  return launched("rope_rows_kernel");
 }
 
 }  // namespace cca
@@ -113,20 +165,8 @@ cca_status cca_rope_qk(const void *q, const void *k, cca_dtype src_dtype, int32_
   if ((q && (!aligned16(q) || !aligned16(q_out))) || (k && (!aligned16(k) || !aligned16(k_out))) ||
       !aligned16(pos) || (reinterpret_cast<uintptr_t>(freq) & 3))
     return fail(CCA_ERR_INVALID_ARG, "cca_rope_qk: tensors and pos must be 16-byte aligned, freq 4-byte aligned");
-  const int64_t n_vec = static_cast<int64_t>(n_tok) * n_heads * head_dim / 8;
-  int64_t blocks = (n_vec + 256 * kRopeUnroll - 1) / (256 * kRopeUnroll);
-  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
-  if (blocks > cap) blocks = cap;
-  const dim3 grid(static_cast<unsigned>(blocks), 2);
-  const RopeArgs r{pos, freq};
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (src_dtype == CCA_F32)
-    rope_qk_kernel<true><<<grid, 256, 0, st>>>(q, k, static_cast<uint4 *>(q_out), static_cast<uint4 *>(k_out), r,
-                                                n_heads, head_dim, n_vec);
-  else
-    rope_qk_kernel<false><<<grid, 256, 0, st>>>(q, k, static_cast<uint4 *>(q_out), static_cast<uint4 *>(k_out), r,
-                                                 n_heads, head_dim, n_vec);
-  return launched("rope_qk_kernel");
+  return launch_rope_rows(q, k, q_out, k_out, q != nullptr, k != nullptr, src_dtype == CCA_F32,
+                          RopeArgs{pos, freq}, n_tok, n_heads, head_dim, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -15,6 +15,8 @@
 
 #include <cstdint>
 
+#include "common.cuh"
+
 namespace cca {
 
 struct RopeArgs {
@@ -41,5 +43,10 @@ __device__ __forceinline__ void rope8(const RopeArgs &r, int64_t tok, int d0, in
     x[2 * j + 1] = fmaf(a, sn, b * cs);
   }
 }
+
+// Rotate (rot0 / rot1) or copy two [n_tok][H][D] tensors (bf16 or fp32 input)
+// into bf16 outputs in one launch; x1 may be NULL.  Defined in rope.cu.
+cca_status launch_rope_rows(const void *x0, const void *x1, void *y0, void *y1, bool rot0, bool rot1, bool f32,
+                            RopeArgs r, int n_tok, int H, int D, cudaStream_t st);
 
 }  // namespace cca

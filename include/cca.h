@@ -35,6 +35,13 @@
  *  - Every device buffer must be 16-byte aligned unless stated otherwise.
  *  - Tensors are dense and row-major.  [L][H][D] means token-major: element
  *    (l, h, d) is at ((l * H) + h) * D + d.
+ *  - E4M3 mode: queries and keys are e4m3 codes (one byte); values are the
+ *    e4m3-quantised values widened to fp16 (two bytes, exact: every e4m3
+ *    value is an fp16 value), each tensor with fp32 per-head scales.  The
+ *    attention keeps P in 16 bits (its e4m3 rounding alone moved outputs by
+ *    0.1 on heavy-tailed inputs), so the PV product is 16-bit and reads V
+ *    16-bit; widening V once, where it is quantised, spares every CTA a
+ *    conversion of every V tile.  QK runs on the e4m3 tensor cores.
  *  - Handles are not thread-safe; distinct handles are independent.
  *  - On any non-CCA_OK status nothing has been launched unless the status is
  *    CCA_ERR_CUDA (a launch failed part-way); cca_last_error() then describes it.
@@ -85,7 +92,7 @@ typedef struct cca_kv_ring_desc {
   int32_t window;     /* W >= 0 most recent non-sink chunks kept                 */
   cca_dtype dtype;    /* CCA_BF16 or CCA_E4M3                                    */
   void *k_slots;      /* device, [(1+W)][L][H][D] elements of dtype              */
-  void *v_slots;      /* device, same shape as k_slots                           */
+  void *v_slots;      /* device, same shape; E4M3: fp16 (widened e4m3 values)    */
   float *k_scale;     /* device, [(1+W)][H] fp32 dequantisation scales (E4M3)    */
   float *v_scale;     /* device, [(1+W)][H] (E4M3); both NULL for BF16           */
   int32_t *dev_status;/* device, one int32 (CCA_DEV_*), may be NULL              */
@@ -123,7 +130,8 @@ cca_status cca_kv_ring_restore(cca_kv_ring *ring, int64_t n_appended);
  * CCA_F32).  BF16 ring: bf16 copy (F32 input is rounded to nearest even).
  * E4M3 ring: per-head absmax quantisation, scale = absmax/448 (1 if all zero),
  * code = e4m3_rn_satfinite(x / scale) with an IEEE fp32 division; the scales
- * go to k_scale/v_scale[slot][h].  Eviction is the overwrite of the slot.
+ * go to k_scale/v_scale[slot][h]; V is stored as the codes' values widened
+ * to fp16.  Eviction is the overwrite of the slot.
  * Errors: CCA_ERR_INVALID_ARG, CCA_ERR_CUDA. */
 cca_status cca_kv_append(cca_kv_ring *ring, const void *k_new, const void *v_new,
                          cca_dtype src_dtype, cca_stream_t stream);
@@ -180,6 +188,12 @@ cca_status cca_quant_e4m3(const void *x, cca_dtype src_dtype, int32_t n_tok,
                           int32_t n_heads, int32_t head_dim, uint8_t *x8,
                           float *scale, cca_stream_t stream);
 
+/* The same quantisation, writing the codes' values widened to fp16 (device
+ * [n_tok][H][D], two bytes each) instead of the codes: the form E4M3 attention
+ * takes its V-side tensors in.  Errors: as cca_quant_e4m3. */
+cca_status cca_quant_e4m3_f16(const void *x, cca_dtype src_dtype, int32_t n_tok, int32_t n_heads,
+                              int32_t head_dim, void *x16, float *scale, cca_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Chunk attention                                                           */
 /* ------------------------------------------------------------------------ */
@@ -190,9 +204,10 @@ cca_status cca_quant_e4m3(const void *x, cca_dtype src_dtype, int32_t n_tok,
  * itself from k_cur / v_cur (never from the ring: at a denoising step they are
  * computed from the noisy input).  No element mask inside that set.
  *
- *  q, k_cur, v_cur: device [L][H][D] in the ring's dtype (BF16, or E4M3 codes
- *      with per-head scales q_scale / kcur_scale / vcur_scale, device [H]
- *      fp32; the scale pointers must be NULL for BF16).  Scales must be finite
+ *  q, k_cur, v_cur: device [L][H][D] in the ring's dtype (BF16; or E4M3: q and
+ *      k_cur e4m3 codes, v_cur fp16-widened e4m3 values as cca_quant_e4m3_f16
+ *      writes them, with per-head scales q_scale / kcur_scale / vcur_scale,
+ *      device [H] fp32; the scale pointers must be NULL for BF16).  Scales must be finite
  *      and >= 0; a zero scale means all values of that head are zero.
  *  q_idx: NULL (queries are rows 0 .. n_q-1 of q) or device int32 row indices
  *      into q (the compacted active tokens of the mask cache).
@@ -294,8 +309,10 @@ cca_status cca_attn_workspace_size(int32_t head_dim, size_t *bytes);
  * cached chunks (the sink and the window, exactly as cca_chunk_attn) and to
  * itself.  No element mask inside that set.  The history chunks of the ring
  * hold the clean tokens of earlier chunks (chunk_len rows each).
- *  q, k_cur, v_cur: device [n_cur][H][D] in the ring's dtype; 0 <= n_cur <= 2^24.
- *  k_ref, v_ref: device [n_ref][H][D] (ring dtype), NULL when n_ref = 0.
+ *  q, k_cur, v_cur: device [n_cur][H][D] in the ring's dtype (E4M3: v_cur
+ *      fp16-widened values); 0 <= n_cur <= 2^24.
+ *  k_ref, v_ref: device [n_ref][H][D] (ring dtype; E4M3: v_ref fp16-widened),
+ *      NULL when n_ref = 0.
  *  q_scale, kcur_scale, vcur_scale, kref_scale, vref_scale: E4M3 only,
  *      device [H] fp32 (NULL for BF16; the ref scales also NULL when n_ref = 0).
  *  out: device [n_cur][H][D] bf16.
@@ -320,8 +337,9 @@ cca_status cca_chunk_attn_groups(const cca_kv_ring *ring, const void *q, const v
  * tensors equal to the current ones this is plain windowed block-causal
  * attention (W >= T-1: full block-causal), which also gives the clean
  * chunks' own outputs.
- *  k_cur, v_cur, k_hist, v_hist: device [T][L][H][D] (dtype); the history
- *      tensors may alias the current ones.
+ *  k_cur, v_cur, k_hist, v_hist: device [T][L][H][D] (dtype; E4M3: the V
+ *      tensors fp16-widened values); the history tensors may alias the current
+ *      ones.
  *  k_ref, v_ref: device [ref_len][H][D] or NULL with ref_len = 0.
  *  Scales (E4M3 only, else NULL): kcur/vcur/khist/vhist [T][H], kref/vref [H].
  *  dev_status: device int32 (CCA_DEV_*), may be NULL. */

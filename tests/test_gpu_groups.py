@@ -99,9 +99,9 @@ def test_groups_step_e4m3():
     names, (q, k, v) = _packed(s.groups)
     q8, qs = cca.cca_quant_e4m3(bf(q))
     k8, ks = cca.cca_quant_e4m3(bf(k))
-    v8, vs = cca.cca_quant_e4m3(bf(v))
+    v8, vs = cca.cca_quant_e4m3_f16(bf(v))
     kr8, krs = cca.cca_quant_e4m3(bf(s.ref[1]))
-    vr8, vrs = cca.cca_quant_e4m3(bf(s.ref[2]))
+    vr8, vrs = cca.cca_quant_e4m3_f16(bf(s.ref[2]))
     o = cca.cca_chunk_attn_groups(ring, q8, k8, v8, k_ref=kr8, v_ref=vr8, q_scale=qs, kcur_scale=ks, vcur_scale=vs,
                                   kref_scale=krs, vref_scale=vrs)
     deq = lambda x: ofp8.dequantize_per_head(*ofp8.quantize_per_head(x))
@@ -168,9 +168,9 @@ def test_block_attn_e4m3():
     p = synth.packed_sequence(seed=64, n_chunks=T, n_heads=H, head_dim=D, chunk_len=L, window=W, heavy_tailed=True)
     qz = [cca.cca_quant_e4m3(bf(p.q[c])) for c in range(T)]
     kz = [cca.cca_quant_e4m3(bf(p.k_cur[c])) for c in range(T)]
-    vz = [cca.cca_quant_e4m3(bf(p.v_cur[c])) for c in range(T)]
+    vz = [cca.cca_quant_e4m3_f16(bf(p.v_cur[c])) for c in range(T)]
     khz = [cca.cca_quant_e4m3(bf(p.k_hist[c])) for c in range(T)]
-    vhz = [cca.cca_quant_e4m3(bf(p.v_hist[c])) for c in range(T)]
+    vhz = [cca.cca_quant_e4m3_f16(bf(p.v_hist[c])) for c in range(T)]
     st = lambda z, i: torch.stack([x[i] for x in z]).contiguous()
     o = cca.cca_block_attn(st(qz, 0), st(kz, 0), st(vz, 0), W, k_hist=st(khz, 0), v_hist=st(vhz, 0),
                            q_scale=st(qz, 1), kcur_scale=st(kz, 1), vcur_scale=st(vz, 1), khist_scale=st(khz, 1),

@@ -144,6 +144,17 @@ def test_quant_e4m3_bit_exact(src_dtype):
     assert np.array_equal(codes.cpu().numpy(), ref_codes)
 
 
+def test_quant_e4m3_f16_widens_the_codes_exactly():
+    g = np.random.default_rng(7)
+    x = synth.bf16_round(g.standard_t(4.0, size=(777, 5, 128)).astype(np.float32))
+    x[:, 2] = 0.0
+    x16, scale = cca.cca_quant_e4m3_f16(synth.as_torch_bf16(x, dev()))
+    ref_codes, ref_scale = ofp8.quantize_per_head(x)
+    torch.cuda.synchronize()
+    assert np.array_equal(scale.cpu().numpy(), ref_scale)
+    assert np.array_equal(x16.cpu().numpy(), ofp8.e4m3_decode(ref_codes).astype(np.float16))
+
+
 def test_ring_append_e4m3_bit_exact():
     s = synth.fp8_720p(n_steps=1, n_prefill=5)
     ring = cca.KVRing(s.n_heads, s.head_dim, s.chunk_len, s.window, dtype="e4m3", device=dev())
@@ -156,7 +167,8 @@ def test_ring_append_e4m3_bit_exact():
         kc, ks = ofp8.quantize_per_head(s.ring_k[c])
         vc, vs = ofp8.quantize_per_head(s.ring_v[c])
         assert np.array_equal(ring.k_slots[sl].cpu().numpy(), kc)
-        assert np.array_equal(ring.v_slots[sl].cpu().numpy(), vc)
+        # V is stored as the codes' values widened to fp16 (exact)
+        assert np.array_equal(ring.v_slots[sl].cpu().numpy(), ofp8.e4m3_decode(vc).astype(np.float16))
         assert np.array_equal(ring.k_scale[sl].cpu().numpy(), ks)
         assert np.array_equal(ring.v_scale[sl].cpu().numpy(), vs)
 
@@ -463,7 +475,7 @@ def test_fused_scatter_fp8_and_empty():
     idx, n = cca.cca_compact(mask)
     q8, qs = cca.cca_quant_e4m3(bf(s.q[0]))
     k8, ks = cca.cca_quant_e4m3(bf(s.k_cur[0]))
-    v8, vs = cca.cca_quant_e4m3(bf(s.v_cur[0]))
+    v8, vs = cca.cca_quant_e4m3_f16(bf(s.v_cur[0]))
     o_c = cca.cca_chunk_attn(ring, q8, k8, v8, q_scale=qs, kcur_scale=ks, vcur_scale=vs, q_idx=idx, n_q_dev=n,
                              n_q_max=s.chunk_len)
     two_pass = torch.zeros((s.chunk_len, s.n_heads, s.head_dim), dtype=torch.bfloat16, device=dev())
@@ -539,7 +551,7 @@ def _fp8_stream_ref(ring_k, ring_v, q, kc, vc, t, window):
 def _fp8_call(ring, q, kc, vc, **kw):
     q8, qs = cca.cca_quant_e4m3(bf(q))
     k8, ks = cca.cca_quant_e4m3(bf(kc))
-    v8, vs = cca.cca_quant_e4m3(bf(vc))
+    v8, vs = cca.cca_quant_e4m3_f16(bf(vc))
     return cca.cca_chunk_attn(ring, q8, k8, v8, q_scale=qs, kcur_scale=ks, vcur_scale=vs, **kw)
 
 
@@ -602,7 +614,7 @@ def test_attention_fp8_zero_and_tiny_v_scales():
     ring.v_scale[slots[1]] *= 2.0 ** -30
     q8, qs = cca.cca_quant_e4m3(bf(q))
     k8, ks = cca.cca_quant_e4m3(bf(k[3]))
-    v8, vs = cca.cca_quant_e4m3(bf(v[3]))
+    v8, vs = cca.cca_quant_e4m3_f16(bf(v[3]))
     o = cca.cca_chunk_attn(ring, q8, k8, v8, q_scale=qs, kcur_scale=ks, vcur_scale=torch.zeros_like(vs))
 
     def deq(x, f=1.0):
