@@ -40,8 +40,6 @@
 #include <cstdlib>
 #include <cstring>
 #include <algorithm>
-#include <atomic>
-#include <chrono>
 #include <initializer_list>
 #include <mutex>
 #include <vector>
@@ -130,9 +128,6 @@ struct AttnArgs {
   int scatter_out;         // 1: query i's row goes to out row q_idx[i] (fused scatter-back)
   float *ws_o;             // [2 x grid][256][D] partial O of split items (unnormalised)
   float *ws_ml;            // [2 x grid][256][2] (running max in log2 units, row sum)
-  unsigned long long *ws_flag;  // [grid] piece-done flags of the in-kernel merge
-  unsigned long long token;     // value this launch writes into the flags (unique per launch)
-  int merge_in_kernel;     // 1: launched cooperatively; aligned pieces are merged by their CTAs
   int32_t *dev_status;
   // e4m3 only: per-head dequantisation scales, [slots][H] per tensor.
   const float *q_scale;
@@ -944,88 +939,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  // Aligned pieces of a leftover item are merged by the CTAs that computed them
-  // (all resident: cooperative launch): each publishes its piece with the
-  // launch's token, waits (bounded) for the other pieces of its item, then the
-  // softmax warps merge its share of the item's 256 rows.
-  if (a.merge_in_kernel && sch.s > 0 && sch.tr > 0 && !*abort_flag) {
-    const int G = gridDim.x, c = blockIdx.x;
-    const int u = sch.rem0 + c / sch.s;
-    if (u < sch.n_items) {
-      const int c_first = c - c % sch.s, j_me = c % sch.s;
-      int p, pair, head;
-      item_coords(a, n_q0, u, p, pair, head);
-      const int n_kv = a.prob[p].n_kv;
-      if (threadIdx.x == 0) {
-        __threadfence();
-        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(a.ws_flag + c), "l"(a.token) : "memory");
-      }
-      __shared__ int s_ok;
-      if (threadIdx.x == 32) {  // warp 1, lane 0: wait for every non-empty piece of the item
-        int ok = 1;
-        const long long t0 = clock64();
-        for (int j = 0; j < sch.s && ok; ++j) {
-          if (j * n_kv / sch.s >= (j + 1) * n_kv / sch.s) continue;  // empty piece: nothing published
-          while (true) {
-            unsigned long long f;
-            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(f) : "l"(a.ws_flag + c_first + j) : "memory");
-            if (f == a.token) break;
-            if (clock64() - t0 > budget) {
-              ok = 0;
-              break;
-            }
-          }
-        }
-        s_ok = ok;
-        if (!ok && a.dev_status) atomicExch(a.dev_status, CCA_DEV_TIMEOUT);
-      }
-      __syncthreads();
-      (void)G;
-      if (s_ok && warp >= 4) {
-        constexpr int kV = D / 32;
-        const int n_q = prob_nq(a, p, n_q0);
-        const int r0 = j_me * (kNQ * kBM) / sch.s, r1 = (j_me + 1) * (kNQ * kBM) / sch.s;
-        for (int rr = r0 + (warp - 4); rr < r1; rr += 8) {
-          const int row = pair * (kNQ * kBM) + rr;
-          if (row >= n_q) break;
-          float mmax = -INFINITY;
-          for (int j = 0; j < sch.s; ++j) {
-            if (j * n_kv / sch.s >= (j + 1) * n_kv / sch.s) continue;
-            mmax = fmaxf(mmax, __ldcg(a.ws_ml + (static_cast<int64_t>(2 * (c_first + j)) * (kNQ * kBM) + rr) * 2));
-          }
-          float den = 0.f, acc[kV];
-#pragma unroll
-          for (int k = 0; k < kV; ++k) acc[k] = 0.f;
-          for (int j = 0; j < sch.s; ++j) {
-            if (j * n_kv / sch.s >= (j + 1) * n_kv / sch.s) continue;
-            const int64_t prow = static_cast<int64_t>(2 * (c_first + j)) * (kNQ * kBM) + rr;
-            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(a.ws_ml + prow * 2));
-            const float w = exp2f(ml.x - mmax);
-            den += w * ml.y;
-            const float *o = a.ws_o + prow * D + lane * kV;
-            if constexpr (kV == 4) {
-              const float4 v = __ldcg(reinterpret_cast<const float4 *>(o));
-              acc[0] += w * v.x, acc[1] += w * v.y, acc[2] += w * v.z, acc[3] += w * v.w;
-            } else {
-              const float2 v = __ldcg(reinterpret_cast<const float2 *>(o));
-              acc[0] += w * v.x, acc[1] += w * v.y;
-            }
-          }
-          const float inv = 1.f / den;
-          const int orow = a.scatter_out ? __ldg(a.q_idx + row) : row;
-          if (orow < 0 || orow >= a.out_rows) continue;
-          __nv_bfloat16 *dst =
-              a.out + ((static_cast<int64_t>(a.prob[p].out_slot) * a.out_rows + orow) * a.H + head) * D + lane * kV;
-          if constexpr (kV == 4) {
-            *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
-                                                         pack_bf16x2(acc[2] * inv, acc[3] * inv));
-          } else {
-            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-          }
-        }
-      }
-    }
-  }
   if (threadIdx.x == 0 && *abort_flag && a.dev_status) atomicExch(a.dev_status, CCA_DEV_TIMEOUT);
 }
 
@@ -1060,7 +973,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n_q0 = a.n_q_dev ? min(max(*a.n_q_dev, 0), a.prob[0].n_q) : a.prob[0].n_q;
   const Sched sch = make_sched(a, n_q0, G);
-  if (sch.tr == 0 || (sch.s > 0 && a.merge_in_kernel)) return;  // nothing split, or merged in the attention kernel
+  if (sch.tr == 0) return;  // nothing split
   const int lane = threadIdx.x & 31;
   const int64_t tr = sch.tr;
   // Range bounds floor(c * tr / G) and ceil(x * G / tr) in 32-bit arithmetic when
@@ -1260,11 +1173,10 @@ static int attn_grid(int64_t work) {
   return g;
 }
 
-// Partial-piece slots: 2 per CTA, 256 rows each, O (D fp32) plus (m, l); then
-// one 8-byte merge flag per CTA.
+// Partial-piece slots: 2 per CTA, 256 rows each, O (D fp32) plus (m, l).
 static size_t workspace_bytes_for_grid(int grid, int D) {
   const size_t rows = static_cast<size_t>(2) * grid * (kNQ * kBM);
-  return rows * (static_cast<size_t>(D) + 2) * sizeof(float) + static_cast<size_t>(grid) * 8 + 256;
+  return rows * (static_cast<size_t>(D) + 2) * sizeof(float) + 256;
 }
 
 // Workspace that suffices for every attention launch with this head_dim on
@@ -1304,14 +1216,6 @@ static int host_split_mode(const AttnArgs &a, int G) {
   return pieces >= 2 && (nkv_first + pieces - 1) / pieces <= even + 2 ? 2 : 1;
 }
 
-// Unique value per launch for the merge flags (a per-process counter above a
-// seed from the clock, so stale flags of earlier launches never match).
-static unsigned long long next_token() {
-  static std::atomic<unsigned long long> ctr{
-      (static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count()) << 20) | 1ull};
-  return ctr.fetch_add(1ull);
-}
-
 static std::mutex g_attr_mu;
 
 template <int D, bool kFp8>
@@ -1329,9 +1233,6 @@ static cca_status launch_attn(AttnLaunch &L, void *workspace, size_t workspace_b
     return fail(CCA_ERR_INVALID_ARG, "attention: workspace of %zu bytes (16-byte aligned) required", need);
   args.ws_o = static_cast<float *>(workspace);
   args.ws_ml = args.ws_o + static_cast<size_t>(2) * grid * (kNQ * kBM) * D;
-  args.ws_flag = reinterpret_cast<unsigned long long *>(
-      (reinterpret_cast<uintptr_t>(args.ws_ml + static_cast<size_t>(2) * grid * (kNQ * kBM) * 2) + 15) & ~uintptr_t(15));
-  args.token = next_token();
   CUtensorMap tq, tk[kMaxSrc], tv[kMaxSrc];
   std::memset(&tq, 0, sizeof(tq));
   if (!args.q_idx) CCA_TRY(make_tmap(&tq, L.q, dt, es, D, H, L.q_rows_map, L.q_slots));
@@ -1343,60 +1244,24 @@ static cca_status launch_attn(AttnLaunch &L, void *workspace, size_t workspace_b
     CCA_TRY(make_tmap(&tk[s], kp, dt, es, D, H, rows, slots));
     CCA_TRY(make_tmap(&tv[s], vp, dt_v, 2, D, H, rows, slots));
   }
-  int resident = 0;  // co-resident CTAs on this device (1 per SM at this shared-memory size)
   {
     // The shared-memory opt-in is per device and kernel: set it once per device.
     static bool done[64] = {false};
-    static int max_blocks[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lk(g_attr_mu);
     if (dev < 0 || dev >= 64 || !done[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(S::kAlloc));
+      const cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(S::kAlloc));
       if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "attention: %s", cudaGetErrorString(e));
-      int per_sm = 0;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_kernel<D, kFp8>, kThreads, S::kAlloc);
-      if (e != cudaSuccess) per_sm = 0;
-      if (dev >= 0 && dev < 64) {
-        done[dev] = true;
-        max_blocks[dev] = per_sm * num_sms();
-      } else {
-        resident = per_sm * num_sms();
-      }
+      if (dev >= 0 && dev < 64) done[dev] = true;
     }
-    if (dev >= 0 && dev < 64) resident = max_blocks[dev];
   }
-  // Aligned pieces are merged inside the attention kernel when every CTA is
-  // resident at once (a cooperative launch guarantees it); otherwise by the
-  // combine kernel.
+  attn_kernel<D, kFp8><<<grid, kThreads, S::kAlloc, st>>>(tq, tk[0], tv[0], tk[1], tv[1], tk[2], tv[2], args);
+  CCA_TRY(launched("attn_kernel"));
+  // The combine kernel runs unless the host knows the schedule splits no item.
   const int mode = host_split_mode(args, grid);
-  const bool maybe_aligned = args.n_q_dev != nullptr || mode == 2;
-  args.merge_in_kernel = maybe_aligned && grid <= resident && env_int("CCA_MERGE_IN_KERNEL", 1) != 0;
-  {
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = S::kAlloc;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = args.merge_in_kernel ? 1 : 0;
-    const cudaError_t le =
-        cudaLaunchKernelEx(&cfg, attn_kernel<D, kFp8>, tq, tk[0], tv[0], tk[1], tv[1], tk[2], tv[2], args);
-    if (le != cudaSuccess) {
-      cudaGetLastError();
-      return fail(CCA_ERR_CUDA, "attention: launch failed: %s", cudaGetErrorString(le));
-    }
-    CCA_TRY(launched("attn_kernel"));
-  }
-  // The combine kernel runs unless the host knows the schedule splits nothing,
-  // or splits in aligned pieces that the attention kernel merges itself.
-  const bool need_combine = args.n_q_dev != nullptr || mode == 1 || (mode == 2 && !args.merge_in_kernel);
-  if (need_combine) {
+  if (args.n_q_dev != nullptr || mode != 0) {
     const int64_t warps = static_cast<int64_t>(grid) * (kNQ * kBM);
     int64_t blocks = (warps + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
