@@ -883,6 +883,32 @@ def profile_case(name: str) -> None:
         q, kc, vc = bf(c1.q[0]), bf(c1.k_cur[0]), bf(c1.v_cur[0])
         wsm = torch.empty(max(cca.cca_chunk_attn_workspace_size(ring, L), 16), dtype=torch.uint8, device=dev)
         fn = lambda: cca.cca_chunk_attn(ring, q, kc, vc, q_idx=idx, n_q_dev=n_act, n_q_max=L, workspace=wsm)
+    elif name == "bf16_720p":
+        ring = cca.KVRing(H, D, L, W, device=dev)
+        for _ in range(4):
+            ring.append(torch.randn((L, H, D), device=dev).to(torch.bfloat16),
+                        torch.randn((L, H, D), device=dev).to(torch.bfloat16))
+        q, kc, vc = (torch.randn((L, H, D), device=dev).to(torch.bfloat16) for _ in range(3))
+        ws = torch.empty(cca.cca_chunk_attn_workspace_size(ring, L), dtype=torch.uint8, device=dev)
+        fn = lambda: cca.cca_chunk_attn(ring, q, kc, vc, workspace=ws)
+    elif name == "mask_select_32K":
+        n = 32768
+        src = torch.randn((n, 16), device=dev)
+        edit = src + 0.5 * torch.randn((n, 16), device=dev)
+        mask = torch.empty(n, dtype=torch.uint8, device=dev)
+        fn = lambda: cca.cca_token_mask_l2(src, edit, prune_quantile=0.7, mask=mask)
+    elif name == "rope_qk_720p":
+        import synth
+        pos = torch.from_numpy(synth.grid_positions(4)).to(dev)
+        freq = cca.cca_mrope_freqs(D, device=dev)
+        q, k = (torch.randn((L, H, D), device=dev).to(torch.bfloat16) for _ in range(2))
+        qo, ko = torch.empty_like(q), torch.empty_like(k)
+        fn = lambda: cca.cca_rope_qk(q, k, pos, freq, q_out=qo, k_out=ko)
+    elif name == "append_e4m3_720p":
+        ring = cca.KVRing(H, D, L, W, dtype="e4m3", device=dev)
+        k = torch.randn((L, H, D), device=dev).to(torch.bfloat16)
+        v = torch.randn((L, H, D), device=dev).to(torch.bfloat16)
+        fn = lambda: ring.append(k, v)
     else:
         raise SystemExit(f"unknown profile case {name}")
     for _ in range(3):

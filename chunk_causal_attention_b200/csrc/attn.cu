@@ -238,7 +238,10 @@ __device__ __forceinline__ Sched make_sched(const AttnArgs &a, int n_q0, int G) 
   return s;
 }
 
-// Item u -> (problem, pair, head).
+// Item u -> (problem, pair, head).  When a problem's last pair has at most 128
+// queries (its second Q tile is empty, e.g. 84 of 256 rows at 1620 queries),
+// those single-tile items are listed after the problem's full pairs, so the
+// schedule puts the cheap items into its last round or its split remainder.
 __device__ __forceinline__ void item_coords(const AttnArgs &a, int n_q0, int u, int &p, int &pair, int &head) {
   for (p = 0; p + 1 < a.n_prob; ++p) {
     const int cnt = prob_pairs(a, p, n_q0) * a.H;
@@ -246,8 +249,26 @@ __device__ __forceinline__ void item_coords(const AttnArgs &a, int n_q0, int u, 
     u -= cnt;
   }
   const int np = max(prob_pairs(a, p, n_q0), 1);
+  const int last_rows = prob_nq(a, p, n_q0) - (np - 1) * (kNQ * kBM);
+  if (np > 1 && last_rows <= kBM) {
+    const int full = (np - 1) * a.H;
+    if (u < full) {
+      pair = u % (np - 1);
+      head = u / (np - 1);
+    } else {
+      pair = np - 1;
+      head = u - full;
+    }
+    return;
+  }
   pair = u % np;
   head = u / np;
+}
+
+// Whether the item's second Q tile holds any query (else its MMAs and its
+// softmax warpgroup skip the item).
+__device__ __forceinline__ bool second_tile(const AttnArgs &a, int n_q0, const Seg &g) {
+  return g.pair * (kNQ * kBM) + kBM < prob_nq(a, g.prob, n_q0);
 }
 
 // Remainder item holding tile offset t of the remainder list: its index, first
@@ -597,14 +618,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       issue_pv(i, stage, acc, kBN / 32, kBN / 16);
       return true;
     };
-    uint32_t g = 0;
-    int it = 0;
+    uint32_t g = 0, g1 = 0;  // tiles handled; tiles that had a second Q tile
+    int it = 0, it1 = 0;     // items handled; items that had a second Q tile
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
       if (!get_seg(a, n_q0, sch, gridDim.x, blockIdx.x, kseg, sg)) break;
       const int j0 = sg.j0, j1 = sg.j1;
       const int n = j1 - j0;
+      const bool two = second_tile(a, n_q0, sg);  // else QK1 / PV1 are skipped (softmax 1 sits the item out)
       ok = wait(&q_full[0], it & 1) && wait(&q_full[1], it & 1);
       // K of the segment's first tile; later K tiles are waited for one tile
       // ahead (after QK1), while the softmax still runs, so that PV0(g) and
@@ -620,15 +642,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_qk(0, stage);
         commit(&s_full[0]);
         if (lane == 0) CCA_TRACE_EV(2, g);
-        if (jj > 0) {  // O1 += P1 V for the previous tile
+        if (two && jj > 0) {  // O1 += P1 V for the previous tile
           const uint32_t pst = (g - 1) % kNSV;
-          if (jj == 1 && it > 0 && !(ok = wait(&o_empty[1], (it - 1) & 1))) break;
-          if (!(ok = pv_in_halves(1, pst, jj > 1, (g - 1) & 1))) break;
+          if (jj == 1 && it1 > 0 && !(ok = wait(&o_empty[1], (it1 - 1) & 1))) break;
+          if (!(ok = pv_in_halves(1, pst, jj > 1, (g1 - 1) & 1))) break;
           if (lane == 0) CCA_TRACE_EV(3, g - 1);
           commit(&pv_empty[pst]);
         }
-        issue_qk(1, stage);
-        commit(&s_full[1]);
+        if (two) {
+          issue_qk(1, stage);
+          commit(&s_full[1]);
+        }
         commit(&k_empty[stage]);
         if (lane == 0) CCA_TRACE_EV(4, g);
         if (jj == n - 1) {
@@ -642,17 +666,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) CCA_TRACE_EV(8, g);
         if (jj == 0 && it > 0 && !(ok = wait(&o_empty[0], (it - 1) & 1))) break;
         if (!(ok = pv_in_halves(0, vst, jj > 0, g & 1))) break;
+        if (!two) commit(&pv_empty[vst]);  // no PV1 will read this V stage
         if (lane == 0) CCA_TRACE_EV(5, g);
         if (lane == 0) CCA_TRACE_EV(6, g);
         if (jj == n - 1) commit(&o_full[0]);
+        if (two) ++g1;
       }
       if (!ok) break;
-      {  // O1 += P1 V for the last tile
+      if (two) {  // O1 += P1 V for the last tile
         const uint32_t pst = (g - 1) % kNSV;
-        if (n == 1 && it > 0 && !(ok = wait(&o_empty[1], (it - 1) & 1))) break;
-        if (!(ok = pv_in_halves(1, pst, n > 1, (g - 1) & 1))) break;
+        if (n == 1 && it1 > 0 && !(ok = wait(&o_empty[1], (it1 - 1) & 1))) break;
+        if (!(ok = pv_in_halves(1, pst, n > 1, (g1 - 1) & 1))) break;
         commit(&pv_empty[pst]);
         commit(&o_full[1]);
+        ++it1;
       }
       ++it;
     }
@@ -714,6 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
       if (!get_seg(a, n_q0, sch, gridDim.x, blockIdx.x, kseg, sg)) break;
+      if (wg == 1 && !second_tile(a, n_q0, sg)) continue;  // the item's second Q tile is empty
       const int pair = sg.pair, head = sg.head, j0 = sg.j0, j1 = sg.j1;
       const AttnProb &P = a.prob[sg.prob];
       const int n_q = prob_nq(a, sg.prob, n_q0);
