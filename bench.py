@@ -371,7 +371,21 @@ def extra_workloads(dev, stream, peak_tf, peak_gbs):
             xv = 0.9 * xv + 0.44 * torch.randn((L, H, D), generator=gen, device=dev)
         torch.cuda.synchronize()
         return np.array([a.elapsed_time(b) for a, b in lat])
-    passes = np.stack([stream_pass(2 + k) for k in range(3)])
+    # A first pass from an idle GPU drifted +6-8 % while the clock settled under the power cap
+    # (later passes: within 1 %); it is run as warm-up and not counted.  Each counted pass records
+    # the SM clock (NVML) while it runs.
+    stream_pass(1)
+    pass_clocks = []
+    runs = []
+    for k in range(3):
+        try:
+            smp = NvmlClockSampler(dev.index if dev.index is not None else 0, period_s=0.005)
+            smp.start()
+        except Exception:
+            smp = None
+        runs.append(stream_pass(2 + k))
+        pass_clocks.append(smp.stop() if smp else None)
+    passes = np.stack(runs)
     ms = np.median(passes, axis=0)
     early, late = float(np.median(ms[5:30])), float(np.median(ms[200:225]))
     slope = float(np.polyfit(np.arange(5, 225), ms[5:225], 1)[0])
@@ -379,7 +393,8 @@ def extra_workloads(dev, stream, peak_tf, peak_gbs):
     out["long_stream_225"] = {"ms_per_chunk_median_5_29": early, "ms_per_chunk_median_200_224": late,
                               "drift_pct": (late - early) / early * 100.0, "drift_pct_each_pass": drift_each,
                               "ols_slope_ms_per_chunk": slope, "first_chunks_ms": [float(x) for x in ms[:5]],
-                              "passes": 3}
+                              "passes": 3, "warmup_passes": 1,
+                              "sm_mhz_each_pass": [c.get("sm_mhz") if c else None for c in pass_clocks]}
 
     # ---- memory-bound kernels (bandwidth, L2 flushed before each rep)
     def bw(fn, nbytes, reps=20):

@@ -198,128 +198,133 @@ __global__ void __launch_bounds__(32, 1) append_bulk_kernel(const uint8_t *__res
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
-// Loads 8 consecutive elements (16 B of bf16, 32 B of fp32) as floats.
-template <bool kF32>
-__device__ __forceinline__ void load8(const void *base, int64_t elem, float (&x)[8]) {
-  if constexpr (kF32) {
-    const float4 a = *reinterpret_cast<const float4 *>(static_cast<const float *>(base) + elem);
-    const float4 b = *reinterpret_cast<const float4 *>(static_cast<const float *>(base) + elem + 4);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-  } else {
-    const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(base) + elem);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      x[2 * j] = __uint_as_float(w[j] << 16);
-      x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-    }
-  }
-}
+// Single-launch per-head quantisation: a cluster of kQC CTAs per (tensor,
+// head), each over a quarter of the tokens.  Pass 1: the CTA's absmax (warp
+// shuffles, then shared memory); the cluster's maximum is read from the other
+// CTAs' shared memory after a hardware cluster barrier.  Pass 2: the CTA
+// quantises its rows (read again, from L2), with s = absmax / 448 (1 for an
+// all-zero head), exactly the rule of the multi-kernel path.  Rank 0 writes the
+// scale.  A second cluster barrier keeps every CTA's shared memory alive until
+// the others have read it.
+constexpr int kQC = 4;          // CTAs per (tensor, head)
+constexpr int kQThreads = 512;
 
-// Per-head absmax of up to two tensors x[n_tok][H][D].  grid = (blocks, H,
-// n_tensors); each block strides over tokens of its head and folds its maximum
-// into amax_bits[tensor][h] with atomicMax on the float's bit pattern (valid
-// ordering for non-negative floats).
 template <bool kF32>
-__global__ void __launch_bounds__(256) absmax_kernel(const void *__restrict__ x0, const void *__restrict__ x1,
-                                                     unsigned *amax0, unsigned *amax1, int n_tok, int H,
-                                                     int D, RopeArgs rope0) {
-  const bool rot = blockIdx.z == 0 && rope0.pos != nullptr;  // x0 rotated before it is measured
-  const void *x = blockIdx.z == 0 ? x0 : x1;
-  unsigned *amax = blockIdx.z == 0 ? amax0 : amax1;
-  const int h = blockIdx.y;
-  const int vec_per_row = D / 8;
-  const int rows_per_iter = blockDim.x / vec_per_row;
-  const int r0 = threadIdx.x / vec_per_row, c = threadIdx.x % vec_per_row;
+__global__ void __cluster_dims__(kQC, 1, 1) __launch_bounds__(kQThreads)
+    quant_cluster_kernel(const void *__restrict__ x0, const void *__restrict__ x1, void *__restrict__ y0,
+                         void *__restrict__ y1, float *__restrict__ s0, float *__restrict__ s1, int n_tok, int H,
+                         int D, RopeArgs rope0, int wide0, int wide1) {
+  const int tensor = blockIdx.z, h = blockIdx.y, rank = blockIdx.x;  // cluster = the kQC CTAs of (tensor, h)
+  const void *x = tensor == 0 ? x0 : x1;
+  void *y = tensor == 0 ? y0 : y1;
+  float *scale = tensor == 0 ? s0 : s1;
+  const bool wide = (tensor == 0 ? wide0 : wide1) != 0;
+  const bool rot = tensor == 0 && rope0.pos != nullptr;
+  const int vpr = D / 8;  // 16-byte (8-element) vectors per row of one head
+  const int t0 = static_cast<int>(static_cast<int64_t>(n_tok) * rank / kQC);
+  const int t1 = static_cast<int>(static_cast<int64_t>(n_tok) * (rank + 1) / kQC);
+  const int n_vec = (t1 - t0) * vpr;
+  __shared__ float red[kQThreads / 32];
+  __shared__ float cta_max;
+  // kQU raw 16-byte loads in flight per thread before any is used
+  constexpr int kQU = 4;
+  constexpr int kW = kF32 ? 2 : 1;  // 16-byte words per 8 elements
+  auto fetch = [&](int i, uint4 (&w)[kW]) {
+    const int l = t0 + i / vpr, c = i % vpr;
+    const int64_t e = (static_cast<int64_t>(l) * H + h) * D + c * 8;
+    if constexpr (kF32) {
+      w[0] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + e));
+      w[1] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + e) + 1);
+    } else {
+      w[0] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + e));
+    }
+  };
+  auto unpack = [&](int i, const uint4 (&w)[kW], float (&v)[8]) {
+    if constexpr (kF32) {
+      const uint32_t u[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(u[j]);
+    } else {
+      const uint32_t u[4] = {w[0].x, w[0].y, w[0].z, w[0].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[2 * j] = __uint_as_float(u[j] << 16);
+        v[2 * j + 1] = __uint_as_float(u[j] & 0xffff0000u);
+      }
+    }
+    if (rot) rope8(rope0, t0 + i / vpr, (i % vpr) * 8, D, v);
+  };
   float m = 0.f;
-  if (r0 < rows_per_iter) {
-    for (int l = blockIdx.x * rows_per_iter + r0; l < n_tok; l += gridDim.x * rows_per_iter) {
+  for (int b = threadIdx.x; b < n_vec; b += kQU * kQThreads) {
+    uint4 w[kQU][kW];
+#pragma unroll
+    for (int u = 0; u < kQU; ++u)
+      if (b + u * kQThreads < n_vec) fetch(b + u * kQThreads, w[u]);
+#pragma unroll
+    for (int u = 0; u < kQU; ++u) {
+      if (b + u * kQThreads >= n_vec) continue;
       float v[8];
-      load8<kF32>(x, (static_cast<int64_t>(l) * H + h) * D + c * 8, v);
-      if (rot) rope8(rope0, l, c * 8, D, v);
+      unpack(b + u * kQThreads, w[u], v);
 #pragma unroll
       for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  __shared__ float red[8];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int w = 1; w < static_cast<int>(blockDim.x / 32); ++w) m = fmaxf(m, red[w]);
-    atomicMax(amax + h, __float_as_uint(m));
+    for (int w = 1; w < kQThreads / 32; ++w) m = fmaxf(m, red[w]);
+    cta_max = m;
   }
-}
-
-__global__ void zero_u32_kernel(unsigned *a, unsigned *b, int n) {
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    a[i] = 0u;
-    if (b) b[i] = 0u;
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  float a = 0.f;
+  for (int r = 0; r < kQC; ++r) {  // the cluster's CTAs' maxima, read through distributed shared memory
+    uint32_t local = smem_u32(&cta_max), remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(r));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    a = fmaxf(a, v);
   }
-}
-
-// code = e4m3_rn_satfinite(x / s), s = absmax / 448 (fp32 IEEE divisions).
-// A tensor whose wide flag is set gets the codes' values widened to fp16
-// (exact: every e4m3 value is an fp16 value) instead of the codes.
-template <bool kF32>
-__global__ void __launch_bounds__(256) quant_e4m3_kernel(const void *__restrict__ x0, const void *__restrict__ x1,
-                                                         const unsigned *amax0, const unsigned *amax1,
-                                                         void *__restrict__ y0, void *__restrict__ y1,
-                                                         int n_tok, int H, int D, RopeArgs rope0, int wide0,
-                                                         int wide1) {
-  const bool rot = blockIdx.z == 0 && rope0.pos != nullptr;
-  const void *x = blockIdx.z == 0 ? x0 : x1;
-  const unsigned *amax = blockIdx.z == 0 ? amax0 : amax1;
-  void *y = blockIdx.z == 0 ? y0 : y1;
-  const bool wide = (blockIdx.z == 0 ? wide0 : wide1) != 0;
-  const int h = blockIdx.y;
-  const float a = __uint_as_float(amax[h]);
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
-  const int vec_per_row = D / 8;
-  const int rows_per_iter = blockDim.x / vec_per_row;
-  const int r0 = threadIdx.x / vec_per_row, c = threadIdx.x % vec_per_row;
-  if (r0 >= rows_per_iter) return;
-  for (int l = blockIdx.x * rows_per_iter + r0; l < n_tok; l += gridDim.x * rows_per_iter) {
-    const int64_t e = (static_cast<int64_t>(l) * H + h) * D + c * 8;
-    float v[8];
-    load8<kF32>(x, e, v);
-    if (rot) rope8(rope0, l, c * 8, D, v);  // same rotation as the absmax pass
-    uint32_t w[2];
+  if (rank == 0 && threadIdx.x == 0) scale[h] = s;
+  for (int b = threadIdx.x; b < n_vec; b += kQU * kQThreads) {
+    uint4 wr[kQU][kW];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const __nv_fp8x2_storage_t lo =
-          __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[4 * j], s), __fdiv_rn(v[4 * j + 1], s)),
-                                   __NV_SATFINITE, __NV_E4M3);
-      const __nv_fp8x2_storage_t hi =
-          __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[4 * j + 2], s), __fdiv_rn(v[4 * j + 3], s)),
-                                   __NV_SATFINITE, __NV_E4M3);
-      w[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-    }
-    if (!wide) {
-      *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(y) + e) = make_uint2(w[0], w[1]);
-    } else {
-      uint32_t h[4];
+    for (int u = 0; u < kQU; ++u)
+      if (b + u * kQThreads < n_vec) fetch(b + u * kQThreads, wr[u]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const __half2_raw p2 = __nv_cvt_fp8x2_to_halfraw2(
-            static_cast<__nv_fp8x2_storage_t>((w[j >> 1] >> (16 * (j & 1))) & 0xffffu), __NV_E4M3);
-        h[j] = static_cast<uint32_t>(p2.x) | (static_cast<uint32_t>(p2.y) << 16);
+    for (int u = 0; u < kQU; ++u) {
+      const int i = b + u * kQThreads;
+      if (i >= n_vec) continue;
+      float v[8];
+      unpack(i, wr[u], v);
+      const int l = t0 + i / vpr, c = i % vpr;
+      const int64_t e = (static_cast<int64_t>(l) * H + h) * D + c * 8;
+      uint32_t w[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const __nv_fp8x2_storage_t lo =
+            __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[4 * j], s), __fdiv_rn(v[4 * j + 1], s)),
+                                     __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi =
+            __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[4 * j + 2], s), __fdiv_rn(v[4 * j + 3], s)),
+                                     __NV_SATFINITE, __NV_E4M3);
+        w[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
       }
-      *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(y) + e) = make_uint4(h[0], h[1], h[2], h[3]);
-    }
-  }
-}
-
-// amax bits -> scale (in place): s = absmax/448, or 1 for an all-zero head.
-__global__ void finalize_scale_kernel(unsigned *a, unsigned *b, int n) {
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const float x = __uint_as_float(a[i]);
-    reinterpret_cast<float *>(a)[i] = x > 0.f ? __fdiv_rn(x, 448.f) : 1.f;
-    if (b) {
-      const float y = __uint_as_float(b[i]);
-      reinterpret_cast<float *>(b)[i] = y > 0.f ? __fdiv_rn(y, 448.f) : 1.f;
+      if (!wide) {
+        *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(y) + e) = make_uint2(w[0], w[1]);
+      } else {
+        uint32_t hw[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2_raw p2 = __nv_cvt_fp8x2_to_halfraw2(
+              static_cast<__nv_fp8x2_storage_t>((w[j >> 1] >> (16 * (j & 1))) & 0xffffu), __NV_E4M3);
+          hw[j] = static_cast<uint32_t>(p2.x) | (static_cast<uint32_t>(p2.y) << 16);
+        }
+        *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(y) + e) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      }
     }
   }
 }
@@ -351,29 +356,12 @@ static cca_status bulk_copy_pair(const uint8_t *k_src, const uint8_t *v_src, uin
 static cca_status quantize_pair(const void *x0, const void *x1, cca_dtype src, int n_tok, int H, int D,
                                 void *y0, void *y1, float *s0, float *s1, cudaStream_t st,
                                 RopeArgs r0 = RopeArgs{nullptr, nullptr}, int wide0 = 0, int wide1 = 0) {
-  const int nt = x1 ? 2 : 1;
-  unsigned *a0 = reinterpret_cast<unsigned *>(s0), *a1 = reinterpret_cast<unsigned *>(s1);
-  zero_u32_kernel<<<1, 256, 0, st>>>(a0, x1 ? a1 : nullptr, H);
-  CCA_TRY(launched("zero_u32_kernel"));
-  if (n_tok > 0) {
-    const int rows_per_block = 256 / (D / 8);
-    int bx = (n_tok + rows_per_block - 1) / rows_per_block;
-    const int target = (num_sms() * 8 + H * nt - 1) / (H * nt);  // ~8 blocks per SM in total
-    if (bx > target) bx = target > 0 ? target : 1;
-    dim3 grid(bx, H, nt);
-    if (src == CCA_F32) {
-      absmax_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D, r0);
-      CCA_TRY(launched("absmax_kernel"));
-      quant_e4m3_kernel<true><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D, r0, wide0, wide1);
-    } else {
-      absmax_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, n_tok, H, D, r0);
-      CCA_TRY(launched("absmax_kernel"));
-      quant_e4m3_kernel<false><<<grid, 256, 0, st>>>(x0, x1, a0, a1, y0, y1, n_tok, H, D, r0, wide0, wide1);
-    }
-    CCA_TRY(launched("quant_e4m3_kernel"));
-  }
-  finalize_scale_kernel<<<1, 256, 0, st>>>(a0, x1 ? a1 : nullptr, H);
-  return launched("finalize_scale_kernel");
+  const dim3 grid(kQC, H, x1 ? 2 : 1);
+  if (src == CCA_F32)
+    quant_cluster_kernel<true><<<grid, kQThreads, 0, st>>>(x0, x1, y0, y1, s0, s1, n_tok, H, D, r0, wide0, wide1);
+  else
+    quant_cluster_kernel<false><<<grid, kQThreads, 0, st>>>(x0, x1, y0, y1, s0, s1, n_tok, H, D, r0, wide0, wide1);
+  return launched("quant_cluster_kernel");
 }
 
 }  // namespace cca

@@ -15,23 +15,6 @@
 
 namespace cca {
 
-template <bool kF32>
-__device__ __forceinline__ void load8f(const void *base, int64_t elem, float (&x)[8]) {
-  if constexpr (kF32) {
-    const float4 a = __ldcs(reinterpret_cast<const float4 *>(static_cast<const float *>(base) + elem));
-    const float4 b = __ldcs(reinterpret_cast<const float4 *>(static_cast<const float *>(base) + elem + 4));
-    x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = b.x, x[5] = b.y, x[6] = b.z, x[7] = b.w;
-  } else {
-    const uint4 u = __ldcs(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(base) + elem));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      x[2 * j] = __uint_as_float(w[j] << 16);
-      x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-    }
-  }
-}
-
 __device__ __forceinline__ uint4 pack8_bf16(const float (&x)[8]) {
   uint32_t w[4];
 #pragma unroll
@@ -42,23 +25,28 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&x)[8]) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Rows kernel: a block takes kRopeTok tokens at a time.  It first fills a
-// shared table of (cos, sin) for their D/2 planes -- one sincosf per plane and
-// token, shared by all heads -- then streams both tensors' 16-byte vectors of
-// those tokens: rotated (rot0 / rot1) or only copied, rounded to bf16.
-constexpr int kRopeTok = 4;
+// A block takes kRopeTok tokens at a time: it first fills a shared table of
+// (cos, sin) for their D/2 planes -- one sincosf per token and plane, shared by
+// all heads (an accurate sincosf costs on the order of a hundred instructions,
+// so computing it per element made the rotation compute-bound) -- then streams
+// both tensors' 16-byte vectors of those tokens, kRopeU raw loads in flight per
+// thread before any is converted, rotated (or only copied) and stored as bf16.
+constexpr int kRopeTok = 8;
+constexpr int kRopeU = 8;
 constexpr int kRopeThreads = 256;
 
-template <bool kF32>
+template <bool kF32, int D>
 __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(const void *__restrict__ x0,
                                                                  const void *__restrict__ x1, uint4 *__restrict__ y0,
                                                                  uint4 *__restrict__ y1, int rot0, int rot1,
-                                                                 RopeArgs r, int n_tok, int H, int D) {
-  __shared__ float2 cs[kRopeTok][64];  // (cos, sin) per token and plane, D/2 <= 64
-  const int P = D / 2;
-  const int vpt = H * D / 8;  // 16-byte vectors (8 elements) per token and tensor
+                                                                 RopeArgs r, int H, int n_tok) {
+  constexpr int P = D / 2;
+  constexpr int kVpd = D / 8;  // vectors per head row
+  __shared__ float2 cs[kRopeTok][P];
+  const int vpt = H * kVpd;  // vectors per token
   for (int t0 = blockIdx.x * kRopeTok; t0 < n_tok; t0 += gridDim.x * kRopeTok) {
     const int nt = min(kRopeTok, n_tok - t0);
+    __syncthreads();  // the previous tokens' table is no longer read
     if (rot0 | rot1) {
       for (int e = threadIdx.x; e < nt * P; e += kRopeThreads) {
         const int tt = e / P, i = e - tt * P;
@@ -71,59 +59,83 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(const void *__r
         sincosf(th, &sn, &c);
         cs[tt][i] = make_float2(c, sn);
       }
-      __syncthreads();
     }
+    __syncthreads();
     const int nv = nt * vpt;
+    const int64_t v0 = static_cast<int64_t>(t0) * vpt;
     for (int tensor = 0; tensor < 2; ++tensor) {
       const void *x = tensor == 0 ? x0 : x1;
       uint4 *y = tensor == 0 ? y0 : y1;
       const bool rot = (tensor == 0 ? rot0 : rot1) != 0;
       if (!x) continue;
-      const int64_t v0 = static_cast<int64_t>(t0) * vpt;
-      constexpr int kU = 6;  // vectors in flight per thread
-      for (int b = threadIdx.x; b < nv; b += kU * kRopeThreads) {
-        float v[kU][8];
+      for (int b = threadIdx.x; b < nv; b += kRopeU * kRopeThreads) {
+        uint4 raw[kRopeU][kF32 ? 2 : 1];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
+        for (int u = 0; u < kRopeU; ++u) {
           const int i = b + u * kRopeThreads;
-          if (i < nv) load8f<kF32>(x, (v0 + i) * 8, v[u]);
+          if (i < nv) {
+            if constexpr (kF32) {
+              raw[u][0] = __ldcs(reinterpret_cast<const uint4 *>(x) + 2 * (v0 + i));
+              raw[u][1] = __ldcs(reinterpret_cast<const uint4 *>(x) + 2 * (v0 + i) + 1);
+            } else {
+              raw[u][0] = __ldcs(reinterpret_cast<const uint4 *>(x) + v0 + i);
+            }
+          }
         }
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
+        for (int u = 0; u < kRopeU; ++u) {
           const int i = b + u * kRopeThreads;
           if (i >= nv) continue;
+          float v[8];
+          if constexpr (kF32) {
+            const uint32_t w[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                                   raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(w[j]);
+          } else {
+            const uint32_t w[4] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              v[2 * j] = __uint_as_float(w[j] << 16);
+              v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+            }
+          }
           if (rot) {
             const int tt = i / vpt;
-            const int pl = ((i - tt * vpt) * 4) % P;  // first plane of the vector: (8 elements / 2) per vector
+            const int pl = (i % kVpd) * 4;  // first of the vector's 4 planes
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const float2 c = cs[tt][pl + j];
-              const float a = v[u][2 * j], bb = v[u][2 * j + 1];
-              v[u][2 * j] = fmaf(a, c.x, -bb * c.y);
-              v[u][2 * j + 1] = fmaf(a, c.y, bb * c.x);
+              const float a = v[2 * j], bb = v[2 * j + 1];
+              v[2 * j] = fmaf(a, c.x, -bb * c.y);
+              v[2 * j + 1] = fmaf(a, c.y, bb * c.x);
             }
           }
-          y[v0 + i] = pack8_bf16(v[u]);
+          y[v0 + i] = pack8_bf16(v);
         }
       }
     }
-    __syncthreads();
   }
 }
 
 // Launcher shared with the clean-KV append (ring.cu).
 cca_status launch_rope_rows(const void *x0, const void *x1, void *y0, void *y1, bool rot0, bool rot1, bool f32,
                             RopeArgs r, int n_tok, int H, int D, cudaStream_t st) {
+  if (n_tok == 0) return CCA_OK;
+  if (static_cast<int64_t>(kRopeTok) * H * D / 8 >= (int64_t(1) << 31))
+    return fail(CCA_ERR_INVALID_ARG, "rotary encoding: H * D too large");
   int blocks = (n_tok + kRopeTok - 1) / kRopeTok;
   const int cap = num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  if (blocks < 1) return CCA_OK;
-  if (f32)
-    rope_rows_kernel<true><<<blocks, kRopeThreads, 0, st>>>(x0, x1, static_cast<uint4 *>(y0), static_cast<uint4 *>(y1),
-                                                           rot0, rot1, r, n_tok, H, D);
-  else
-    rope_rows_kernel<false><<<blocks, kRopeThreads, 0, st>>>(x0, x1, static_cast<uint4 *>(y0),
-                                                            static_cast<uint4 *>(y1), rot0, rot1, r, n_tok, H, D);
+  uint4 *a = static_cast<uint4 *>(y0), *b = static_cast<uint4 *>(y1);
+  const int r0 = rot0, r1 = rot1;
+  if (f32) {
+    if (D == 128) rope_rows_kernel<true, 128><<<blocks, kRopeThreads, 0, st>>>(x0, x1, a, b, r0, r1, r, H, n_tok);
+    else rope_rows_kernel<true, 64><<<blocks, kRopeThreads, 0, st>>>(x0, x1, a, b, r0, r1, r, H, n_tok);
+  } else {
+    if (D == 128) rope_rows_kernel<false, 128><<<blocks, kRopeThreads, 0, st>>>(x0, x1, a, b, r0, r1, r, H, n_tok);
+    else rope_rows_kernel<false, 64><<<blocks, kRopeThreads, 0, st>>>(x0, x1, a, b, r0, r1, r, H, n_tok);
+  }
   return launched("rope_rows_kernel");
 }
 
