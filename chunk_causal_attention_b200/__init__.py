@@ -23,7 +23,7 @@ __all__ = [
     "cca_kv_append", "cca_quant_e4m3", "cca_chunk_attn", "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc",
     "cca_chunk_attn_scatter", "cca_attn_workspace_size", "cca_chunk_attn_groups", "cca_block_attn",
     "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope", "cca_token_mask_l2_frames", "cca_quant_e4m3_f16",
-    "cca_token_mask_l2", "cca_compact", "cca_compact_workspace_size", "cca_scatter", "cca_selftest_bounded_wait",
+    "cca_quant_e4m3_qkv", "cca_token_mask_l2", "cca_compact", "cca_compact_workspace_size", "cca_scatter", "cca_selftest_bounded_wait",
     "cca_version",
     "cca_take_launch_count",
 ]
@@ -36,7 +36,8 @@ _STATUS = {0: "CCA_OK", 1: "CCA_ERR_INVALID_ARG", 2: "CCA_ERR_UNSUPPORTED", 3: "
 # Every entry point declared in include/cca.h.
 EXPORTED = (
     "cca_kv_ring_create", "cca_kv_ring_destroy", "cca_kv_ring_reset", "cca_kv_ring_query",
-    "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_quant_e4m3_f16", "cca_chunk_attn",
+    "cca_kv_ring_restore", "cca_kv_append", "cca_quant_e4m3", "cca_quant_e4m3_f16", "cca_quant_e4m3_qkv",
+    "cca_chunk_attn",
     "cca_chunk_attn_workspace_size", "cca_chunk_attn_noalloc", "cca_chunk_attn_scatter", "cca_attn_workspace_size",
     "cca_chunk_attn_groups", "cca_block_attn", "cca_mrope_freqs", "cca_rope_qk", "cca_kv_append_rope",
     "cca_token_mask_l2", "cca_token_mask_l2_frames", "cca_compact",
@@ -96,6 +97,7 @@ def lib() -> ctypes.CDLL:
         "cca_kv_append": [vp, vp, vp, ctypes.c_int, vp],
         "cca_quant_e4m3": [vp, ctypes.c_int, i32, i32, i32, vp, vp, vp],
         "cca_quant_e4m3_f16": [vp, ctypes.c_int, i32, i32, i32, vp, vp, vp],
+        "cca_quant_e4m3_qkv": [vp, vp, vp, ctypes.c_int, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp],
         "cca_chunk_attn": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp],
         "cca_chunk_attn_workspace_size": [vp, i32, ctypes.POINTER(sz)],
         "cca_chunk_attn_noalloc": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp],
@@ -306,6 +308,25 @@ def cca_quant_e4m3_f16(x: torch.Tensor, x16: Optional[torch.Tensor] = None, scal
     _check(lib().cca_quant_e4m3_f16(_ptr(x, "x"), _src_dtype(x), n, h, d, _ptr(x16, "x16", torch.float16),
                                     _ptr(scale, "scale", torch.float32), _stream(stream)), "cca_quant_e4m3_f16")
     return x16, scale
+
+
+def cca_quant_e4m3_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None):
+    """The three inputs of an E4M3 attention call quantised in one launch:
+    returns (q8, q_scale, k8, k_scale, v16, v_scale), the same values as
+    cca_quant_e4m3(q), cca_quant_e4m3(k) and cca_quant_e4m3_f16(v)."""
+    n, h, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("cca_quant_e4m3_qkv: q, k and v must share shape and dtype")
+    q8 = torch.empty((n, h, d), dtype=torch.uint8, device=q.device)
+    k8 = torch.empty_like(q8)
+    v16 = torch.empty((n, h, d), dtype=torch.float16, device=q.device)
+    qs, ks, vs = (torch.empty(h, dtype=torch.float32, device=q.device) for _ in range(3))
+    _check(lib().cca_quant_e4m3_qkv(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _src_dtype(q), n, h, d,
+                                    _ptr(q8, "q8", torch.uint8), _ptr(k8, "k8", torch.uint8),
+                                    _ptr(v16, "v16", torch.float16), _ptr(qs, "q_scale", torch.float32),
+                                    _ptr(ks, "k_scale", torch.float32), _ptr(vs, "v_scale", torch.float32),
+                                    _stream(stream)), "cca_quant_e4m3_qkv")
+    return q8, qs, k8, ks, v16, vs
 
 
 def cca_chunk_attn_workspace_size(ring: KVRing, n_q_max: int) -> int:

@@ -199,132 +199,207 @@ __global__ void __launch_bounds__(32, 1) append_bulk_kernel(const uint8_t *__res
 }
 
 // Single-launch per-head quantisation: a cluster of kQC CTAs per (tensor,
-// head), each over a quarter of the tokens.  Pass 1: the CTA's absmax (warp
+// head), each over an eighth of the tokens.  Pass 1: the CTA's absmax (warp
 // shuffles, then shared memory); the cluster's maximum is read from the other
 // CTAs' shared memory after a hardware cluster barrier.  Pass 2: the CTA
-// quantises its rows (read again, from L2), with s = absmax / 448 (1 for an
-// all-zero head), exactly the rule of the multi-kernel path.  Rank 0 writes the
-// scale.  A second cluster barrier keeps every CTA's shared memory alive until
-// the others have read it.
-constexpr int kQC = 4;          // CTAs per (tensor, head)
-constexpr int kQThreads = 512;
+// quantises its rows with s = absmax / 448 (1 for an all-zero head) and codes
+// e4m3_rn_satfinite(x / s), both IEEE fp32 divisions.  Rank 0 writes the scale.  A second
+// cluster barrier keeps every CTA's shared memory alive until the others have
+// read it.  Two kernels share this structure:
+//   quant_cpa_kernel: every thread copies its vectors into shared memory with
+//     cp.async, all in flight at once, so the tensor is read from HBM once
+//     (up to 64 KB of rows per CTA: 2048 tokens of a 128-wide bf16 head);
+//   quant_cluster_kernel: larger heads are streamed twice from global memory
+//     (pass 2 mostly from L2), kQU loads in flight per thread.
+constexpr int kQC = 8;          // CTAs per (tensor, head): a portable cluster
+constexpr int kQThreads = 256;
 
+// 8 elements (16 bytes of bf16, or 2 x 16 bytes of fp32) -> fp32, optionally rotated.
 template <bool kF32>
-__global__ void __cluster_dims__(kQC, 1, 1) __launch_bounds__(kQThreads)
-    quant_cluster_kernel(const void *__restrict__ x0, const void *__restrict__ x1, void *__restrict__ y0,
-                         void *__restrict__ y1, float *__restrict__ s0, float *__restrict__ s1, int n_tok, int H,
-                         int D, RopeArgs rope0, int wide0, int wide1) {
-  const int tensor = blockIdx.z, h = blockIdx.y, rank = blockIdx.x;  // cluster = the kQC CTAs of (tensor, h)
-  const void *x = tensor == 0 ? x0 : x1;
-  void *y = tensor == 0 ? y0 : y1;
-  float *scale = tensor == 0 ? s0 : s1;
-  const bool wide = (tensor == 0 ? wide0 : wide1) != 0;
-  const bool rot = tensor == 0 && rope0.pos != nullptr;
-  const int vpr = D / 8;  // 16-byte (8-element) vectors per row of one head
-  const int t0 = static_cast<int>(static_cast<int64_t>(n_tok) * rank / kQC);
-  const int t1 = static_cast<int>(static_cast<int64_t>(n_tok) * (rank + 1) / kQC);
-  const int n_vec = (t1 - t0) * vpr;
-  __shared__ float red[kQThreads / 32];
-  __shared__ float cta_max;
-  // kQU raw 16-byte loads in flight per thread before any is used
-  constexpr int kQU = 4;
-  constexpr int kW = kF32 ? 2 : 1;  // 16-byte words per 8 elements
-  auto fetch = [&](int i, uint4 (&w)[kW]) {
-    const int l = t0 + i / vpr, c = i % vpr;
-    const int64_t e = (static_cast<int64_t>(l) * H + h) * D + c * 8;
-    if constexpr (kF32) {
-      w[0] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + e));
-      w[1] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + e) + 1);
-    } else {
-      w[0] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + e));
-    }
-  };
-  auto unpack = [&](int i, const uint4 (&w)[kW], float (&v)[8]) {
-    if constexpr (kF32) {
-      const uint32_t u[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+__device__ __forceinline__ void q_unpack(const uint4 *w, float (&v)[8]) {
+  if constexpr (kF32) {
+    const uint32_t u[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(u[j]);
-    } else {
-      const uint32_t u[4] = {w[0].x, w[0].y, w[0].z, w[0].w};
+    for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(u[j]);
+  } else {
+    const uint32_t u[4] = {w[0].x, w[0].y, w[0].z, w[0].w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[2 * j] = __uint_as_float(u[j] << 16);
-        v[2 * j + 1] = __uint_as_float(u[j] & 0xffff0000u);
-      }
-    }
-    if (rot) rope8(rope0, t0 + i / vpr, (i % vpr) * 8, D, v);
-  };
-  float m = 0.f;
-  for (int b = threadIdx.x; b < n_vec; b += kQU * kQThreads) {
-    uint4 w[kQU][kW];
-#pragma unroll
-    for (int u = 0; u < kQU; ++u)
-      if (b + u * kQThreads < n_vec) fetch(b + u * kQThreads, w[u]);
-#pragma unroll
-    for (int u = 0; u < kQU; ++u) {
-      if (b + u * kQThreads >= n_vec) continue;
-      float v[8];
-      unpack(b + u * kQThreads, w[u], v);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(u[j] << 16);
+      v[2 * j + 1] = __uint_as_float(u[j] & 0xffff0000u);
     }
   }
+}
+
+// Codes of 8 elements at element offset e of y: e4m3 bytes, or (wide) their values as fp16.
+__device__ __forceinline__ void q_store8(void *y, int64_t e, const float (&v)[8], float s, bool wide) {
+  uint32_t w[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(v[4 * j], s), __fdiv_rn(v[4 * j + 1], s)), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(v[4 * j + 2], s), __fdiv_rn(v[4 * j + 3], s)), __NV_SATFINITE, __NV_E4M3);
+    w[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+  }
+  if (!wide) {
+    *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(y) + e) = make_uint2(w[0], w[1]);
+  } else {
+    uint32_t hw[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2_raw p2 = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((w[j >> 1] >> (16 * (j & 1))) & 0xffffu), __NV_E4M3);
+      hw[j] = static_cast<uint32_t>(p2.x) | (static_cast<uint32_t>(p2.y) << 16);
+    }
+    *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(y) + e) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  }
+}
+
+// The cluster-wide absmax: CTA maximum m (every thread's partial), then the
+// maximum over the cluster's CTAs through distributed shared memory.  Ends
+// with the second cluster barrier, after which the shared words may be reused.
+__device__ __forceinline__ float q_cluster_max(float m, float *red, float *cta_max) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   if (threadIdx.x == 0) {
     for (int w = 1; w < kQThreads / 32; ++w) m = fmaxf(m, red[w]);
-    cta_max = m;
+    *cta_max = m;
   }
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   float a = 0.f;
-  for (int r = 0; r < kQC; ++r) {  // the cluster's CTAs' maxima, read through distributed shared memory
-    uint32_t local = smem_u32(&cta_max), remote;
+  for (int r = 0; r < kQC; ++r) {
+    uint32_t local = smem_u32(cta_max), remote;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(r));
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
     a = fmaxf(a, v);
   }
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  return a;
+}
+
+struct QuantArgs {  // up to three tensors of one shape, blockIdx.z selects one
+  const void *x[3];
+  void *y[3];
+  float *scale[3];
+  int wide[3];
+  RopeArgs rope0;  // rotation of tensor 0 before quantising (pos == nullptr: none)
+  int n_tok, H, n_tensors;
+};
+
+// 16-byte word(s) of the 8 elements of vector i (row t0 + i / vpr, column i % vpr) of head h.
+template <bool kF32, int D>
+__device__ __forceinline__ void q_fetch(const void *x, int H, int h, int t0, int i, uint4 *w) {
+  constexpr int vpr = D / 8;
+  const int64_t e = (static_cast<int64_t>(t0 + i / vpr) * H + h) * D + (i % vpr) * 8;
+  if constexpr (kF32) {
+    w[0] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + e));
+    w[1] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + e) + 1);
+  } else {
+    w[0] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + e));
+  }
+}
+
+// Shared-memory form: every thread copies its vectors into shared memory
+// with cp.async (all in flight at once, no registers held), then both passes
+// read shared memory.
+template <bool kF32, int D>
+__global__ void __cluster_dims__(kQC, 1, 1) __launch_bounds__(kQThreads)
+    quant_cpa_kernel(const __grid_constant__ QuantArgs q) {
+  extern __shared__ __align__(16) uint4 rows16[];
+  __shared__ float red[kQThreads / 32];
+  __shared__ float cta_max;
+  const int tensor = blockIdx.z, h = blockIdx.y, rank = blockIdx.x;
+  const bool rot = tensor == 0 && q.rope0.pos != nullptr;
+  constexpr int kW = kF32 ? 2 : 1;
+  constexpr int vpr = D / 8;
+  const int t0 = static_cast<int>(static_cast<int64_t>(q.n_tok) * rank / kQC);
+  const int t1 = static_cast<int>(static_cast<int64_t>(q.n_tok) * (rank + 1) / kQC);
+  const int n_vec = (t1 - t0) * vpr;
+  const uint4 *x = static_cast<const uint4 *>(q.x[tensor]);
+  for (int i = threadIdx.x; i < n_vec; i += kQThreads) {
+    const int64_t e = ((static_cast<int64_t>(t0 + i / vpr) * q.H + h) * D + (i % vpr) * 8) / (8 / kW);
+#pragma unroll
+    for (int k = 0; k < kW; ++k)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(rows16 + i * kW + k)),
+                   "l"(x + e + k)
+                   : "memory");
+  }
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  float m = 0.f;
+  for (int i = threadIdx.x; i < n_vec; i += kQThreads) {  // a thread reads back only what it copied
+    float v[8];
+    q_unpack<kF32>(rows16 + i * kW, v);
+    if (rot) rope8(q.rope0, t0 + i / vpr, (i % vpr) * 8, D, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+  }
+  const float a = q_cluster_max(m, red, &cta_max);
   const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
-  if (rank == 0 && threadIdx.x == 0) scale[h] = s;
+  if (rank == 0 && threadIdx.x == 0) q.scale[tensor][h] = s;
+  const bool wide = q.wide[tensor] != 0;
+  for (int i = threadIdx.x; i < n_vec; i += kQThreads) {
+    float v[8];
+    q_unpack<kF32>(rows16 + i * kW, v);
+    const int l = t0 + i / vpr, c = i % vpr;
+    if (rot) rope8(q.rope0, l, c * 8, D, v);
+    q_store8(q.y[tensor], (static_cast<int64_t>(l) * q.H + h) * D + c * 8, v, s, wide);
+  }
+}
+
+template <bool kF32, int D>
+__global__ void __cluster_dims__(kQC, 1, 1) __launch_bounds__(kQThreads)
+    quant_cluster_kernel(const __grid_constant__ QuantArgs q) {
+  __shared__ float red[kQThreads / 32];
+  __shared__ float cta_max;
+  const int tensor = blockIdx.z, h = blockIdx.y, rank = blockIdx.x;
+  const void *x = q.x[tensor];
+  const bool rot = tensor == 0 && q.rope0.pos != nullptr;
+  constexpr int vpr = D / 8;
+  const int t0 = static_cast<int>(static_cast<int64_t>(q.n_tok) * rank / kQC);
+  const int t1 = static_cast<int>(static_cast<int64_t>(q.n_tok) * (rank + 1) / kQC);
+  const int n_vec = (t1 - t0) * vpr;
+  // kQU raw 16-byte loads in flight per thread before any is used
+  constexpr int kQU = 4;
+  constexpr int kW = kF32 ? 2 : 1;
+  float m = 0.f;
   for (int b = threadIdx.x; b < n_vec; b += kQU * kQThreads) {
-    uint4 wr[kQU][kW];
+    uint4 w[kQU][kW];
 #pragma unroll
     for (int u = 0; u < kQU; ++u)
-      if (b + u * kQThreads < n_vec) fetch(b + u * kQThreads, wr[u]);
+      if (b + u * kQThreads < n_vec) q_fetch<kF32, D>(x, q.H, h, t0, b + u * kQThreads, w[u]);
 #pragma unroll
     for (int u = 0; u < kQU; ++u) {
       const int i = b + u * kQThreads;
       if (i >= n_vec) continue;
       float v[8];
-      unpack(i, wr[u], v);
+      q_unpack<kF32>(w[u], v);
+      if (rot) rope8(q.rope0, t0 + i / vpr, (i % vpr) * 8, D, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    }
+  }
+  const float a = q_cluster_max(m, red, &cta_max);
+  const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+  if (rank == 0 && threadIdx.x == 0) q.scale[tensor][h] = s;
+  const bool wide = q.wide[tensor] != 0;
+  for (int b = threadIdx.x; b < n_vec; b += kQU * kQThreads) {
+    uint4 wr[kQU][kW];
+#pragma unroll
+    for (int u = 0; u < kQU; ++u)
+      if (b + u * kQThreads < n_vec) q_fetch<kF32, D>(x, q.H, h, t0, b + u * kQThreads, wr[u]);
+#pragma unroll
+    for (int u = 0; u < kQU; ++u) {
+      const int i = b + u * kQThreads;
+      if (i >= n_vec) continue;
+      float v[8];
+      q_unpack<kF32>(wr[u], v);
       const int l = t0 + i / vpr, c = i % vpr;
-      const int64_t e = (static_cast<int64_t>(l) * H + h) * D + c * 8;
-      uint32_t w[2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const __nv_fp8x2_storage_t lo =
-            __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[4 * j], s), __fdiv_rn(v[4 * j + 1], s)),
-                                     __NV_SATFINITE, __NV_E4M3);
-        const __nv_fp8x2_storage_t hi =
-            __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[4 * j + 2], s), __fdiv_rn(v[4 * j + 3], s)),
-                                     __NV_SATFINITE, __NV_E4M3);
-        w[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-      }
-      if (!wide) {
-        *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(y) + e) = make_uint2(w[0], w[1]);
-      } else {
-        uint32_t hw[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const __half2_raw p2 = __nv_cvt_fp8x2_to_halfraw2(
-              static_cast<__nv_fp8x2_storage_t>((w[j >> 1] >> (16 * (j & 1))) & 0xffffu), __NV_E4M3);
-          hw[j] = static_cast<uint32_t>(p2.x) | (static_cast<uint32_t>(p2.y) << 16);
-        }
-        *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(y) + e) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      }
+      if (rot) rope8(q.rope0, l, c * 8, D, v);
+      q_store8(q.y[tensor], (static_cast<int64_t>(l) * q.H + h) * D + c * 8, v, s, wide);
     }
   }
 }
@@ -353,15 +428,46 @@ static cca_status bulk_copy_pair(const uint8_t *k_src, const uint8_t *v_src, uin
 }
 
 // Quantise one or two [n_tok][H][D] tensors; scale arrays are [H] each.
+constexpr int kQStageMax = 64 * 1024;  // shared memory per CTA of the staged form: at least 3 CTAs per SM
+
+template <bool kF32, int D>
+static cca_status quant_launch(const QuantArgs &q, cudaStream_t st) {
+  const dim3 grid(kQC, q.H, q.n_tensors);
+  const int64_t per_cta = (static_cast<int64_t>(q.n_tok) + kQC - 1) / kQC * (D / 8);  // vectors
+  const int64_t stage = per_cta * 16 * (kF32 ? 2 : 1);
+  if (stage <= kQStageMax) {
+    static std::mutex mu;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err == cudaSuccess && (dev < 0 || dev >= 64)) return fail(CCA_ERR_UNSUPPORTED, "quantise: device %d", dev);
+    if (err == cudaSuccess) {
+      std::lock_guard<std::mutex> lock(mu);
+      if (!attr_set[dev]) {
+        err = cudaFuncSetAttribute(quant_cpa_kernel<kF32, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   kQStageMax);
+        attr_set[dev] = err == cudaSuccess;
+      }
+    }
+    if (err != cudaSuccess) return fail(CCA_ERR_CUDA, "quantise: %s", cudaGetErrorString(err));
+    quant_cpa_kernel<kF32, D><<<grid, kQThreads, static_cast<size_t>(stage), st>>>(q);
+    return launched("quant_cpa_kernel");
+  }
+  quant_cluster_kernel<kF32, D><<<grid, kQThreads, 0, st>>>(q);
+  return launched("quant_cluster_kernel");
+}
+
+static cca_status quantize_args(const QuantArgs &q, cca_dtype src, int D, cudaStream_t st) {
+  if (src == CCA_F32) return D == 128 ? quant_launch<true, 128>(q, st) : quant_launch<true, 64>(q, st);
+  return D == 128 ? quant_launch<false, 128>(q, st) : quant_launch<false, 64>(q, st);
+}
+
 static cca_status quantize_pair(const void *x0, const void *x1, cca_dtype src, int n_tok, int H, int D,
                                 void *y0, void *y1, float *s0, float *s1, cudaStream_t st,
                                 RopeArgs r0 = RopeArgs{nullptr, nullptr}, int wide0 = 0, int wide1 = 0) {
-  const dim3 grid(kQC, H, x1 ? 2 : 1);
-  if (src == CCA_F32)
-    quant_cluster_kernel<true><<<grid, kQThreads, 0, st>>>(x0, x1, y0, y1, s0, s1, n_tok, H, D, r0, wide0, wide1);
-  else
-    quant_cluster_kernel<false><<<grid, kQThreads, 0, st>>>(x0, x1, y0, y1, s0, s1, n_tok, H, D, r0, wide0, wide1);
-  return launched("quant_cluster_kernel");
+  const QuantArgs q{{x0, x1, nullptr}, {y0, y1, nullptr}, {s0, s1, nullptr}, {wide0, wide1, 0}, r0, n_tok, H,
+                    x1 ? 2 : 1};
+  return quantize_args(q, src, D, st);
 }
 
 }  // namespace cca
@@ -513,6 +619,26 @@ cca_status cca_quant_e4m3_f16(const void *x, cca_dtype src_dtype, int32_t n_tok,
     return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_f16: scale must be 4-byte aligned");
   return quantize_pair(x, nullptr, src_dtype, n_tok, n_heads, head_dim, x16, nullptr, scale, nullptr,
                        reinterpret_cast<cudaStream_t>(stream), RopeArgs{nullptr, nullptr}, 1, 0);
+}
+
+cca_status cca_quant_e4m3_qkv(const void *q, const void *k, const void *v, cca_dtype src_dtype, int32_t n_tok,
+                              int32_t n_heads, int32_t head_dim, uint8_t *q8, uint8_t *k8, void *v16, float *q_scale,
+                              float *k_scale, float *v_scale, cca_stream_t stream) {
+  if (!q_scale || !k_scale || !v_scale || (n_tok > 0 && (!q || !k || !v || !q8 || !k8 || !v16)))
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_qkv: NULL argument");
+  if (n_tok < 0 || n_heads < 1 || (head_dim != 64 && head_dim != 128))
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_qkv: need n_tok >= 0, H >= 1, D in {64,128}");
+  if (src_dtype != CCA_BF16 && src_dtype != CCA_F32)
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_qkv: src_dtype must be CCA_BF16 or CCA_F32");
+  if (n_tok > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) ||
+                    !aligned16(v16)))
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_qkv: tensors must be 16-byte aligned");
+  if (((reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale) |
+        reinterpret_cast<uintptr_t>(v_scale)) & 3u) != 0)
+    return fail(CCA_ERR_INVALID_ARG, "cca_quant_e4m3_qkv: scales must be 4-byte aligned");
+  const QuantArgs a{{q, k, v}, {q8, k8, v16}, {q_scale, k_scale, v_scale}, {0, 0, 1}, RopeArgs{nullptr, nullptr},
+                    n_tok, n_heads, 3};
+  return quantize_args(a, src_dtype, head_dim, reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char *cca_last_error(void) { return last_error().c_str(); }

@@ -25,13 +25,15 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&x)[8]) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// A block takes kRopeTok tokens at a time: it first fills a shared table of
-// (cos, sin) for their D/2 planes -- one sincosf per token and plane, shared by
-// all heads (an accurate sincosf costs on the order of a hundred instructions,
-// so computing it per element made the rotation compute-bound) -- then streams
-// both tensors' 16-byte vectors of those tokens, kRopeU raw loads in flight per
-// thread before any is converted, rotated (or only copied) and stored as bf16.
-constexpr int kRopeTok = 8;
+// A block takes kRopeTok tokens at a time (810 blocks at 1620 tokens, so that
+// several blocks' loads are in flight on every SM): it first fills a shared
+// table of (cos, sin) for their D/2 planes -- one sincosf per token and plane,
+// shared by all heads (an accurate sincosf costs on the order of a hundred
+// instructions, so computing it per element made the rotation compute-bound)
+// -- then streams the 16-byte vectors of those tokens of both tensors as one
+// index range, kRopeU raw loads in flight per thread before any is converted,
+// rotated (or only copied) and stored as bf16.  x1 == nullptr: one tensor.
+constexpr int kRopeTok = 2;
 constexpr int kRopeU = 8;
 constexpr int kRopeThreads = 256;
 
@@ -47,45 +49,56 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(const void *__r
   for (int t0 = blockIdx.x * kRopeTok; t0 < n_tok; t0 += gridDim.x * kRopeTok) {
     const int nt = min(kRopeTok, n_tok - t0);
     __syncthreads();  // the previous tokens' table is no longer read
-    if (rot0 | rot1) {
-      for (int e = threadIdx.x; e < nt * P; e += kRopeThreads) {
-        const int tt = e / P, i = e - tt * P;
-        const int4 p = __ldg(reinterpret_cast<const int4 *>(r.pos) + t0 + tt);
-        const float th = fmaf(static_cast<float>(p.w), __ldg(r.freq + 3 * P + i),
-                              fmaf(static_cast<float>(p.z), __ldg(r.freq + 2 * P + i),
-                                   fmaf(static_cast<float>(p.y), __ldg(r.freq + P + i),
-                                        static_cast<float>(p.x) * __ldg(r.freq + i))));
-        float sn, c;
-        sincosf(th, &sn, &c);
-        cs[tt][i] = make_float2(c, sn);
-      }
-    }
-    __syncthreads();
     const int nv = nt * vpt;
+    const int n_all = x1 ? 2 * nv : nv;
     const int64_t v0 = static_cast<int64_t>(t0) * vpt;
-    for (int tensor = 0; tensor < 2; ++tensor) {
-      const void *x = tensor == 0 ? x0 : x1;
-      uint4 *y = tensor == 0 ? y0 : y1;
-      const bool rot = (tensor == 0 ? rot0 : rot1) != 0;
-      if (!x) continue;
-      for (int b = threadIdx.x; b < nv; b += kRopeU * kRopeThreads) {
-        uint4 raw[kRopeU][kF32 ? 2 : 1];
+    // The first batch of loads is issued before the table is computed, so the
+    // sincosf work overlaps their latency; every thread runs the first batch.
+    int b = threadIdx.x;
+    bool first = true;
+    do {
+      uint4 raw[kRopeU][kF32 ? 2 : 1];
 #pragma unroll
-        for (int u = 0; u < kRopeU; ++u) {
-          const int i = b + u * kRopeThreads;
-          if (i < nv) {
-            if constexpr (kF32) {
-              raw[u][0] = __ldcs(reinterpret_cast<const uint4 *>(x) + 2 * (v0 + i));
-              raw[u][1] = __ldcs(reinterpret_cast<const uint4 *>(x) + 2 * (v0 + i) + 1);
-            } else {
-              raw[u][0] = __ldcs(reinterpret_cast<const uint4 *>(x) + v0 + i);
-            }
+      for (int u = 0; u < kRopeU; ++u) {
+        const int c = b + u * kRopeThreads;
+        if (c < n_all) {
+          const bool second = c >= nv;
+          const void *x = second ? x1 : x0;
+          const int64_t e = v0 + (second ? c - nv : c);
+          if constexpr (kF32) {
+            raw[u][0] = __ldcs(reinterpret_cast<const uint4 *>(x) + 2 * e);
+            raw[u][1] = __ldcs(reinterpret_cast<const uint4 *>(x) + 2 * e + 1);
+          } else {
+            raw[u][0] = __ldcs(reinterpret_cast<const uint4 *>(x) + e);
           }
         }
+      }
+      if (first) {
+        first = false;
+        if (rot0 | rot1) {
+          for (int e = threadIdx.x; e < nt * P; e += kRopeThreads) {
+            const int tt = e / P, i = e - tt * P;
+            const int4 p = __ldg(reinterpret_cast<const int4 *>(r.pos) + t0 + tt);
+            const float th = fmaf(static_cast<float>(p.w), __ldg(r.freq + 3 * P + i),
+                                  fmaf(static_cast<float>(p.z), __ldg(r.freq + 2 * P + i),
+                                       fmaf(static_cast<float>(p.y), __ldg(r.freq + P + i),
+                                            static_cast<float>(p.x) * __ldg(r.freq + i))));
+            float sn, cn;
+            sincosf(th, &sn, &cn);
+            cs[tt][i] = make_float2(cn, sn);
+          }
+        }
+        __syncthreads();
+      }
 #pragma unroll
-        for (int u = 0; u < kRopeU; ++u) {
-          const int i = b + u * kRopeThreads;
-          if (i >= nv) continue;
+      for (int u = 0; u < kRopeU; ++u) {
+        const int c = b + u * kRopeThreads;
+        if (c >= n_all) continue;
+        const bool second = c >= nv;
+        const int i = second ? c - nv : c;
+        uint4 *y = second ? y1 : y0;
+        const bool rot = (second ? rot1 : rot0) != 0;
+        {
           float v[8];
           if constexpr (kF32) {
             const uint32_t w[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
@@ -101,20 +114,23 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(const void *__r
             }
           }
           if (rot) {
-            const int tt = i / vpt;
+            int tt = 0;
+#pragma unroll
+            for (int k = 1; k < kRopeTok; ++k) tt += i >= k * vpt;
             const int pl = (i % kVpd) * 4;  // first of the vector's 4 planes
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float2 c = cs[tt][pl + j];
+              const float2 cw = cs[tt][pl + j];
               const float a = v[2 * j], bb = v[2 * j + 1];
-              v[2 * j] = fmaf(a, c.x, -bb * c.y);
-              v[2 * j + 1] = fmaf(a, c.y, bb * c.x);
+              v[2 * j] = fmaf(a, cw.x, -bb * cw.y);
+              v[2 * j + 1] = fmaf(a, cw.y, bb * cw.x);
             }
           }
           y[v0 + i] = pack8_bf16(v);
         }
       }
-    }
+      b += kRopeU * kRopeThreads;
+    } while (b < n_all);
   }
 }
 
@@ -122,8 +138,12 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(const void *__r
 cca_status launch_rope_rows(const void *x0, const void *x1, void *y0, void *y1, bool rot0, bool rot1, bool f32,
                             RopeArgs r, int n_tok, int H, int D, cudaStream_t st) {
   if (n_tok == 0) return CCA_OK;
-  if (static_cast<int64_t>(kRopeTok) * H * D / 8 >= (int64_t(1) << 31))
+  if (2 * static_cast<int64_t>(kRopeTok) * H * D / 8 >= (int64_t(1) << 31))
     return fail(CCA_ERR_INVALID_ARG, "rotary encoding: H * D too large");
+  if (!x0) {  // only the second tensor given: run it as the first
+    x0 = x1, y0 = y1, rot0 = rot1;
+    x1 = nullptr, y1 = nullptr;
+  }
   int blocks = (n_tok + kRopeTok - 1) / kRopeTok;
   const int cap = num_sms() * 8;
   if (blocks > cap) blocks = cap;

@@ -194,6 +194,16 @@ cca_status cca_quant_e4m3(const void *x, cca_dtype src_dtype, int32_t n_tok,
 cca_status cca_quant_e4m3_f16(const void *x, cca_dtype src_dtype, int32_t n_tok, int32_t n_heads,
                               int32_t head_dim, void *x16, float *scale, cca_stream_t stream);
 
+/* The current chunk's three attention inputs in one launch, each with its own
+ * per-head scales: q8 = codes of q, k8 = codes of k, v16 = codes of v widened
+ * to fp16 -- exactly cca_quant_e4m3(q), cca_quant_e4m3(k) and
+ * cca_quant_e4m3_f16(v), the operands of an E4M3 cca_chunk_attn call.  All
+ * tensors [n_tok][H][D], 16-byte aligned; scales device [H] fp32.
+ * Errors: as cca_quant_e4m3. */
+cca_status cca_quant_e4m3_qkv(const void *q, const void *k, const void *v, cca_dtype src_dtype, int32_t n_tok,
+                              int32_t n_heads, int32_t head_dim, uint8_t *q8, uint8_t *k8, void *v16,
+                              float *q_scale, float *k_scale, float *v_scale, cca_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Chunk attention                                                           */
 /* ------------------------------------------------------------------------ */

@@ -140,6 +140,14 @@ def test_call_validation_without_device_work(L):
     assert L.cca_scatter(vp(0x1000), vp(0x1000), vp(0x1000), 4, 20, vp(0x1000), None) == 1
     assert L.cca_scatter(None, None, None, 0, 16, None, None) == 0
     assert L.cca_quant_e4m3(vp(0x1000), cca.CCA_BF16, 4, 2, 80, vp(0x1000), vp(0x1000), None) == 1
+    qkv = L.cca_quant_e4m3_qkv
+    a = vp(0x1000)
+    assert qkv(a, a, a, cca.CCA_BF16, 4, 2, 80, a, a, a, a, a, a, None) == 1  # D not in {64, 128}
+    assert qkv(a, None, a, cca.CCA_BF16, 4, 2, 64, a, a, a, a, a, a, None) == 1  # missing k
+    assert qkv(a, a, a, cca.CCA_BF16, 4, 2, 64, a, a, a, a, None, a, None) == 1  # missing k_scale
+    assert qkv(a, a, vp(0x1008), cca.CCA_BF16, 4, 2, 64, a, a, a, a, a, a, None) == 1  # v misaligned
+    assert qkv(a, a, a, cca.CCA_E4M3, 4, 2, 64, a, a, a, a, a, a, None) == 1  # source must be BF16 / F32
+    assert qkv(a, a, a, cca.CCA_BF16, 4, 2, 64, a, a, a, a, a, vp(0x1002), None) == 1  # scale misaligned
     assert L.cca_kv_append(h, None, vp(0x1000), cca.CCA_BF16, None) == 1
     assert L.cca_kv_append(h, vp(0x1000), vp(0x1000), cca.CCA_E4M3, None) == 1
     # workspace queries and the allocation-free variant: argument errors come first

@@ -144,6 +144,93 @@ def test_quant_e4m3_bit_exact(src_dtype):
     assert np.array_equal(codes.cpu().numpy(), ref_codes)
 
 
+@pytest.mark.parametrize(
+    "n_tok,H,D,src_dtype",
+    [
+        (7, 3, 64, torch.bfloat16),  # fewer tokens than the CTAs of a head's cluster
+        (6400, 2, 128, torch.bfloat16),  # 800 rows of 256 B per CTA: the largest shared-memory staging
+        (6408, 2, 128, torch.bfloat16),  # 801 rows: streamed from global memory twice
+        (3201, 2, 128, torch.float32),  # fp32 rows of 512 B: streamed
+        (3200, 3, 64, torch.float32),
+    ],
+)
+def test_quant_e4m3_staged_and_streamed_sizes(n_tok, H, D, src_dtype):
+    g = np.random.default_rng(n_tok + H)
+    x = g.standard_t(3.0, size=(n_tok, H, D)).astype(np.float32)
+    x[n_tok // 2, H - 1, D - 1] = 900.0  # the absmax sits in one CTA's rows only
+    if src_dtype == torch.bfloat16:
+        x = synth.bf16_round(x)
+    xt = torch.from_numpy(x).to(dev()).to(src_dtype)
+    codes, scale = cca.cca_quant_e4m3(xt)
+    x16, scale16 = cca.cca_quant_e4m3_f16(xt)
+    ref_codes, ref_scale = ofp8.quantize_per_head(x)
+    torch.cuda.synchronize()
+    assert np.array_equal(scale.cpu().numpy(), ref_scale)
+    assert np.array_equal(scale16.cpu().numpy(), ref_scale)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    assert np.array_equal(x16.cpu().numpy(), ofp8.e4m3_decode(ref_codes).astype(np.float16))
+
+
+def _boundary_head(s0, n_tok, D, g):
+    """One head whose quotients x / s sit on and next to every e4m3 rounding
+    boundary (midpoints between neighbouring codes) and every code value, up to
+    4 units in the last place away, both signs; the absmax fixes s."""
+    a = np.float32(448.0 * s0)
+    s = np.float32(a / np.float32(448.0))
+    vals = ofp8.e4m3_decode(np.arange(127, dtype=np.uint8))
+    pts = np.concatenate([(vals[:-1] + vals[1:]) / 2.0, vals])
+    xs = []
+    for m in pts:
+        x = np.float32(m * np.float64(s))
+        for k in range(-4, 5):
+            y = x
+            for _ in range(abs(k)):
+                y = np.nextafter(y, np.float32(np.inf if k > 0 else -np.inf), dtype=np.float32)
+            xs += [y, -y]
+    xs = np.array(xs, dtype=np.float32)
+    xs = xs[np.abs(xs) <= a]
+    head = (g.standard_normal(n_tok * D) * float(s)).astype(np.float32)
+    head = np.clip(head, -a, a)
+    head[: len(xs)] = xs
+    head[len(xs)] = a
+    g.shuffle(head)
+    return head.reshape(n_tok, D)
+
+
+def test_quant_e4m3_quotients_next_to_rounding_boundaries():
+    # A quantiser that multiplies by a rounded reciprocal instead of dividing
+    # disagrees with the fp32 division on about 1 % of these values.
+    g = np.random.default_rng(11)
+    n_tok, D = 48, 128
+    scales = [3.0, 0.7, 1e-3 * np.pi, 12345.678, 1.0 / 3.0, 7.1e-5]
+    x = np.stack([_boundary_head(s0, n_tok, D, g) for s0 in scales], axis=1)  # [n_tok][H][D] fp32
+    xt = torch.from_numpy(x).to(dev())
+    codes, scale = cca.cca_quant_e4m3(xt)
+    x16, _ = cca.cca_quant_e4m3_f16(xt)
+    ref_codes, ref_scale = ofp8.quantize_per_head(x)
+    torch.cuda.synchronize()
+    assert np.array_equal(scale.cpu().numpy(), ref_scale)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    assert np.array_equal(x16.cpu().numpy(), ofp8.e4m3_decode(ref_codes).astype(np.float16))
+
+
+@pytest.mark.parametrize("n_tok,H,D,src_dtype", [(1620, 24, 128, torch.bfloat16), (301, 3, 64, torch.float32)])
+def test_quant_e4m3_qkv_equals_three_quantisations(n_tok, H, D, src_dtype):
+    g = np.random.default_rng(n_tok)
+    xs = [g.standard_t(4.0, size=(n_tok, H, D)).astype(np.float32) * sc for sc in (1.0, 30.0, 1e-3)]
+    xs[1][:, H - 1] = 0.0  # an all-zero head of K -> scale 1
+    if src_dtype == torch.bfloat16:
+        xs = [synth.bf16_round(x) for x in xs]
+    q8, qs, k8, ks, v16, vs = cca.cca_quant_e4m3_qkv(*(torch.from_numpy(x).to(dev()).to(src_dtype) for x in xs))
+    refs = [ofp8.quantize_per_head(x) for x in xs]
+    torch.cuda.synchronize()
+    for (codes, scale), (rc, rs) in zip(((q8, qs), (k8, ks)), refs[:2]):
+        assert np.array_equal(scale.cpu().numpy(), rs)
+        assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(vs.cpu().numpy(), refs[2][1])
+    assert np.array_equal(v16.cpu().numpy(), ofp8.e4m3_decode(refs[2][0]).astype(np.float16))
+
+
 def test_quant_e4m3_f16_widens_the_codes_exactly():
     g = np.random.default_rng(7)
     x = synth.bf16_round(g.standard_t(4.0, size=(777, 5, 128)).astype(np.float32))
