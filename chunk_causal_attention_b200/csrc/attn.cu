@@ -472,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pair = sg.pair, head = sg.head, j0 = sg.j0, j1 = sg.j1;
       const int q_slot = a.prob[sg.prob].q_slot;
       const int n_q = prob_nq(a, sg.prob, n_q0);
+      if (lane == 0) CCA_TRACE_EV(28, it);
       for (int i = 0; i < kNQ && ok; ++i) {
         if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[i], (it - 1) & 1, abort_flag, budget));
         if (!ok) break;
@@ -484,44 +485,32 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_4d(&tm_q, &q_full[i], dstq + b * S::kBox, b * kBoxElems, head, row0, q_slot);
           }
         } else {
-          // Gather: row r of the tile is query q_idx[row0 + r], copied with
-          // cp.async (zero-filled for rows past n_q) into the same 128B-swizzled
-          // layout the TMA would produce.  Lane l first reads the indices of rows
-          // l, l+32, l+64, l+96; every 16-byte copy is then issued back to back.
-          constexpr int kChunks = D * S::kEsz / 16;  // 16-byte chunks per row (8 or 16)
-          constexpr int kRowsPerPass = 32 / kChunks;
-          const uint8_t *qb = static_cast<const uint8_t *>(a.q);
-          int src_row[4];
+          // Gather: row r of the tile is query q_idx[row0 + r], fetched by TMA
+          // row-gather loads (four rows per instruction, one per 128-byte column
+          // box; the map views Q as [q_rows][H*D]) into the layout a tile load
+          // produces.  Lane l takes rows 4l .. 4l+3.  Rows past n_q, and indices
+          // outside [0, q_rows) (flagged), point one row past the tensor, where
+          // the TMA reads zeros.
+          int sr[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int qr = row0 + lane + 32 * k;
-            int sr = qr < n_q ? __ldg(a.q_idx + qr) : -1;
-            if (qr < n_q && (sr < 0 || sr >= a.q_rows)) {
+            const int qr = row0 + 4 * lane + k;
+            int v = qr < n_q ? __ldg(a.q_idx + qr) : a.q_rows;
+            if (qr < n_q && (v < 0 || v >= a.q_rows)) {
               if (a.dev_status) *a.dev_status = CCA_DEV_BAD_INDEX;  // out-of-range index: row read as zeros
-              sr = -1;
+              v = a.q_rows;
             }
-            src_row[k] = sr;
+            sr[k] = v;
           }
-          const int c = lane % kChunks;
-#pragma unroll 4
-          for (int r0 = 0; r0 < kBM; r0 += kRowsPerPass) {
-            const int r = r0 + lane / kChunks;
-            const int k = r >> 5;
-            const int v = k == 0 ? src_row[0] : k == 1 ? src_row[1] : k == 2 ? src_row[2] : src_row[3];
-            const int sr = __shfl_sync(0xffffffffu, v, r & 31);
-            const uint8_t *src = qb + (static_cast<int64_t>(sr < 0 ? 0 : sr) * a.H + head) * D * S::kEsz + c * 16;
-            const uint32_t box = c >> 3, cc = c & 7;
-            const uint32_t dst = dstq + box * S::kBox + r * 128 + ((cc ^ (r & 7)) << 4);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sr < 0 ? 0 : 16)
-                         : "memory");
-          }
-          asm volatile("cp.async.wait_all;" ::: "memory");
-          fence_proxy_async_smem();
+          if (lane == 0) mbar_arrive_expect_tx(&q_full[i], S::kTile);
           __syncwarp();
-          if (lane == 0) mbar_arrive(&q_full[i]);
+          for (uint32_t b = 0; b < S::kNBox; ++b)
+            tma_gather4(&tm_q, &q_full[i], dstq + b * S::kBox + lane * 4 * 128, head * D + b * kBoxElems, sr[0], sr[1],
+                        sr[2], sr[3]);
         }
       }
       if (!ok) break;
+      if (lane == 0) CCA_TRACE_EV(29, it);
       q_armed = it + 1;
       TileCursor cu;
       cursor_begin(a, sg.prob, cu);
@@ -1175,6 +1164,22 @@ static cca_status make_tmap(CUtensorMap *tm, const void *ptr, CUtensorMapDataTyp
   return CCA_OK;
 }
 
+// [rows][H][D] tensor viewed as [rows][H*D] for TMA row gathers: box = 128
+// bytes x one row (the gather4 form), 128-byte swizzle, zeros past the rows.
+static cca_status make_gather_map(CUtensorMap *tm, const void *ptr, CUtensorMapDataType dt, int esize, int D, int H,
+                                  int rows) {
+  auto enc = tmap_encoder();
+  if (!enc) return fail(CCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(H) * D, static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * D * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CCA_ERR_CUDA, "cuTensorMapEncodeTiled (gather) failed (%d)", static_cast<int>(r));
+  return CCA_OK;
+}
+
 static int env_int(const char *name, int dflt) {
   const char *s = std::getenv(name);
   return s && *s ? std::atoi(s) : dflt;
@@ -1263,7 +1268,10 @@ static cca_status launch_attn(AttnLaunch &L, void *workspace, size_t workspace_b
   args.ws_ml = args.ws_o + static_cast<size_t>(2) * grid * (kNQ * kBM) * D;
   CUtensorMap tq, tk[kMaxSrc], tv[kMaxSrc];
   std::memset(&tq, 0, sizeof(tq));
-  if (!args.q_idx) CCA_TRY(make_tmap(&tq, L.q, dt, es, D, H, L.q_rows_map, L.q_slots));
+  if (!args.q_idx)
+    CCA_TRY(make_tmap(&tq, L.q, dt, es, D, H, L.q_rows_map, L.q_slots));
+  else
+    CCA_TRY(make_gather_map(&tq, args.q, dt, es, D, H, args.q_rows));
   for (int s = 0; s < kMaxSrc; ++s) {
     // An unused source reuses source 1's tensor (never read: no segment names it).
     const bool used = args.src_len[s] > 0;

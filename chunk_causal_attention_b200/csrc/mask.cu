@@ -285,8 +285,8 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
   uint8_t(*ring)[kSubTok] = reinterpret_cast<uint8_t(*)[kSubTok]>(seg_dyn);
   __shared__ uint64_t full[kSegStages];
   __shared__ int s_cnt[kMaxSubPerCta];  // counts per sub-tile, then exclusive offsets within the run
-  __shared__ uint16_t s_idx[kSubTok];
-  __shared__ int warp_sum[kSegThreads / 32];
+  __shared__ uint16_t s_idx[kSubTok];                // pass 3: warp w stages its indices in [1024 w, 1024 w + 1024)
+  __shared__ int warp_sum[2][kSegThreads / 32];      // pass 3, by sub-tile parity
   __shared__ unsigned long long s_part[kSegThreads / 32];
   __shared__ int s_total, s_fail;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -397,25 +397,29 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    if (lane == 31) warp_sum[warp] = incl;
-    __syncthreads();  // stage st consumed; the previous sub-tile's s_idx reads are done
+    // The warps' counts by sub-tile parity: a warp writes this buffer again two
+    // sub-tiles later, past a barrier that every other warp reaches only after
+    // reading it here.
+    int *ws = warp_sum[k & 1];
+    if (lane == 31) ws[warp] = incl;
+    __syncthreads();  // stage st consumed by every thread; the warps' counts published
     if (s_fail) break;
     if (threadIdx.x == 0 && issued < n_items) issue();
-    int wofs = 0, stot = 0;
+    int wofs = 0;
 #pragma unroll
-    for (int w = 0; w < kSegThreads / 32; ++w) {
-      const int x = warp_sum[w];
-      wofs += w < warp ? x : 0;
-      stot += x;
-    }
-    int pos = wofs + incl - cnt;
+    for (int w = 0; w < kSegThreads / 32; ++w) wofs += w < warp ? ws[w] : 0;
+    // Each warp stages its own indices and stores them as one contiguous run.
+    uint16_t *mine = s_idx + warp * 1024;
+    int pos = incl - cnt;
     while (bits) {  // set bits only, lowest first
-      s_idx[pos++] = static_cast<uint16_t>(a + __ffs(bits) - 1);
+      mine[pos++] = static_cast<uint16_t>(a + __ffs(bits) - 1);
       bits &= bits - 1;
     }
-    __syncthreads();
-    int32_t *dst = idx + excl + s_cnt[s - sub0];
-    for (int i = threadIdx.x; i < stot; i += kSegThreads) __stcs(dst + i, static_cast<int32_t>(t0 + s_idx[i]));
+    __syncwarp();
+    const int wcnt = __shfl_sync(0xffffffffu, incl, 31);
+    int32_t *dst = idx + excl + s_cnt[s - sub0] + wofs;
+    for (int i = lane; i < wcnt; i += 32) __stcs(dst + i, static_cast<int32_t>(t0 + mine[i]));
+    __syncwarp();  // the next sub-tile's staging overwrites what this loop read
   }
   __syncthreads();
   if (threadIdx.x == 0) {

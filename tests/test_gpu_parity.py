@@ -527,6 +527,29 @@ def test_mask_cached_chunk_end_to_end(c1, c1_ring, c1_ref):
     assert diff <= 1e-2
 
 
+def test_gathered_queries_with_out_of_range_indices(c1, c1_ref):
+    """A query index outside [0, L) sets CCA_DEV_BAD_INDEX and that query
+    reads as zeros (uniform weights: the mean of the visible values); the
+    other queries are unaffected."""
+    ring = cca.KVRing(c1.n_heads, c1.head_dim, c1.chunk_len, c1.window, device=dev())
+    for t in range(c1.t):
+        ring.append(bf(c1.ring_k[t]), bf(c1.ring_v[t]))
+    sel = [5, 1619, 99999, 0, -3, 777]
+    idx = torch.tensor(sel, dtype=torch.int32, device=dev())
+    n = torch.tensor([len(sel)], dtype=torch.int32, device=dev())
+    o = cca.cca_chunk_attn(ring, bf(c1.q[0]), bf(c1.k_cur[0]), bf(c1.v_cur[0]), q_idx=idx, n_q_dev=n, n_q_max=16)
+    torch.cuda.synchronize()
+    assert int(ring.status.item()) == cca.CCA_DEV_BAD_INDEX
+    got = to_np(o)[: len(sel)]
+    good = [i for i, r in enumerate(sel) if 0 <= r < c1.chunk_len]
+    assert_attn_close(got[good], c1_ref[0][[sel[i] for i in good]], what="valid rows beside bad indices")
+    zero_q = np.zeros((1, c1.n_heads, c1.head_dim), dtype=np.float32)
+    ref0 = oca.chunk_attention(zero_q, c1.ring_k, c1.ring_v, c1.t, c1.window, k_cur=c1.k_cur[0], v_cur=c1.v_cur[0])
+    for i, r in enumerate(sel):
+        if not 0 <= r < c1.chunk_len:
+            assert_attn_close(got[i:i + 1], ref0, what=f"bad index {r} reads as a zero query")
+
+
 @pytest.mark.parametrize("ctas", ["auto", "37"])
 def test_fused_scatter_equals_attention_then_scatter(c1, c1_ring, monkeypatch, ctas):
     """cca_chunk_attn_scatter writes every active query's row straight into the
