@@ -257,7 +257,9 @@ def run_reference(args, rank, world):
             "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": L, "kv_len": LK,
                        "parallelism": "replicas"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": "each step: 128 queries x 1 head of the 720p call over 8100 keys, fp64"},
+                             "sample": "each step: 128 queries x 1 head of the 720p call over 8100 keys, fp64 (small "
+                                       "products: below the whole-call BLAS throughput of the main line's "
+                                       "cpu_baseline)"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
