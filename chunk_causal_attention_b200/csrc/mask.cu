@@ -11,6 +11,7 @@
 // found by a 4 x 8-bit radix select on their bit patterns (for non-negative
 // floats the unsigned order of the bits is the numeric order).
 #include <cmath>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -220,7 +221,11 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(const uint8_t 
 constexpr int kSegThreads = 256;
 constexpr int kSubTok = kSegThreads * 32;  // 8192 tokens per sub-tile: 32 per thread
 constexpr int kSegStages = 4;
-constexpr int kSegDynSmem = kSegStages * kSubTok;
+constexpr int kBitsSub = 16;  // sub-tiles whose activity bits a CTA can keep (1 KB each)
+// dynamic shared memory: the mask ring, then 16 KB that hold either the run's
+// activity bits (runs of <= kBitsSub sub-tiles) or the index staging
+constexpr int kSegDynSmem = kSegStages * kSubTok + kBitsSub * kSegThreads * 4;
+static_assert(kBitsSub * kSegThreads * 4 == kSubTok * 2, "the bits area doubles as the uint16 index staging");
 constexpr int kMaxSubPerCta = 1024;
 constexpr int kMaxSegCtas = 4096;
 constexpr long long kSegBudget = 2000000000LL;  // clock64 cycles per wait, about 1 s
@@ -281,11 +286,11 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
                                                                                int32_t *n_active,
                                                                                unsigned long long *status,
                                                                                int n_sub) {
-  extern __shared__ __align__(128) uint8_t seg_dyn[];  // kSegStages x kSubTok bytes
-  uint8_t(*ring)[kSubTok] = reinterpret_cast<uint8_t(*)[kSubTok]>(seg_dyn);
+  extern __shared__ __align__(128) uint8_t seg_dyn[];
+  uint8_t(*ring)[kSubTok] = reinterpret_cast<uint8_t(*)[kSubTok]>(seg_dyn);  // kSegStages x kSubTok bytes
+  uint8_t *ext = seg_dyn + kSegStages * kSubTok;                            // 16 KB
   __shared__ uint64_t full[kSegStages];
   __shared__ int s_cnt[kMaxSubPerCta];  // counts per sub-tile, then exclusive offsets within the run
-  __shared__ uint16_t s_idx[kSubTok];                // pass 3: warp w stages its indices in [1024 w, 1024 w + 1024)
   __shared__ int warp_sum[2][kSegThreads / 32];      // pass 3, by sub-tile parity
   __shared__ unsigned long long s_part[kSegThreads / 32];
   __shared__ int s_total, s_fail;
@@ -294,6 +299,13 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
   const int sub0 = static_cast<int>(static_cast<int64_t>(n_sub) * c / G);
   const int sub1 = static_cast<int>(static_cast<int64_t>(n_sub) * (c + 1) / G);
   const int n_mine = sub1 - sub0, n_items = 2 * n_mine;
+  // A short run keeps each thread's 32 activity bits per sub-tile from pass 1
+  // (in ext), so pass 3 neither re-reads nor re-decodes the mask and stages its
+  // indices in the then idle ring; a long run re-reads the mask in pass 3.
+  const bool keep_bits = n_mine <= kBitsSub;
+  uint32_t *s_bits = reinterpret_cast<uint32_t *>(ext);                       // [sub-tile][thread]
+  uint16_t *s_idx = keep_bits ? reinterpret_cast<uint16_t *>(seg_dyn) : reinterpret_cast<uint16_t *>(ext);
+  const int n_loads = keep_bits ? n_mine : n_items;  // items whose mask bytes come through the ring
   // item k: pass 1 reads sub-tile sub0 + k, pass 3 reads sub1 - 1 - (k - n_mine)
   auto item_sub = [&](int k) { return k < n_mine ? sub0 + k : sub1 - 1 - (k - n_mine); };
   auto item_len = [&](int k) {
@@ -313,7 +325,7 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
     s_fail = 0;
     for (int st = 0; st < kSegStages; ++st) sm100::mbar_init(&full[st], 1);
     sm100::fence_mbar_init();
-    while (issued < n_items && issued < kSegStages) issue();
+    while (issued < n_loads && issued < kSegStages) issue();
   }
   __syncthreads();
   const int a = 32 * threadIdx.x;  // this thread's 32 tokens within a sub-tile
@@ -326,14 +338,22 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
     uint32_t w[8];
     seg_words(ring[st], mask, t0, a, item_len(k) & ~15, n_tok, w);
     int cnt = 0;  // bytes are 0 / 1 here: a byte dot product counts them
+    if (keep_bits) {
+      uint32_t bits = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) cnt = static_cast<int>(__dp4a(w[i], 0x01010101u, static_cast<unsigned>(cnt)));
+      for (int i = 0; i < 8; ++i) bits |= gather4(w[i]) << (4 * i);
+      s_bits[k * kSegThreads + threadIdx.x] = bits;
+      cnt = __popc(bits);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cnt = static_cast<int>(__dp4a(w[i], 0x01010101u, static_cast<unsigned>(cnt)));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     if (lane == 0) atomicAdd(&s_cnt[k], cnt);
     __syncthreads();  // stage st consumed by every thread; s_fail is uniform until the next wait
     if (s_fail) break;
-    if (threadIdx.x == 0 && issued < n_items) issue();
+    if (threadIdx.x == 0 && issued < n_loads) issue();
   }
   if (warp == 0) {  // exclusive scan of the run's counts, 32 at a time
     int carry = 0;
@@ -381,15 +401,19 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
   // 3. indices, last sub-tile first
   if (s_fail) k = n_items;  // uniform: read after the barrier above
   for (; k < n_items; ++k) {
-    const int st = k % kSegStages;
-    sm100::mbar_wait(&full[st], static_cast<uint32_t>((k / kSegStages) & 1), &s_fail, kSegBudget);
     const int s = item_sub(k);
     const int64_t t0 = static_cast<int64_t>(s) * kSubTok;
-    uint32_t w[8];
-    seg_words(ring[st], mask, t0, a, item_len(k) & ~15, n_tok, w);
     uint32_t bits = 0;
+    if (keep_bits) {
+      bits = s_bits[(s - sub0) * kSegThreads + threadIdx.x];
+    } else {
+      const int st = k % kSegStages;
+      sm100::mbar_wait(&full[st], static_cast<uint32_t>((k / kSegStages) & 1), &s_fail, kSegBudget);
+      uint32_t w[8];
+      seg_words(ring[st], mask, t0, a, item_len(k) & ~15, n_tok, w);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) bits |= gather4(w[i]) << (4 * i);
+      for (int i = 0; i < 8; ++i) bits |= gather4(w[i]) << (4 * i);
+    }
     const int cnt = __popc(bits);
     int incl = cnt;
 #pragma unroll
@@ -404,7 +428,7 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
     if (lane == 31) ws[warp] = incl;
     __syncthreads();  // stage st consumed by every thread; the warps' counts published
     if (s_fail) break;
-    if (threadIdx.x == 0 && issued < n_items) issue();
+    if (threadIdx.x == 0 && issued < n_loads) issue();
     int wofs = 0;
 #pragma unroll
     for (int w = 0; w < kSegThreads / 32; ++w) wofs += w < warp ? ws[w] : 0;
@@ -566,6 +590,11 @@ cca_status cca_compact(const uint8_t *mask, int32_t n_tok, int32_t *idx, int32_t
   int G = seg_max_ctas();
   if (G <= 0) return fail(CCA_ERR_CUDA, "cca_compact: occupancy query failed");
   if (G > kMaxSegCtas) G = kMaxSegCtas;
+  // CCA_COMPACT_CTAS caps the grid (tests use it to give each CTA long runs)
+  if (const char *e = std::getenv("CCA_COMPACT_CTAS")) {
+    const int cap = std::atoi(e);
+    if (cap > 0 && cap < G) G = cap;
+  }
   if (G > n_sub) G = n_sub;
   if ((n_sub + G - 1) / G > kMaxSubPerCta)
     return fail(CCA_ERR_INVALID_ARG, "cca_compact: %d tokens exceed %d per CTA", n_tok, kMaxSubPerCta * kSubTok);

@@ -372,6 +372,23 @@ def test_compaction_ragged_sizes(n_tok, p):
     assert torch.equal(idx2[:n2.item()], idx[:n.item()]) and torch.equal(idx3[:n3.item()], idx[:n.item()])
 
 
+@pytest.mark.parametrize("ctas", ["2", "8", "64"])
+def test_compaction_long_and_short_runs(ctas, monkeypatch):
+    """Few CTAs give each a long run of 8192-token sub-tiles: up to 16 sub-tiles
+    a CTA keeps its activity bits between the passes, beyond that it reads the
+    mask again in the second pass.  (2^20 + 77 tokens: runs of 65, 17 and 3.)"""
+    monkeypatch.setenv("CCA_COMPACT_CTAS", ctas)
+    n_tok = (1 << 20) + 77
+    g = np.random.default_rng(int(ctas))
+    m = (g.random(n_tok) < 0.37).astype(np.uint8)
+    m[-77:] = 1  # an active ragged tail
+    idx, n = cca.cca_compact(torch.from_numpy(m).to(dev()))
+    torch.cuda.synchronize()
+    want = np.flatnonzero(m).astype(np.int32)
+    assert n.item() == want.shape[0]
+    assert np.array_equal(idx[:n.item()].cpu().numpy(), want)
+
+
 @pytest.mark.parametrize("n_tok", [1000, 16385, 300007])
 def test_compaction_counts_any_nonzero_byte(n_tok):
     """A token is active when its mask byte is nonzero, whatever the value."""
