@@ -964,9 +964,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // whose KV range meets the item.  The schedule is recomputed exactly as the
 // attention kernel (launched with G CTAs) computed it; items that fell whole
 // inside one CTA's range were written by that CTA and are skipped.  Lane i
-// examines candidate CTA c_first + i; the O rows of up to 8 found pieces are
+// examines candidate CTA c_first + i; the O rows of up to 4 found pieces are
 // then loaded by the whole warp at once (lane = D/32 columns) before they are
-// summed, so a row costs about two memory round trips.  Launched as a
+// summed, so a row costs about two memory round trips when it has at most 4
+// pieces.  (4 rather than 8 at once: 64 instead of 73 registers, so 4 blocks
+// per SM instead of 3; the 486-query call's combine is latency-bound.)  Launched as a
 // programmatic dependent of the attention kernel: it is resident before the
 // attention grid ends and waits (griddepcontrol.wait) for that grid's memory
 // before reading.
@@ -986,7 +988,7 @@ __device__ __forceinline__ int64_t rem_offset(const AttnArgs &a, int n_q0, const
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ AttnArgs a, int G) {
   constexpr int kV = D / 32;  // columns per lane
-  constexpr int kBatch = 8;   // pieces loaded at once
+  constexpr int kBatch = 4;   // pieces loaded at once
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n_q0 = a.n_q_dev ? min(max(*a.n_q_dev, 0), a.prob[0].n_q) : a.prob[0].n_q;
   const Sched sch = make_sched(a, n_q0, G);
