@@ -85,6 +85,7 @@ class NvmlClockSampler:
         self.h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
         self.period = period_s
         self.rows = []
+        self.times = []  # time.perf_counter() of each row
         self.stop_flag = False
 
     def _run(self):
@@ -95,6 +96,7 @@ class NvmlClockSampler:
                 mx = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
                 rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
                 self.rows.append((float(mhz), float(mx), int(rs)))
+                self.times.append(time.perf_counter())
             except Exception:
                 pass
             time.sleep(self.period)
@@ -383,21 +385,43 @@ def extra_workloads(dev, stream, peak_tf, peak_gbs):
             xk = 0.9 * xk + 0.44 * torch.randn((L, H, D), generator=gen, device=dev)
             xv = 0.9 * xv + 0.44 * torch.randn((L, H, D), generator=gen, device=dev)
         torch.cuda.synchronize()
-        return np.array([a.elapsed_time(b) for a, b in lat])
+        t_end = time.perf_counter()
+        lat_ms = np.array([a.elapsed_time(b) for a, b in lat])
+        start_ms = np.array([lat[0][0].elapsed_time(a) for a, _ in lat])  # chunk starts on the GPU's timeline
+        span_ms = lat[0][0].elapsed_time(lat[-1][1])
+        return lat_ms, start_ms, span_ms, t_end
+
+    def window_mhz(smp, t_end, span_ms, lo_ms, hi_ms):
+        """Median SM clock of the samples taken while the GPU ran [lo_ms, hi_ms)
+        of a pass (the pass ended at host time t_end, span_ms after it began)."""
+        if smp is None:
+            return None
+        t0 = t_end - span_ms * 1e-3
+        sel = [r[0] for r, t in zip(smp.rows, smp.times) if lo_ms <= (t - t0) * 1e3 < hi_ms]
+        return float(np.median(sel)) if sel else None
     # A first pass from an idle GPU drifted +6-8 % while the clock settled under the power cap
     # (later passes: within 1 %); it is run as warm-up and not counted.  Each counted pass records
     # the SM clock (NVML) while it runs.
     stream_pass(1)
     pass_clocks = []
     runs = []
+    drift_norm = []  # per pass: (time x SM clock) of chunks 200-224 against chunks 5-29
     for k in range(3):
         try:
-            smp = NvmlClockSampler(dev.index if dev.index is not None else 0, period_s=0.005)
+            smp = NvmlClockSampler(dev.index if dev.index is not None else 0, period_s=0.002)
             smp.start()
         except Exception:
             smp = None
-        runs.append(stream_pass(2 + k))
+        lat_ms, start_ms, span_ms, t_end = stream_pass(2 + k)
+        runs.append(lat_ms)
         pass_clocks.append(smp.stop() if smp else None)
+        f_early = window_mhz(smp, t_end, span_ms, start_ms[5], start_ms[30])
+        f_late = window_mhz(smp, t_end, span_ms, start_ms[200], start_ms[224] + lat_ms[224])
+        if f_early and f_late:
+            e, l_ = float(np.median(lat_ms[5:30])) * f_early, float(np.median(lat_ms[200:225])) * f_late
+            drift_norm.append({"pct": (l_ - e) / e * 100.0, "sm_mhz_5_29": f_early, "sm_mhz_200_224": f_late})
+        else:
+            drift_norm.append(None)
     passes = np.stack(runs)
     ms = np.median(passes, axis=0)
     early, late = float(np.median(ms[5:30])), float(np.median(ms[200:225]))
@@ -407,7 +431,12 @@ def extra_workloads(dev, stream, peak_tf, peak_gbs):
                               "drift_pct": (late - early) / early * 100.0, "drift_pct_each_pass": drift_each,
                               "ols_slope_ms_per_chunk": slope, "first_chunks_ms": [float(x) for x in ms[:5]],
                               "passes": 3, "warmup_passes": 1,
-                              "sm_mhz_each_pass": [c.get("sm_mhz") if c else None for c in pass_clocks]}
+                              "sm_mhz_each_pass": [c.get("sm_mhz") if c else None for c in pass_clocks],
+                              "drift_pct_clock_normalised_each_pass": drift_norm,
+                              "drift_pct_clock_normalised": (float(np.median([d["pct"] for d in drift_norm if d]))
+                                                             if any(drift_norm) else None),
+                              "note": "clock-normalised: per pass, median ms x median SM MHz (NVML every 2 ms) "
+                                      "of chunks 200-224 against chunks 5-29"}
 
     # ---- memory-bound kernels (bandwidth, L2 flushed before each rep)
     def bw(fn, nbytes, reps=20):
@@ -833,6 +862,7 @@ def row_summary(line, ex):
         "a6_active_486_attn_us": g("mask_cached_720p", "attn_us"),
         "a7_scatter_sweep_2^18_frac_hbm": g("sweep_scatter_log2_active_rows", 18, "frac_of_hbm"),
         "c2_drift_pct": g("long_stream_225", "drift_pct"),
+        "c2_drift_pct_clock_normalised": g("long_stream_225", "drift_pct_clock_normalised"),
         "f1_groups_us": g("groups_720p", "us"), "f1_groups_frac": g("groups_720p", "frac_of_bf16_peak"),
         "f2_rope_qk_frac_hbm": g("rope_qk_720p", "frac_of_hbm"),
         "f2_append_rope_frac_hbm": g("append_rope_720p", "frac_of_hbm"),
