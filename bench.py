@@ -402,7 +402,7 @@ def extra_workloads(dev, stream, peak_tf, peak_gbs):
     # A first pass from an idle GPU drifted +6-8 % while the clock settled under the power cap
     # (later passes: within 1 %); it is run as warm-up and not counted.  Each counted pass records
     # the SM clock (NVML) while it runs.
-    stream_pass(1)
+    warm_lat = stream_pass(1)[0]
     pass_clocks = []
     runs = []
     drift_norm = []  # per pass: (time x SM clock) of chunks 200-224 against chunks 5-29
@@ -433,6 +433,11 @@ def extra_workloads(dev, stream, peak_tf, peak_gbs):
                               "passes": 3, "warmup_passes": 1,
                               "sm_mhz_each_pass": [c.get("sm_mhz") if c else None for c in pass_clocks],
                               "drift_pct_clock_normalised_each_pass": drift_norm,
+                              # late chunks of a pass against the early chunks of the pass that follows it
+                              # (seconds apart, so both run in the same power and clock state of the GPU)
+                              "drift_pct_adjacent_passes": [
+                                  float((np.median(prev[200:225]) - np.median(nxt[5:30])) / np.median(nxt[5:30])
+                                        * 100) for prev, nxt in zip([warm_lat] + runs[:-1], runs)],
                               "drift_pct_clock_normalised": (float(np.median([d["pct"] for d in drift_norm if d]))
                                                              if any(drift_norm) else None),
                               "note": "clock-normalised: per pass, median ms x median SM MHz (NVML every 2 ms) "
@@ -863,6 +868,8 @@ def row_summary(line, ex):
         "a7_scatter_sweep_2^18_frac_hbm": g("sweep_scatter_log2_active_rows", 18, "frac_of_hbm"),
         "c2_drift_pct": g("long_stream_225", "drift_pct"),
         "c2_drift_pct_clock_normalised": g("long_stream_225", "drift_pct_clock_normalised"),
+        "c2_drift_pct_adjacent_passes_median": (float(np.median(ex["long_stream_225"]["drift_pct_adjacent_passes"]))
+                                                 if "long_stream_225" in ex else None),
         "f1_groups_us": g("groups_720p", "us"), "f1_groups_frac": g("groups_720p", "frac_of_bf16_peak"),
         "f2_rope_qk_frac_hbm": g("rope_qk_720p", "frac_of_hbm"),
         "f2_append_rope_frac_hbm": g("append_rope_720p", "frac_of_hbm"),
