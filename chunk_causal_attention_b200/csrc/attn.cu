@@ -160,8 +160,9 @@ struct AttnSmem {
   static constexpr uint32_t kK = kQ + kNQ * kTile;
   static constexpr uint32_t kV = kK + kNSK * kTile;
   static constexpr uint32_t kBar = kV + kNSV * kVTile;
-  static constexpr uint32_t kNumBars = 4 + 2 * kNSK + 2 * kNSV + 8 + 1 + 2;
-  static constexpr uint32_t kBytes = kBar + kNumBars * 8 + 16;
+  static constexpr uint32_t kNumBars = 4 + 2 * kNSK + 2 * kNSV + 8 + 1 + 2 + 1;
+  static constexpr uint32_t kXchg = kBar + kNumBars * 8 + 16;  // [2][128] fp32: (m, l) of warpgroup 1's rows
+  static constexpr uint32_t kBytes = kXchg + 2 * 128 * 4;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
@@ -375,7 +376,12 @@ __device__ __forceinline__ float seg_scale(const float *const *tab, int src, int
   return __ldg(tab[src] + slot * H + head);
 }
 
-template <int D, bool kFp8>
+// kSplit: items with one Q tile and two KV tiles or more are split between the
+// softmax warpgroups along their KV tiles.  Built only for calls whose queries
+// are contiguous rows: a call with gathered queries fills its Q tiles (a few
+// hundred rows over the chunk's KV tiles), and the split branch's code in the
+// MMA warp alone costs it time.
+template <int D, bool kFp8, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k0,
                 const __grid_constant__ CUtensorMap tm_v0, const __grid_constant__ CUtensorMap tm_k1,
@@ -402,7 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *o_empty = o_full + 2;       // [2] softmax -> MMA: O read out
   uint64_t *p_half = o_empty + 2;       // [2] softmax -> MMA: first half of P ready (and O rescaled)
   uint64_t *drain = p_half + 2;         // [1] teardown: all MMAs complete
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *split_done = drain + 1;     // [1] softmax 1 -> softmax 0: (m, l) of a split item's rows written
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(split_done + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -433,6 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_empty[s], 1);  // released by the MMA
     }
     mbar_init(drain, 1);
+    mbar_init(split_done, kBM / 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -563,8 +571,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kVStageBytes = S::kVTile;
     uint64_t *pv_full = v_full;
     uint64_t *pv_empty = v_empty;
-    auto issue_qk = [=](int i, uint32_t stage) {
-      const uint64_t qa = dQ0 + ((i * S::kTile) >> 4), kb = dK0 + ((stage * S::kTile) >> 4);
+    // S_i = Q tile qt x K(stage)
+    auto issue_qk = [=](int i, uint32_t stage, int qt) {
+      const uint64_t qa = dQ0 + ((qt * S::kTile) >> 4), kb = dK0 + ((stage * S::kTile) >> 4);
       const uint32_t d = tm + i * 128u;
       if (elect_one()) {
 #pragma unroll
@@ -607,8 +616,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       issue_pv(i, stage, acc, kBN / 32, kBN / 16);
       return true;
     };
-    uint32_t g = 0, g1 = 0;  // tiles handled; tiles that had a second Q tile
-    int it = 0, it1 = 0;     // items handled; items that had a second Q tile
+    uint32_t g = 0;           // KV tiles handled (their K and V stages)
+    uint32_t g0 = 0, g1 = 0;  // tiles of softmax warpgroup 0 / 1 (phases of their S and P barriers)
+    int it = 0, it1 = 0;      // items with an O of warpgroup 0 / 1 (phases of their O barriers)
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
@@ -623,12 +633,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ok && wait(&k_full[g % kNSK], (g / kNSK) & 1);
       if (!ok) break;
       tc_fence_after();
-      for (int jj = 0; jj < n && ok; ++jj, ++g) {
+      if (kSplit && !two && n >= 2) {
+        // An item whose second Q tile is empty: both warpgroups work on its one
+        // Q tile, warpgroup w on the item's tiles jj = w, w + 2, ... with its
+        // own S, P, O and running maximum and sum; the softmax of warpgroup 0
+        // merges the two halves at the end.  Per tile: QK of this tile, then the
+        // PV of the previous tile (the other warpgroup's), so a warpgroup's
+        // PV(jj) and QK(jj + 2) reach the tensor core back to back.
+        uint32_t pc0 = g0, pc1 = g1;  // tiles each warpgroup has had before
+        bool fresh0 = true, fresh1 = true;  // no PV into this item's O_w yet
+        auto pv_of = [&](int u, uint32_t gt) -> bool {  // O_u += P_u V(gt)
+          const uint32_t vst = gt % kNSV, vph = (gt / kNSV) & 1;
+          if (!wait(&pv_full[vst], vph)) return false;
+          const int prev = u == 0 ? it : it1;
+          const bool fresh = u == 0 ? fresh0 : fresh1;
+          const uint32_t pc = u == 0 ? pc0 : pc1;
+          if (fresh && prev > 0 && !wait(&o_empty[u], (prev - 1) & 1)) return false;
+          if (!pv_in_halves(u, vst, !fresh, pc & 1)) return false;
+          commit(&pv_empty[vst]);
+          if (u == 0) {
+            fresh0 = false;
+            ++pc0;
+          } else {
+            fresh1 = false;
+            ++pc1;
+          }
+          return true;
+        };
+        for (int jj = 0; jj < n && ok; ++jj, ++g) {
+          const int w = jj & 1;
+          const uint32_t stage = g % kNSK;
+          tc_fence_after();
+          issue_qk(w, stage, 0);
+          commit(&s_full[w]);
+          commit(&k_empty[stage]);
+          if (jj == n - 1) {
+            commit(&q_empty[0]);
+            commit(&q_empty[1]);
+          }
+          if (jj > 0 && !(ok = pv_of(w ^ 1, g - 1))) break;
+          if (jj < n - 1 && !(ok = wait(&k_full[(g + 1) % kNSK], ((g + 1) / kNSK) & 1))) break;
+        }
+        if (!ok || !(ok = pv_of((n - 1) & 1, g - 1))) break;
+        commit(&o_full[0]);
+        commit(&o_full[1]);
+        g0 = pc0;
+        g1 = pc1;
+        ++it;
+        ++it1;
+        continue;
+      }
+      for (int jj = 0; jj < n && ok; ++jj, ++g, ++g0) {
         const uint32_t stage = g % kNSK;
         const uint32_t vst = g % kNSV, vph = (g / kNSV) & 1;
         if (lane == 0) CCA_TRACE_EV(1, g);
         tc_fence_after();
-        issue_qk(0, stage);
+        issue_qk(0, stage, 0);
         commit(&s_full[0]);
         if (lane == 0) CCA_TRACE_EV(2, g);
         if (two && jj > 0) {  // O1 += P1 V for the previous tile
@@ -639,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           commit(&pv_empty[pst]);
         }
         if (two) {
-          issue_qk(1, stage);
+          issue_qk(1, stage, 1);
           commit(&s_full[1]);
         }
         commit(&k_empty[stage]);
@@ -654,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait(&pv_full[vst], vph))) break;
         if (lane == 0) CCA_TRACE_EV(8, g);
         if (jj == 0 && it > 0 && !(ok = wait(&o_empty[0], (it - 1) & 1))) break;
-        if (!(ok = pv_in_halves(0, vst, jj > 0, g & 1))) break;
+        if (!(ok = pv_in_halves(0, vst, jj > 0, g0 & 1))) break;
         if (!two) commit(&pv_empty[vst]);  // no PV1 will read this V stage
         if (lane == 0) CCA_TRACE_EV(5, g);
         if (lane == 0) CCA_TRACE_EV(6, g);
@@ -724,14 +784,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_off + wg * 128u;
     const uint32_t tO = tmem + lane_off + 256u + wg * D;
     CCA_TRACE_ROLE(2 + wg);
-    uint32_t g = 0;
-    int it = 0;
+    uint32_t g = 0;  // tiles this warpgroup has had (phases of its S and P barriers)
+    int it = 0;      // items this warpgroup has had (phases of its O barriers)
+    int it1 = 0;     // warpgroup 0: items in which warpgroup 1 had an O (phases of o_full[1])
+    int ns = 0;      // warpgroup 0: split items (phases of split_done)
     bool ok = true;
     for (int kseg = 0; ok; ++kseg) {
       Seg sg;
       if (!get_seg(a, n_q0, sch, gridDim.x, blockIdx.x, kseg, sg)) break;
-      if (wg == 1 && !second_tile(a, n_q0, sg)) continue;  // the item's second Q tile is empty
+      // An item whose second Q tile is empty is split between the warpgroups
+      // along its KV tiles (warpgroup w: tiles j0 + w, j0 + w + 2, ...) when it
+      // has two tiles or more; warpgroup 0 merges the halves at the end.
+      const bool two = second_tile(a, n_q0, sg);
+      const bool split = kSplit && !two && sg.j1 - sg.j0 >= 2;
+      if (wg == 1 && !two && !split) continue;
       const int pair = sg.pair, head = sg.head, j0 = sg.j0, j1 = sg.j1;
+      const int jfirst = j0 + (split ? wg : 0), jstep = split ? 2 : 1;
       const AttnProb &P = a.prob[sg.prob];
       const int n_q = prob_nq(a, sg.prob, n_q0);
       // e4m3: scores carry the factor s_q * s_k(chunk); V's factor s_v(chunk) is
@@ -748,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_ref = -INFINITY, l_sum = 0.f;
       TileCursor cu;
       cursor_begin(a, sg.prob, cu);
-      for (int j = j0; j < j1; ++j, ++g) {
+      for (int j = jfirst; j < j1; j += jstep, ++g) {
         int row0, valid;
         cursor_at(a, sg.prob, cu, j, row0, valid);
         (void)row0;
@@ -831,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Rescale this row of O when the reference maximum moved (O of the
         // previous tile is complete: S of this tile was committed after it);
         // done before the first half of P is released to the PV MMAs.
-        if (j > j0 && __any_sync(0xffffffffu, need)) {
+        if (j > jfirst && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
@@ -893,9 +961,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && (warp & 3) == 0) CCA_TRACE_EV(12 + 10 * wg, g);
       }
       if (!ok) break;
+      float *xm1 = reinterpret_cast<float *>(gbase + S::kXchg), *xl1 = xm1 + 128;
+      if (split && wg == 1) {
+        // hand this half's (m, l) to warpgroup 0, which reads O1 from TMEM and
+        // frees it (o_empty[1]) before this warpgroup takes another item
+        xm1[r] = m_ref;
+        xl1[r] = l_sum;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(split_done);
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_empty[1], it & 1, abort_flag, budget));
+        if (!ok) break;
+        ++it;
+        continue;
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(&o_full[wg], it & 1, abort_flag, budget));
+      // split: both halves' PVs done and warpgroup 1's (m, l) written
+      if (split && ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[1], it1 & 1, abort_flag, budget));
+      if (split && ok) ok = __all_sync(0xffffffffu, mbar_wait(split_done, ns & 1, abort_flag, budget));
       if (!ok) break;
       tc_fence_after();
+      // merge weights of the two halves (1 and 0 when not split)
+      float w0 = 1.f, w1 = 0.f;
+      if (split) {
+        const float m1 = xm1[r], l1 = xl1[r];
+        const float mm = fmaxf(m_ref, m1);
+        w0 = ex2_approx(m_ref - mm);
+        w1 = ex2_approx(m1 - mm);
+        l_sum = w0 * l_sum + w1 * l1;
+        m_ref = mm;
+      }
+      if (split) {
+        // fold warpgroup 1's half (its O in the columns after O0) into O0, so
+        // that the output code below is the same for every item
+        const uint32_t tO1 = tmem + lane_off + 256u + D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32], o1[32];
+          tmem_ld32(tO + c0, o);
+          tmem_ld32(tO1 + c0, o1);
+          tmem_ld_wait32(o);
+          tmem_ld_wait32(o1);
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            o[c] = __float_as_uint(fmaf(w0, __uint_as_float(o[c]), w1 * __uint_as_float(o1[c])));
+          tmem_st32(tO + c0, o);
+        }
+        tmem_st_wait();
+      }
       const int row = pair * (kNQ * kBM) + wg * kBM + r;
       const bool row_ok = row < n_q;
       if (sg.slot < 0) {
@@ -944,8 +1056,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[wg]);
+      if (lane == 0) {
+        mbar_arrive(&o_empty[wg]);
+        if (split) mbar_arrive(&o_empty[1]);  // O1 read as well
+      }
       ++it;
+      if (two || split) ++it1;
+      if (split) ++ns;
     }
   }
 
@@ -1289,13 +1406,18 @@ static cca_status launch_attn(AttnLaunch &L, void *workspace, size_t workspace_b
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lk(g_attr_mu);
     if (dev < 0 || dev >= 64 || !done[dev]) {
-      const cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(S::kAlloc));
-      if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "attention: %s", cudaGetErrorString(e));
+      for (auto fn : {attn_kernel<D, kFp8, true>, attn_kernel<D, kFp8, false>}) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kAlloc));
+        if (e != cudaSuccess) return fail(CCA_ERR_CUDA, "attention: %s", cudaGetErrorString(e));
+      }
       if (dev >= 0 && dev < 64) done[dev] = true;
     }
   }
-  attn_kernel<D, kFp8><<<grid, kThreads, S::kAlloc, st>>>(tq, tk[0], tv[0], tk[1], tv[1], tk[2], tv[2], args);
+  if (args.q_idx)
+    attn_kernel<D, kFp8, false><<<grid, kThreads, S::kAlloc, st>>>(tq, tk[0], tv[0], tk[1], tv[1], tk[2], tv[2], args);
+  else
+    attn_kernel<D, kFp8, true><<<grid, kThreads, S::kAlloc, st>>>(tq, tk[0], tv[0], tk[1], tv[1], tk[2], tv[2], args);
   CCA_TRY(launched("attn_kernel"));
   // The combine kernel runs unless the host knows the schedule splits no item.
   const int mode = host_split_mode(args, grid);
