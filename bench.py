@@ -485,6 +485,17 @@ def extra_workloads(dev, stream, peak_tf, peak_gbs):
     out["append_720p_stream"] = {"us_per_call": t * 1e6, "gbs": chunk_bytes / t / 1e9,
                                  "frac_of_hbm": chunk_bytes / t / 1e9 / peak_gbs, "calls": n_app}
     del srcs
+    # append bandwidth over chunk sizes (the 720p chunk x 1, 4, 16, 64 tokens), L2 flushed before each call
+    sweep_app = {}
+    for mult in (1, 4, 16, 64):
+        n_tok = L * mult
+        rs = cca.KVRing(H, D, n_tok, 1, device=dev)
+        ks_ = torch.randn((n_tok, H, D), device=dev, dtype=torch.bfloat16)
+        vs_ = torch.randn((n_tok, H, D), device=dev, dtype=torch.bfloat16)
+        rs.append(ks_, vs_)  # the sink slot; the timed calls rotate through the window slot
+        sweep_app[n_tok] = bw(lambda: rs.append(ks_, vs_), 4 * n_tok * H * D * 2, reps=10)
+        del rs, ks_, vs_
+    out["sweep_append_chunk_tokens"] = sweep_app
 
     # latency at the 720p mask-cache size (1620 tokens)
     out["mask_dynamic_720p_us"] = float(np.median(_timed(
@@ -524,7 +535,8 @@ def extra_workloads(dev, stream, peak_tf, peak_gbs):
     out["sweep_mask_fixed_log2_tokens"] = sweep_mask
     out["sweep_compact_log2_tokens"] = sweep_comp
     out["sweep_scatter_log2_active_rows"] = sweep_scat
-    out["sweep_note"] = ("bandwidth = algorithmic bytes / event time of one call, L2 flushed before each; mask "
+    out["sweep_note"] = ("bandwidth = algorithmic bytes / event time of one call, L2 flushed before each; append "
+                         "2 x 2 x L x H x D bf16 bytes (K and V read and written); mask "
                          "128 B read + 1 B written per token; compaction 1 B read per token + 4 B written per active "
                          "token (30 % active); scatter 2 x 6144 B per active row + 4 B index")
     return out
@@ -856,6 +868,7 @@ def row_summary(line, ex):
     mhz = (line.get("clocks") or {}).get("sm_mhz")
     r = {
         "a1_append_720p_us": g("append_720p", "us"), "a1_append_stream_frac_hbm": g("append_720p_stream", "frac_of_hbm"),
+        "a1_append_sweep_103680_tok_frac_hbm": g("sweep_append_chunk_tokens", 103680, "frac_of_hbm"),
         "a2_append_e4m3_720p_us": g("append_e4m3_720p", "us"),
         "a3_bf16_call_us": line["attn_us_per_call"], "a3_bf16_frac": line["roofline"]["frac"],
         "a3_bf16_call_us_at_1965mhz": line["attn_us_per_call"] * mhz / 1965.0 if mhz else None,

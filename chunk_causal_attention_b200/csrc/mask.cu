@@ -292,6 +292,7 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
   __shared__ uint64_t full[kSegStages];
   __shared__ int s_cnt[kMaxSubPerCta];  // counts per sub-tile, then exclusive offsets within the run
   __shared__ int warp_sum[2][kSegThreads / 32];      // pass 3, by sub-tile parity
+  __shared__ int s_wcnt[kBitsSub][kSegThreads / 32];  // kept bits: active tokens per (sub-tile, warp)
   __shared__ unsigned long long s_part[kSegThreads / 32];
   __shared__ int s_total, s_fail;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -300,11 +301,13 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
   const int sub1 = static_cast<int>(static_cast<int64_t>(n_sub) * (c + 1) / G);
   const int n_mine = sub1 - sub0, n_items = 2 * n_mine;
   // A short run keeps each thread's 32 activity bits per sub-tile from pass 1
-  // (in ext), so pass 3 neither re-reads nor re-decodes the mask and stages its
-  // indices in the then idle ring; a long run re-reads the mask in pass 3.
+  // (in ext) and each warp's count per sub-tile, so pass 3 neither re-reads nor
+  // re-decodes the mask, needs no block barrier per sub-tile, and stages its
+  // indices as int32 in the then idle ring; a long run re-reads the mask in
+  // pass 3 and stages 16-bit offsets in ext.
   const bool keep_bits = n_mine <= kBitsSub;
-  uint32_t *s_bits = reinterpret_cast<uint32_t *>(ext);                       // [sub-tile][thread]
-  uint16_t *s_idx = keep_bits ? reinterpret_cast<uint16_t *>(seg_dyn) : reinterpret_cast<uint16_t *>(ext);
+  uint32_t *s_bits = reinterpret_cast<uint32_t *>(ext);  // [sub-tile][thread]
+  uint16_t *s_idx = reinterpret_cast<uint16_t *>(ext);
   const int n_loads = keep_bits ? n_mine : n_items;  // items whose mask bytes come through the ring
   // item k: pass 1 reads sub-tile sub0 + k, pass 3 reads sub1 - 1 - (k - n_mine)
   auto item_sub = [&](int k) { return k < n_mine ? sub0 + k : sub1 - 1 - (k - n_mine); };
@@ -350,7 +353,10 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    if (lane == 0) atomicAdd(&s_cnt[k], cnt);
+    if (lane == 0) {
+      atomicAdd(&s_cnt[k], cnt);
+      if (keep_bits) s_wcnt[k][warp] = cnt;
+    }
     __syncthreads();  // stage st consumed by every thread; s_fail is uniform until the next wait
     if (s_fail) break;
     if (threadIdx.x == 0 && issued < n_loads) issue();
@@ -400,6 +406,56 @@ __global__ void __launch_bounds__(kSegThreads, CCA_SEG_MINB) compact_seg_kernel(
   for (int w = 0; w < kSegThreads / 32; ++w) excl += s_part[w];
   // 3. indices, last sub-tile first
   if (s_fail) k = n_items;  // uniform: read after the barrier above
+  if (keep_bits) {
+    // Warps run independently: a warp's offset within a sub-tile is the sum of
+    // the earlier warps' counts from pass 1.  It stages its indices (int32) in
+    // its 4 KB of the ring at the store address's position modulo 16 bytes, so
+    // that the run leaves as 16-byte stores with at most 3 scalar ones per end.
+    int *mine = reinterpret_cast<int *>(seg_dyn) + warp * 1024;
+    for (; k < n_items; ++k) {
+      const int s = item_sub(k), kk = s - sub0;
+      uint32_t bits = s_bits[kk * kSegThreads + threadIdx.x];
+      const int cnt = __popc(bits);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int wcnt = __shfl_sync(0xffffffffu, incl, 31);
+      int wofs = 0;
+#pragma unroll
+      for (int w = 0; w < kSegThreads / 32; ++w) wofs += w < warp ? s_wcnt[kk][w] : 0;
+      int32_t *dst = idx + excl + s_cnt[kk] + wofs;
+      // dst's position in its 16-byte group; when the run would not fit behind
+      // that offset ((almost) every token of the warp active) it goes out as
+      // scalar stores from offset 0
+      const int mis = static_cast<int>((reinterpret_cast<uintptr_t>(dst) >> 2) & 3u);
+      const bool vec = mis + wcnt <= 1024;
+      const int off = vec ? mis : 0;
+      int pos = off + incl - cnt;
+      const int tb = static_cast<int>(static_cast<int64_t>(s) * kSubTok) + a - 1;
+      while (bits) {  // set bits only, lowest first
+        mine[pos++] = tb + __ffs(bits);
+        bits &= bits - 1;
+      }
+      __syncwarp();
+      const int pend = off + wcnt;
+      const int qa = (off + 3) >> 2, qb = pend >> 2;  // whole 16-byte groups [qa, qb) of the staging
+      if (vec && qa < qb) {
+        for (int q = qa + lane; q < qb; q += 32)
+          __stcs(reinterpret_cast<int4 *>(dst + (4 * q - off)), *reinterpret_cast<const int4 *>(mine + 4 * q));
+        const int nh = 4 * qa - off, nt = pend - 4 * qb;  // 0..3 each
+        if (lane < nh)
+          __stcs(dst + lane, mine[off + lane]);
+        else if (lane >= 4 && lane < 4 + nt)
+          __stcs(dst + (4 * qb - off) + (lane - 4), mine[4 * qb + lane - 4]);
+      } else {
+        for (int i = lane; i < wcnt; i += 32) __stcs(dst + i, mine[off + i]);
+      }
+      __syncwarp();  // the next sub-tile's staging overwrites what this warp read
+    }
+  }
   for (; k < n_items; ++k) {
     const int s = item_sub(k);
     const int64_t t0 = static_cast<int64_t>(s) * kSubTok;
@@ -578,6 +634,8 @@ cca_status cca_compact(const uint8_t *mask, int32_t n_tok, int32_t *idx, int32_t
   if (!n_active_dev || (n_tok > 0 && (!mask || !idx)))
     return fail(CCA_ERR_INVALID_ARG, "cca_compact: NULL argument");
   if (n_tok > 0 && !aligned16(mask)) return fail(CCA_ERR_INVALID_ARG, "cca_compact: mask must be 16-byte aligned");
+  if (n_tok > 0 && (reinterpret_cast<uintptr_t>(idx) & 3u) != 0)
+    return fail(CCA_ERR_INVALID_ARG, "cca_compact: idx must be 4-byte aligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (n_tok <= kCompactSingleMax) {
     compact_kernel<<<1, kCompactThreads, 0, st>>>(mask, n_tok, idx, n_active_dev);

@@ -411,8 +411,8 @@ cca_status cca_token_mask_l2_frames(const float *src, const float *edit, int32_t
                                     float *tau_out, cca_stream_t stream);
 
 /* idx[0 .. n) = ascending positions u with mask[u] != 0; *n_active_dev = n.
- *  mask: device uint8 [n_tok]; idx: device int32 [n_tok] (entries >= n are not
- *  written); n_active_dev: device int32.
+ *  mask: device uint8 [n_tok], 16-byte aligned; idx: device int32 [n_tok],
+ *  4-byte aligned (entries >= n are not written); n_active_dev: device int32.
  *  0 <= n_tok <= 2^30.  n_tok <= 16384: one CTA, workspace may be NULL.
  *  Larger n_tok: one cooperative launch of co-resident CTAs (count, offset of
  *  each CTA's run from the totals of the runs before it, write), which needs

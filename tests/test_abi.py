@@ -132,6 +132,7 @@ def test_call_validation_without_device_work(L):
     assert L.cca_compact(vp(0x1000), -1, vp(0x1000), vp(0x1000), None, 0, None) == 1
     assert L.cca_compact(vp(0x1000), 10, vp(0x1000), None, None, 0, None) == 1
     assert L.cca_compact(vp(0x1000), 100000, vp(0x1000), vp(0x1000), None, 0, None) == 1  # needs a workspace
+    assert L.cca_compact(vp(0x1000), 10, vp(0x1002), vp(0x1000), None, 0, None) == 1  # idx not 4-byte aligned
     sz = ctypes.c_size_t()
     assert L.cca_compact_workspace_size(16384, ctypes.byref(sz)) == 0 and sz.value == 0
     assert L.cca_compact_workspace_size(16385, ctypes.byref(sz)) == 0 and sz.value == 4096 * 8 + 16

@@ -389,6 +389,28 @@ def test_compaction_long_and_short_runs(ctas, monkeypatch):
     assert np.array_equal(idx[:n.item()].cpu().numpy(), want)
 
 
+@pytest.mark.parametrize("shift", [1, 2, 3])
+@pytest.mark.parametrize("p", [0.3, 1.0])
+def test_compaction_index_array_at_any_4_byte_offset(shift, p):
+    """The write pass stores 16-byte groups where the index array allows: an
+    array that starts 4, 8 or 12 bytes past a 16-byte boundary, and warps whose
+    1024 tokens are all active (a run too long to shift onto the boundary),
+    still give exactly the list of active positions, and nothing outside it is
+    written."""
+    n_tok = (1 << 20) + 77
+    g = np.random.default_rng(100 + shift)
+    m = (g.random(n_tok) < p).astype(np.uint8)
+    buf = torch.full((n_tok + 8,), -7, dtype=torch.int32, device=dev())
+    idx = buf[shift:shift + n_tok]
+    _, n = cca.cca_compact(torch.from_numpy(m).to(dev()), idx=idx)
+    torch.cuda.synchronize()
+    want = np.flatnonzero(m).astype(np.int32)
+    got = buf.cpu().numpy()
+    assert n.item() == want.shape[0]
+    assert np.array_equal(got[shift:shift + want.shape[0]], want)
+    assert np.all(got[:shift] == -7) and np.all(got[shift + want.shape[0]:] == -7)
+
+
 @pytest.mark.parametrize("n_tok", [1000, 16385, 300007])
 def test_compaction_counts_any_nonzero_byte(n_tok):
     """A token is active when its mask byte is nonzero, whatever the value."""
