@@ -53,7 +53,12 @@ namespace cca {
 constexpr int kBM = 128;       // query rows per Q tile (TMEM lanes)
 constexpr int kBN = 128;       // key rows per KV tile
 constexpr int kNQ = 2;         // Q tiles per work item
-constexpr int kNSK = 3;        // K pipeline stages
+// K pipeline stages: 3 for bf16 (what its shared memory holds next to two Q
+// tiles and two V stages); the e4m3 K tiles are half the size, so 5.
+#ifndef CCA_NSK_FP8
+#define CCA_NSK_FP8 5
+#endif
+constexpr int kNSK = 3;
 constexpr int kNSV = 2;        // V pipeline stages
 constexpr int kThreads = 384;  // 12 warps
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
@@ -156,6 +161,7 @@ struct AttnSmem {
   static constexpr uint32_t kTile = kBox * kNBox;            // bytes of one loaded Q/K tile
   static constexpr uint32_t kNBoxV = D * 2 / 128;            // boxes per 128-row V tile
   static constexpr uint32_t kVTile = kBox * kNBoxV;          // bytes of one loaded V tile
+  static constexpr int kNSK = kFp8 ? CCA_NSK_FP8 : ::cca::kNSK;  // K pipeline stages
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + kNQ * kTile;
   static constexpr uint32_t kV = kK + kNSK * kTile;
@@ -389,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tm_v2, const __grid_constant__ AttnArgs a) {
   using namespace sm100;
   using S = AttnSmem<D, kFp8>;
+  constexpr int kNSK = S::kNSK;
   static_assert(!kFp8 || D == 128, "e4m3 path is built for head_dim 128");
   constexpr int kBoxElems = 128 / S::kEsz;  // elements of D per TMA box
   extern __shared__ uint8_t smem_raw[];
