@@ -676,6 +676,20 @@ def extra_rows(dev, stream, peak_tf, peak_gbs):
     e8["note"] = ("algorithmic bytes: read bf16 K and V once (each CTA stages its rows in shared memory for the "
                   "absmax and quantise passes), write K's e4m3 codes and V's codes widened to fp16")
     out["append_e4m3_720p"] = e8
+    # the same two kernels over larger token counts (the 720p chunk x 4 and x 16), L2 flushed before each call
+    sw_rope, sw_e8 = {}, {}
+    for mult in (4, 16):
+        n = L * mult
+        qn, kn = rnd(n, H, D), rnd(n, H, D)
+        qno, kno = torch.empty_like(qn), torch.empty_like(kn)
+        posn = pos.repeat((mult,) + (1,) * (pos.dim() - 1))
+        sw_rope[n] = bw(lambda: cca.cca_rope_qk(qn, kn, posn, freq, q_out=qno, k_out=kno), 4 * n * H * D * 2,
+                        reps=10)
+        rn8 = cca.KVRing(H, D, n, 1, dtype="e4m3", device=dev)
+        sw_e8[n] = bw(lambda: rn8.append(qn, kn), 2 * n * H * D * 2 + n * H * D + n * H * D * 2, reps=10)
+        del qn, kn, qno, kno, rn8
+    out["sweep_rope_qk_tokens"] = sw_rope
+    out["sweep_append_e4m3_tokens"] = sw_e8
     return out
 
 
@@ -870,6 +884,7 @@ def row_summary(line, ex):
         "a1_append_720p_us": g("append_720p", "us"), "a1_append_stream_frac_hbm": g("append_720p_stream", "frac_of_hbm"),
         "a1_append_sweep_103680_tok_frac_hbm": g("sweep_append_chunk_tokens", 103680, "frac_of_hbm"),
         "a2_append_e4m3_720p_us": g("append_e4m3_720p", "us"),
+        "a2_append_e4m3_sweep_25920_tok_frac_hbm": g("sweep_append_e4m3_tokens", 25920, "frac_of_hbm"),
         "a3_bf16_call_us": line["attn_us_per_call"], "a3_bf16_frac": line["roofline"]["frac"],
         "a3_bf16_call_us_at_1965mhz": line["attn_us_per_call"] * mhz / 1965.0 if mhz else None,
         "a3_clean_pass_us": g("clean_pass_720p", "us"),
@@ -885,6 +900,7 @@ def row_summary(line, ex):
                                                  if "long_stream_225" in ex else None),
         "f1_groups_us": g("groups_720p", "us"), "f1_groups_frac": g("groups_720p", "frac_of_bf16_peak"),
         "f2_rope_qk_frac_hbm": g("rope_qk_720p", "frac_of_hbm"),
+        "f2_rope_qk_sweep_25920_tok_frac_hbm": g("sweep_rope_qk_tokens", 25920, "frac_of_hbm"),
         "f2_append_rope_frac_hbm": g("append_rope_720p", "frac_of_hbm"),
         "f3_liveedit_ms_per_chunk": g("liveedit_3frame_chunk", "ms_per_chunk"),
         "f3_liveedit_full_call_frac": g("liveedit_3frame_chunk", "full_call_frac_of_bf16_peak"),

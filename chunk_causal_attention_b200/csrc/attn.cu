@@ -1347,8 +1347,10 @@ static size_t workspace_bytes_any(int D) {
 }
 
 // Host copy of the device schedule's decision (make_sched with every
-// problem's n_q): 0 = no item split, 1 = ranges, 2 = aligned pieces.
-static int host_split_mode(const AttnArgs &a, int G) {
+// problem's n_q): 0 = no item split, 1 = ranges, 2 = aligned pieces; *n_split
+// = the items that are split.
+static int host_split_mode(const AttnArgs &a, int G, int *n_split) {
+  *n_split = 0;
   int n = 0;
   int64_t total = 0;
   for (int p = 0; p < a.n_prob; ++p) {
@@ -1370,6 +1372,7 @@ static int host_split_mode(const AttnArgs &a, int G) {
     i0 = i1;
   }
   if (static_cast<int64_t>(nkv_first) * 8 * G <= total) return 0;
+  *n_split = r;
   const int pieces = G / r;
   const int64_t even = (tr + G - 1) / G;
   return pieces >= 2 && (nkv_first + pieces - 1) / pieces <= even + 2 ? 2 : 1;
@@ -1427,9 +1430,12 @@ static cca_status launch_attn(AttnLaunch &L, void *workspace, size_t workspace_b
     attn_kernel<D, kFp8, true><<<grid, kThreads, S::kAlloc, st>>>(tq, tk[0], tv[0], tk[1], tv[1], tk[2], tv[2], args);
   CCA_TRY(launched("attn_kernel"));
   // The combine kernel runs unless the host knows the schedule splits no item.
-  const int mode = host_split_mode(args, grid);
+  int n_split = 0;
+  const int mode = host_split_mode(args, grid, &n_split);
   if (args.n_q_dev != nullptr || mode != 0) {
-    const int64_t warps = static_cast<int64_t>(grid) * (kNQ * kBM);
+    // one warp per row of a split item: every item may be split when the query
+    // count is read on the device, else the host knows how many are
+    const int64_t warps = static_cast<int64_t>(args.n_q_dev != nullptr ? grid : n_split) * (kNQ * kBM);
     int64_t blocks = (warps + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
