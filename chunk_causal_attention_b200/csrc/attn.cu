@@ -823,18 +823,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_ref = -INFINITY, l_sum = 0.f;
       TileCursor cu;
       cursor_begin(a, sg.prob, cu);
+      // e4m3: a tile's scale factors are loaded and derived one tile ahead (on a
+      // second cursor), off the path from S ready to P released.
+      TileCursor cn = cu;
+      float sl2_n = a.scale_log2, pf_n = 1.f, lpf_n = 0.f, ipf_n = 1.f;
+      auto fp8_factors = [&](int jn) {
+        int r0, vv;
+        cursor_at(a, sg.prob, cn, jn, r0, vv);
+        const int src = cursor_src(a, cn), slot = cursor_slot(a, cn);
+        sl2_n = a.scale_log2 * (s_q * seg_scale(a.k_scale, src, slot, a.H, head));
+        // Floored at 2^-100 so that a zero V scale (all values of that chunk
+        // zero) still gives finite exponentials whose sum is the sum of P: their
+        // 16-bit PV operand rounds to zero, which is the chunk's exact share.
+        pf_n = fmaxf(seg_scale(a.v_scale, src, slot, a.H, head) / s_vmax, 0x1p-100f);
+        lpf_n = __log2f(pf_n);
+        ipf_n = 1.f / pf_n;
+      };
+      if constexpr (kFp8)
+        if (jfirst < j1) fp8_factors(jfirst);
       for (int j = jfirst; j < j1; j += jstep, ++g) {
         int row0, valid;
         cursor_at(a, sg.prob, cu, j, row0, valid);
         (void)row0;
-        float sl2 = a.scale_log2, pf = 1.f;
+        float sl2 = a.scale_log2, lpf = 0.f, ipf = 1.f;
         if constexpr (kFp8) {
-          const int src = cursor_src(a, cu), slot = cursor_slot(a, cu);
-          sl2 *= s_q * seg_scale(a.k_scale, src, slot, a.H, head);
-          // Floored at 2^-100 so that a zero V scale (all values of that chunk
-          // zero) still gives finite exponentials whose sum is the sum of P: their
-          // 16-bit PV operand rounds to zero, which is the chunk's exact share.
-          pf = fmaxf(seg_scale(a.v_scale, src, slot, a.H, head) / s_vmax, 0x1p-100f);
+          sl2 = sl2_n;
+          lpf = lpf_n;
+          ipf = ipf_n;
+          if (j + jstep < j1) fp8_factors(j + jstep);
         }
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], g & 1, abort_flag, budget));
         if (!ok) break;
@@ -900,8 +916,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 16-bit pairs stored to TMEM over the first 64 columns of S, 16 at a time.
         // e4m3: the V-scale ratio pf enters as log2(pf) in the exponent, so the
         // exponential is already P * pf (the 16-bit PV operand); its sum is
-        // divided by pf.
-        const float m_off = kFp8 ? m_new - __log2f(pf) : m_new;
+        // multiplied by 1 / pf.
+        const float m_off = kFp8 ? m_new - lpf : m_new;
         const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_off, -m_off);
         // Rescale this row of O when the reference maximum moved (O of the
         // previous tile is complete: S of this tile was committed after it);
@@ -958,7 +974,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float s_lo, s_hi;
         f2_unpack(f2_add(f2_add(sums[0], sums[1]), f2_add(sums[2], sums[3])), s_lo, s_hi);
-        const float tile_sum = kFp8 ? (s_lo + s_hi) / pf : (s_lo + s_hi);
+        const float tile_sum = kFp8 ? (s_lo + s_hi) * ipf : (s_lo + s_hi);
         l_sum = l_sum * alpha + tile_sum;
         m_ref = m_new;
         tmem_st_wait();
