@@ -936,7 +936,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t sums[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          if (q4 == 2) {  // first 64 key columns of P (and the O rescale) are in TMEM
+          // The first 64 key columns of P (and the O rescale) are in TMEM after
+          // two groups: released to the PV MMAs before the third group's
+          // exponentials (e4m3) or after them, ahead of its store, so that the
+          // store wait finds the first two groups' stores done (bf16).
+          if (kFp8 && q4 == 2) {
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -969,6 +973,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               else
                 p16[c] = pack_bf16x2(e0, e1);
             }
+          }
+          if (!kFp8 && q4 == 2) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_half[wg]);
           }
           tmem_st16(tS + q4 * 16, p16);
         }
